@@ -1,0 +1,371 @@
+"""Plain fp64 definitions of every result on the attention hot path.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): the product path never
+imports this module.  All arrays are float64 NumPy; inputs arrive as exact
+float64 copies of bfloat16 values, in RASTER token order
+(token n = (t*H + y)*W + x), shaped [B, heads, N, d].
+
+Readings taken where the pages leave a step open (each one is also listed in
+the design notes):
+  * window start: start = clamp(a - floor(w/2), 0, max(N_tiles - w, 0)),
+    extent = min(w, N_tiles); a clamped window always keeps prod(min(w, N))
+    tiles ("Fast Video Generation with Sliding Tile Attention", abstract,
+    tile-by-tile sliding window; the clamp is the plainest reading that keeps
+    every query tile's window fully inside the grid);
+  * tile order and intra-tile order are both raster, t-major, w fastest;
+  * only K and V are pooled (average over p_t x p_h x p_w token blocks); the
+    queries keep full resolution ("AtlasVid ...", abstract, asymmetric
+    global-local attention; "UltraGen ..." §4.2, compressed global modelling);
+  * the fusion factor of "UltraGen ..." §4.1 is a given per-head g in [0, 1]:
+    O = g * O_local + (1 - g) * O_global;
+  * LSE is the natural log of the softmax denominator, scale included.
+
+Parity: pinned by invariants, brute force and finite differences in
+tests/test_oracle.py; the pages print no worked numeric example.
+"""
+from __future__ import annotations
+
+import math
+from typing import NamedTuple
+
+import numpy as np
+
+
+class Geom(NamedTuple):
+    """Latent grid (T, H, W), tile, window (in tiles) and pool sizes, (t, h, w) order."""
+    T: int
+    H: int
+    W: int
+    tile: tuple
+    window: tuple
+    pool: tuple = (1, 1, 1)
+
+    @property
+    def n(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def tiles_per_dim(self) -> tuple:
+        return (self.T // self.tile[0], self.H // self.tile[1], self.W // self.tile[2])
+
+    @property
+    def tile_volume(self) -> int:
+        return self.tile[0] * self.tile[1] * self.tile[2]
+
+    @property
+    def pooled_dims(self) -> tuple:
+        return (self.T // self.pool[0], self.H // self.pool[1], self.W // self.pool[2])
+
+    @property
+    def n_pooled(self) -> int:
+        a, b, c = self.pooled_dims
+        return a * b * c
+
+
+def geom_of(workload) -> Geom:
+    T, H, W = workload.grid
+    return Geom(T, H, W, tuple(workload.tile), tuple(workload.window), tuple(workload.pool))
+
+
+# ---------------------------------------------------------------------------
+# a1: raster <-> tile-major reorder ("AtlasVid ...", abstract: reordered
+# spatiotemporal windows; "Fast Video Generation with Sliding Tile Attention",
+# abstract: tile-by-tile operation)
+# ---------------------------------------------------------------------------
+
+def token_coords(g: Geom) -> np.ndarray:
+    """[N, 3] (t, y, x) of every raster token."""
+    n = np.arange(g.n)
+    x = n % g.W
+    y = (n // g.W) % g.H
+    t = n // (g.W * g.H)
+    return np.stack([t, y, x], axis=1)
+
+
+def tile_major_index(g: Geom) -> np.ndarray:
+    """m[n] = tile-major position of raster token n:
+    m = tile_id * s + local_id, tile_id = ((t/t_t)*N_h + y/t_h)*N_w + x/t_w,
+    local_id = ((t%t_t)*t_h + y%t_h)*t_w + x%t_w."""
+    tt, th, tw = g.tile
+    _, nh, nw = g.tiles_per_dim
+    c = token_coords(g)
+    t, y, x = c[:, 0], c[:, 1], c[:, 2]
+    tile_id = ((t // tt) * nh + y // th) * nw + x // tw
+    local = ((t % tt) * th + y % th) * tw + x % tw
+    return tile_id * g.tile_volume + local
+
+
+def permute(x_raster: np.ndarray, g: Geom) -> np.ndarray:
+    """Raster -> tile-major along axis -2 (a pure row gather)."""
+    m = tile_major_index(g)
+    out = np.empty_like(x_raster)
+    out[..., m, :] = x_raster
+    return out
+
+
+def unpermute(x_tiled: np.ndarray, g: Geom) -> np.ndarray:
+    """Tile-major -> raster along axis -2."""
+    m = tile_major_index(g)
+    return x_tiled[..., m, :]
+
+
+# ---------------------------------------------------------------------------
+# a2: kept-tile list ("Fast Video Generation with Sliding Tile Attention",
+# abstract: each query tile attends to a 3D window of tiles around it)
+# ---------------------------------------------------------------------------
+
+def window_range(a: int, w: int, n: int) -> range:
+    """Tiles kept along one dim for query tile coordinate a: the window of
+    min(w, n) tiles centred on a and shifted inward at the grid boundary."""
+    ext = min(w, n)
+    start = min(max(a - w // 2, 0), max(n - w, 0))
+    return range(start, start + ext)
+
+
+def kept_tiles(g: Geom) -> np.ndarray:
+    """[n_tiles, kept] int32: for every query tile (tile-major id order) the ids
+    of its kept key tiles, t outermost, w fastest."""
+    nt, nh, nw = g.tiles_per_dim
+    rows = []
+    for at in range(nt):
+        for ah in range(nh):
+            for aw in range(nw):
+                ids = [(kt * nh + kh) * nw + kw
+                       for kt in window_range(at, g.window[0], nt)
+                       for kh in window_range(ah, g.window[1], nh)
+                       for kw in window_range(aw, g.window[2], nw)]
+                rows.append(ids)
+    return np.asarray(rows, dtype=np.int32)
+
+
+def kept_count_closed_form(g: Geom) -> int:
+    return math.prod(min(w, n) for w, n in zip(g.window, g.tiles_per_dim))
+
+
+def _tile_token_box(g: Geom, lo: tuple, hi: tuple) -> np.ndarray:
+    """Raster ids of all tokens with tile coordinates in [lo, hi) per dim."""
+    tt, th, tw = g.tile
+    ts = np.arange(lo[0] * tt, hi[0] * tt)
+    ys = np.arange(lo[1] * th, hi[1] * th)
+    xs = np.arange(lo[2] * tw, hi[2] * tw)
+    return ((ts[:, None, None] * g.H + ys[None, :, None]) * g.W + xs[None, None, :]).reshape(-1)
+
+
+# ---------------------------------------------------------------------------
+# softmax attention over an explicit key set (the definition of "UltraGen ..."
+# §3: S = q k^T * scale, softmax over keys, O = P V)
+# ---------------------------------------------------------------------------
+
+def _softmax_attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    s = (q @ k.T) * scale
+    mx = s.max(axis=1, keepdims=True)
+    e = np.exp(s - mx)
+    den = e.sum(axis=1, keepdims=True)
+    p = e / den
+    return p @ v, (mx + np.log(den))[:, 0], p
+
+
+def full_attention(q, k, v, scale):
+    """Dense softmax attention over all keys; [B,h,N,d] -> (O, LSE)."""
+    B, nh, n, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, nh, n))
+    for b in range(B):
+        for h in range(nh):
+            o[b, h], lse[b, h], _ = _softmax_attend(q[b, h], k[b, h], v[b, h], scale)
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# a3: sliding-tile (local) attention
+# ---------------------------------------------------------------------------
+
+def _query_tiles(g: Geom):
+    """Yield (query token ids, key token ids) per query tile, both raster."""
+    nt, nh, nw = g.tiles_per_dim
+    for at in range(nt):
+        for ah in range(nh):
+            for aw in range(nw):
+                qi = _tile_token_box(g, (at, ah, aw), (at + 1, ah + 1, aw + 1))
+                rt = window_range(at, g.window[0], nt)
+                rh = window_range(ah, g.window[1], nh)
+                rw = window_range(aw, g.window[2], nw)
+                kj = _tile_token_box(g, (rt.start, rh.start, rw.start), (rt.stop, rh.stop, rw.stop))
+                yield qi, kj
+
+
+def sta_attention(q, k, v, g: Geom, scale: float):
+    """Local branch: every query attends only to the tokens of its query tile's
+    kept tiles.  Raster in, raster out: (O [B,h,N,d], LSE [B,h,N])."""
+    B, nh, n, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, nh, n))
+    for b in range(B):
+        for h in range(nh):
+            for qi, kj in _query_tiles(g):
+                o[b, h, qi], lse[b, h, qi], _ = _softmax_attend(q[b, h, qi], k[b, h, kj], v[b, h, kj], scale)
+    return o, lse
+
+
+def sta_mask_bruteforce(g: Geom) -> np.ndarray:
+    """[N, N] bool, built token by token: key j is visible to query i iff j's
+    tile lies in the clamped window of i's tile along every dim."""
+    c = token_coords(g)
+    tc = c // np.asarray(g.tile)
+    dims = g.tiles_per_dim
+    mask = np.ones((g.n, g.n), dtype=bool)
+    for ax in range(3):
+        w, nd = g.window[ax], dims[ax]
+        start = np.array([window_range(a, w, nd).start for a in range(nd)])
+        ext = min(w, nd)
+        s_i = start[tc[:, ax]][:, None]
+        mask &= (tc[None, :, ax] >= s_i) & (tc[None, :, ax] < s_i + ext)
+    return mask
+
+
+def sta_attention_bruteforce(q, k, v, g: Geom, scale: float):
+    """Local branch as a masked dense softmax (tiny grids only)."""
+    mask = sta_mask_bruteforce(g)
+    B, nh, n, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, nh, n))
+    for b in range(B):
+        for h in range(nh):
+            s = (q[b, h] @ k[b, h].T) * scale
+            s = np.where(mask, s, -np.inf)
+            mx = s.max(axis=1, keepdims=True)
+            e = np.exp(s - mx)
+            den = e.sum(axis=1, keepdims=True)
+            o[b, h] = (e / den) @ v[b, h]
+            lse[b, h] = (mx + np.log(den))[:, 0]
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# a4: K/V average pooling ("UltraGen ..." §4.2: downsample before global
+# attention, fewer spatial tokens; the spec form is average pooling)
+# ---------------------------------------------------------------------------
+
+def pooled_index(g: Geom) -> np.ndarray:
+    """u[n] = pooled-raster id of the block containing raster token n."""
+    pt, ph, pw = g.pool
+    _, PH, PW = g.pooled_dims
+    c = token_coords(g)
+    return ((c[:, 0] // pt) * PH + c[:, 1] // ph) * PW + c[:, 2] // pw
+
+
+def pool(x_raster: np.ndarray, g: Geom) -> np.ndarray:
+    """Exact fp64 mean over every p_t x p_h x p_w block; [..., N, d] -> [..., N_p, d]."""
+    u = pooled_index(g)
+    cnt = g.pool[0] * g.pool[1] * g.pool[2]
+    # group the tokens of each block together (every block has cnt tokens),
+    # then sum each group
+    order = np.argsort(u, kind="stable")
+    d = x_raster.shape[-1]
+    grouped = x_raster[..., order, :].reshape(x_raster.shape[:-2] + (g.n_pooled, cnt, d))
+    return grouped.sum(axis=-2) / cnt
+
+
+def pool_transpose(y_pooled: np.ndarray, g: Geom) -> np.ndarray:
+    """Adjoint of pool: x[n] = y[u(n)] / count."""
+    cnt = g.pool[0] * g.pool[1] * g.pool[2]
+    return y_pooled[..., pooled_index(g), :] / cnt
+
+
+# ---------------------------------------------------------------------------
+# a5/a6: global branch and blend ("UltraGen ..." §4.1, §4.2)
+# ---------------------------------------------------------------------------
+
+def global_attention(q, kp, vp, scale):
+    """Every full-resolution query attends to all pooled keys."""
+    return full_attention(q, kp, vp, scale)
+
+
+def dual_forward(q, k, v, gvec, g: Geom, scale: float):
+    """Returns dict with O, O_l, LSE_l, O_g, LSE_g, K_p, V_p (all raster)."""
+    o_l, lse_l = sta_attention(q, k, v, g, scale)
+    kp, vp = pool(k, g), pool(v, g)
+    o_g, lse_g = global_attention(q, kp, vp, scale)
+    gb = np.asarray(gvec, dtype=np.float64)[None, :, None, None]
+    o = gb * o_l + (1.0 - gb) * o_g
+    return dict(O=o, O_l=o_l, LSE_l=lse_l, O_g=o_g, LSE_g=lse_g, K_p=kp, V_p=vp)
+
+
+# ---------------------------------------------------------------------------
+# a7: backward, restated from the softmax Jacobian (no saved-statistics split)
+# ---------------------------------------------------------------------------
+
+def _softmax_attend_bwd(q, k, v, do, scale):
+    """Gradients of O = softmax(q k^T scale) v w.r.t. q, k, v for upstream do."""
+    _, _, p = _softmax_attend(q, k, v, scale)
+    dv = p.T @ do
+    dp = do @ v.T
+    # dS_ij = sum_l dP_il * dP_il/dS_ij with dP/dS the softmax Jacobian
+    # diag(p) - p p^T per row.
+    ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+    dq = scale * (ds @ k)
+    dk = scale * (ds.T @ q)
+    return dq, dk, dv
+
+
+def sta_backward(q, k, v, do, g: Geom, scale: float):
+    """Local-branch gradients (raster)."""
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    B, nh = q.shape[:2]
+    for b in range(B):
+        for h in range(nh):
+            for qi, kj in _query_tiles(g):
+                a, bk, c = _softmax_attend_bwd(q[b, h, qi], k[b, h, kj], v[b, h, kj], do[b, h, qi], scale)
+                dq[b, h, qi] += a
+                dk[b, h, kj] += bk
+                dv[b, h, kj] += c
+    return dq, dk, dv
+
+
+def global_backward(q, kp, vp, do, scale):
+    """Global-branch gradients w.r.t. q and the pooled k_p, v_p."""
+    dq = np.zeros_like(q)
+    dkp = np.zeros_like(kp)
+    dvp = np.zeros_like(vp)
+    B, nh = q.shape[:2]
+    for b in range(B):
+        for h in range(nh):
+            dq[b, h], dkp[b, h], dvp[b, h] = _softmax_attend_bwd(q[b, h], kp[b, h], vp[b, h], do[b, h], scale)
+    return dq, dkp, dvp
+
+
+def dual_backward(q, k, v, gvec, do, g: Geom, scale: float):
+    """Gradients of the blended output w.r.t. q, k, v (through the pooling) and g.
+
+    O = g O_l + (1-g) O_g  =>  branch upstream gradients g*dO and (1-g)*dO;
+    dK = dK_l + pool^T(dK_p), dV likewise; dg_h = sum_{b,n} dO . (O_l - O_g).
+    """
+    gb = np.asarray(gvec, dtype=np.float64)[None, :, None, None]
+    dq_l, dk_l, dv_l = sta_backward(q, k, v, gb * do, g, scale)
+    kp, vp = pool(k, g), pool(v, g)
+    dq_g, dkp, dvp = global_backward(q, kp, vp, (1.0 - gb) * do, scale)
+    o_l, _ = sta_attention(q, k, v, g, scale)
+    o_g, _ = global_attention(q, kp, vp, scale)
+    dg = (do * (o_l - o_g)).sum(axis=(0, 2, 3))
+    return dict(dQ=dq_l + dq_g, dK=dk_l + pool_transpose(dkp, g), dV=dv_l + pool_transpose(dvp, g),
+                dK_p=dkp, dV_p=dvp, dg=dg, dQ_l=dq_l, dQ_g=dq_g)
+
+
+# ---------------------------------------------------------------------------
+# work accounting ("UltraGen ..." App. B complexity model; effective FLOPs)
+# ---------------------------------------------------------------------------
+
+def kept_pairs_local(g: Geom, batch: int, heads: int) -> int:
+    """Query-key pairs the local branch computes: every query sees kept*s keys."""
+    return batch * heads * g.n * kept_count_closed_form(g) * g.tile_volume
+
+
+def pairs_global(g: Geom, batch: int, heads: int) -> int:
+    return batch * heads * g.n * g.n_pooled
+
+
+def ultragen_cost_ratio(K: int) -> float:
+    """App. B of "UltraGen ...": (5/(4K^2) + 1/K^4) of full attention's cost."""
+    return 5.0 / (4.0 * K * K) + 1.0 / K ** 4
