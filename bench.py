@@ -1,0 +1,455 @@
+"""Benchmark of the dual-branch 3D attention hot path (one JSON line on rank 0).
+
+Default workload: the 720p-shaped sliding-tile forward (B1 h24 d128, grid
+30x48x80, tile 6x8x8, window 3x3x3, per-head U(0.5, 2) scale).  One step =
+raster->tile-major permute of Q, K, V, the sliding-tile forward (O, LSE), and
+the tile-major->raster unpermute of O and LSE, all through the C ABI.
+Effective FLOPs count 4*d per kept query-key pair (masked work is not
+counted).  Inputs (2.1 GB of Q/K/V) are larger than the 126 MB L2, so no flush
+is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--no-extras]
+
+Multi-GPU: one process per GPU (torchrun); each rank runs its own full
+workload (batch/head slices are independent: no collective on the data path),
+so scaling is weak and `value` sums all ranks' work over the max-over-ranks
+time.  `--impl reference` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective TFLOP/s & ms/call of 3D tile+global attention fwd/bwd; % BF16 TC peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# ncu DRAM traffic per launch of the sliding-tile forward kernel at the 720p
+# workload (read+write bytes), and the hash of the kernel source it was taken
+# from.  When the source changes the figure is stale and reported as null.
+STA_FWD_TRAFFIC = None  # bytes per launch, from profiles/sta_fwd_720p.md
+STA_FWD_TRAFFIC_SRC_SHA = None
+
+
+def _src_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "video_dit_local_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev = dev_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.25)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def _geom(V, w):
+    return V.make_geom(w.batch, w.heads, w.head_dim, w.grid, w.tile, w.window, w.pool)
+
+
+def _flops_fwd(w):
+    from synth import inputs as S  # noqa: F401
+    T, H, W = w.grid
+    nt = [a // b for a, b in zip(w.grid, w.tile)]
+    kept = math.prod(min(x, n) for x, n in zip(w.window, nt))
+    s = math.prod(w.tile)
+    n = T * H * W
+    pairs_local = w.batch * w.heads * n * kept * s
+    pairs_global = 0
+    if w.dual:
+        npool = (T // w.pool[0]) * (H // w.pool[1]) * (W // w.pool[2])
+        pairs_global = w.batch * w.heads * n * npool
+    return 4 * w.head_dim * pairs_local, 4 * w.head_dim * pairs_global
+
+
+def _host_inputs_720p(w):
+    """Seeded Q/K/V (bf16 bits, raster) from the shared generator."""
+    import numpy as np
+    from synth import inputs as S
+    out = []
+    for tid in (S.Q_ID, S.K_ID, S.V_ID):
+        out.append(S.draw(w, tid).view(np.int16))
+    return out
+
+
+def _device_randn(shape, seed, std=1.0, scales=None):
+    import torch
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    x = torch.randn(shape, generator=gen, device="cuda", dtype=torch.float32) * std
+    if scales is not None:
+        x *= torch.as_tensor(scales, device="cuda").view(1, -1, 1, 1)
+    return x.to(torch.bfloat16)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import video_dit_local_b200 as V
+    from synth import inputs as S
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = S.WORKLOADS["720p"]
+    geom = _geom(V, w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    flops_local, _ = _flops_fwd(w)
+
+    host = _host_inputs_720p(w)
+    pinned = [torch.from_numpy(h).pin_memory() for h in host]
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    qr, kr, vr = (p.to(dev).view(torch.bfloat16) for p in pinned)
+    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    o = torch.empty_like(q)
+    o_r = torch.empty_like(q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    lse_r = torch.empty_like(lse)
+    stream = torch.cuda.current_stream()
+    kernel_events = []
+
+    def step(record=False):
+        V.vattn_tile_permute(geom, qr, q)
+        V.vattn_tile_permute(geom, kr, k)
+        V.vattn_tile_permute(geom, vr, v)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        V.vattn_sta_fwd(geom, q, k, v, scale, o, lse)
+        if record:
+            e1.record(stream)
+            kernel_events.append((e0, e1))
+        V.vattn_tile_unpermute(geom, o, o_r)
+        V.vattn_tile_unpermute(geom, lse, lse_r, 4)
+
+    launches_per_step = 6
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if V.vattn_get_status() != 0:
+        raise RuntimeError("device status after warm-up: " + V.vattn_last_error())
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(record=True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    ms_kernel = sum(a.elapsed_time(b) for a, b in kernel_events) / len(kernel_events)
+    if V.vattn_get_status() != 0:
+        raise RuntimeError("device status after timing: " + V.vattn_last_error())
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step, ms_kernel], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_step, ms_kernel = t.tolist()
+
+    # end to end through the C ABI from pinned host buffers
+    o_host = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
+    lse_host = torch.empty(shape[:3], dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        for p, dst in zip(pinned, (qr, kr, vr)):
+            dst.view(torch.int16).copy_(p, non_blocking=True)
+        step()
+        o_host.copy_(o_r, non_blocking=True)
+        lse_host.copy_(lse_r, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = a0.elapsed_time(a1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = t.item()
+    h2d = sum(p.numel() * p.element_size() for p in pinned)
+    d2h = o_host.numel() * 2 + lse_host.numel() * 4
+
+    peaks, peak_src = _peaks()
+    achieved = flops_local / (ms_kernel * 1e-3) / 1e12
+    traffic = STA_FWD_TRAFFIC if STA_FWD_TRAFFIC_SRC_SHA == _src_sha() else None
+    result = {
+        "metric": METRIC,
+        "value": round(world * flops_local / (ms_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, per-head U(0.5,2) scale)",
+        "config": {"workload": "720p sliding-tile fwd: B1 h24 d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
+                   "global_batch": w.batch * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (2.1 GB Q/K/V), no flush",
+                   "step": "permute Q,K,V + sta_fwd + unpermute O,LSE"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "peak_source": f"{peak_src} bf16 (burst)", "traffic": traffic,
+                     "kernel": "attn_fwd_kernel<128> (sliding tile)", "kernel_ms": round(ms_kernel, 4),
+                     "algorithmic_flop_per_launch": flops_local},
+        "e2e": {"value": round(world * flops_local / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_extras:
+        result["extras"] = run_extras(V, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return result
+
+
+def run_extras(V, dev):
+    """Other shipped workloads, kernel-timed (not part of `value`)."""
+    import torch
+    from synth import inputs as S
+    out = {}
+    peaks, _ = _peaks()
+    for name in ("1080p", "4k"):
+        w = S.WORKLOADS[name]
+        geom = _geom(V, w)
+        shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+        q, k, v = (_device_randn(shape, 100 * w.seed + i) for i in range(3))
+        gvec = torch.rand(w.heads, device=dev)
+        o = torch.empty_like(q)
+        ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, geom), dtype=torch.uint8, device=dev)
+        scale = 1 / math.sqrt(w.head_dim)
+        fl, fg = _flops_fwd(w)
+
+        def call():
+            V.vattn_dual_fwd(geom, q, k, v, gvec, scale, o, workspace=ws)
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        n = 4
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        out[f"{name}_dual_fwd"] = {"ms": round(ms, 3), "eff_tflops": round((fl + fg) / ms / 1e9, 1),
+                                   "frac": round((fl + fg) / ms / 1e9 / peaks["bf16_tflops"], 4),
+                                   "status": V.vattn_get_status()}
+        del q, k, v, o, ws
+        torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(budget_s: float):
+    """The fp64 oracle, as it stands, on a bounded sample of the 720p workload:
+    one head (b=0, h=0), query tiles taken in a fixed order until the time
+    budget is spent."""
+    import numpy as np
+
+    from oracle import vattn_oracle as O
+    from synth import inputs as S
+    w = S.WORKLOADS["720p"]
+    g = O.geom_of(w)
+    q, k, v = (S.bf16_bits_to_f64(S.draw_head(w, i, 0, 0)) for i in (S.Q_ID, S.K_ID, S.V_ID))
+    scale = 1 / math.sqrt(w.head_dim)
+    kept = O.kept_count_closed_form(g)
+    s = g.tile_volume
+    n_tiles = math.prod(g.tiles_per_dim)
+    order = np.random.default_rng(0).permutation(n_tiles)
+    done = 0
+    t0 = time.perf_counter()
+    while done < n_tiles and time.perf_counter() - t0 < budget_s:
+        O.sta_attention_tiles(q, k, v, g, scale, [int(order[done])])
+        done += 1
+    dt = time.perf_counter() - t0
+    flops = 4 * w.head_dim * done * s * kept * s
+    cores = len(os.sched_getaffinity(0))
+    return {"value": round(flops / dt / 1e12, 5), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"720p STA fwd, head (0,0), {done} of {n_tiles} query tiles ({done * s} queries), "
+                      f"{dt:.1f} s, numpy fp64 BLAS threads={_blas_threads()}"}
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 0) for i in threadpool_info()), default=None)
+    except Exception:
+        return None
+
+
+def run_reference(args):
+    """Reference arm: the fp64 oracle on the host cores, a bounded sample per step."""
+    import numpy as np
+
+    from oracle import vattn_oracle as O
+    from synth import inputs as S
+    w = S.WORKLOADS["720p"]
+    g = O.geom_of(w)
+    q, k, v = (S.bf16_bits_to_f64(S.draw_head(w, i, 0, 0)) for i in (S.Q_ID, S.K_ID, S.V_ID))
+    scale = 1 / math.sqrt(w.head_dim)
+    kept = O.kept_count_closed_form(g)
+    s = g.tile_volume
+    n_tiles = math.prod(g.tiles_per_dim)
+    tiles_per_step = 2
+    order = np.random.default_rng(0).permutation(n_tiles)
+    for i in range(args.warmup):
+        O.sta_attention_tiles(q, k, v, g, scale, [int(t) for t in order[:tiles_per_step]])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        sel = [int(order[(i * tiles_per_step + j) % n_tiles]) for j in range(tiles_per_step)]
+        O.sta_attention_tiles(q, k, v, g, scale, sel)
+    dt = time.perf_counter() - t0
+    flops = 4 * w.head_dim * args.steps * tiles_per_step * s * kept * s
+    value = flops / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"720p STA fwd, head (0,0), {tiles_per_step} query tiles ({tiles_per_step * s} queries) per step, "
+              f"numpy fp64")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) bf16, per-head U(0.5,2) scale)",
+            "config": {"workload": "720p sliding-tile fwd: B1 h24 d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
+                       "sample": sample},
+            "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        result = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

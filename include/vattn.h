@@ -1,0 +1,176 @@
+/*
+ * vattn — dual-branch 3D video attention on B200 (sm_100a).
+ *
+ * Full 3D attention over a video latent token grid T x H x W is split into
+ *   - a local branch: sliding-tile attention.  Every query tile attends only
+ *     to the key tiles inside a 3D window of tiles around it
+ *     ("Fast Video Generation with Sliding Tile Attention", abstract);
+ *   - a global branch: every full-resolution query attends to average-pooled
+ *     keys and values ("UltraGen: High-Resolution Video Generation with
+ *     Hierarchical Attention" §4.2, spatially compressed global attention;
+ *     "AtlasVid ..." abstract, asymmetric global-local attention);
+ * and the two outputs are blended per head, O = g*O_local + (1-g)*O_global
+ * ("UltraGen ..." §4.1, time-aware fusion factor, taken here as a given g).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates device memory on these calls; scratch space is passed in
+ *    as `workspace` (size from vattn_workspace_size).
+ *  - Q/K/V/O/dQ/dK/dV are [batch, heads, N, head_dim] bfloat16, head_dim
+ *    contiguous, N = T*H*W.  Attention calls take TILE-MAJOR token order
+ *    (see vattn_tile_permute); permute/unpermute take/produce RASTER order,
+ *    raster token n = (t*H + y)*W + x.
+ *  - LSE is [batch, heads, N] float32 in the same token order as O: the
+ *    natural log of the softmax denominator, scale included.
+ *  - K_p/V_p are [batch, heads, N_p, head_dim] bfloat16 in pooled-raster
+ *    order, N_p = (T/p_t)(H/p_h)(W/p_w).
+ *  - g is float32 [heads], shared across the batch, values in [0, 1].
+ *  - Every pointer must be 16-byte aligned (VATTN_ERR_ALIGN otherwise).
+ *  - T, H, W must be divisible by the tile and by the pool sizes
+ *    (VATTN_ERR_SHAPE); head_dim must be 64 or 128 and the tile volume a
+ *    multiple of 16 (VATTN_ERR_UNSUPPORTED).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Argument errors are returned synchronously and nothing is
+ *    launched.  A device-side wait that exceeds its time limit makes the
+ *    kernel record VATTN_ERR_DEVICE_TIMEOUT and return early; read it with
+ *    vattn_get_status.
+ *  - On any non-OK return, vattn_last_error() gives a message (thread-local).
+ */
+#ifndef VATTN_H
+#define VATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Geometry of one call.  All triples are in (t, h, w) order.
+ * tile   : tokens per tile along each dim; tile volume s = t_t*t_h*t_w.
+ * window : tiles kept along each dim around the query tile.  Window start
+ *          along a dim with n tiles is clamp(a - window/2, 0, max(n - window, 0))
+ *          and its extent min(window, n), so every query tile keeps
+ *          prod(min(window, n)) tiles.
+ * pool   : K/V pooling block for the global branch (ignored by STA-only calls). */
+typedef struct {
+  int64_t batch, heads, head_dim;
+  int32_t T, H, W;
+  int32_t tile[3];
+  int32_t window[3];
+  int32_t pool[3];
+} vattn_geom;
+
+typedef enum {
+  VATTN_OK = 0,
+  VATTN_ERR_INVALID_ARG = -1,
+  VATTN_ERR_SHAPE = -2,
+  VATTN_ERR_UNSUPPORTED = -3,
+  VATTN_ERR_ALIGN = -4,
+  VATTN_ERR_CUDA = -5,
+  VATTN_ERR_DEVICE_TIMEOUT = -6,
+  VATTN_ERR_WORKSPACE = -7
+} vattn_status;
+
+/* Operation ids for vattn_workspace_size. */
+enum { VATTN_OP_DUAL_FWD = 1, VATTN_OP_STA_BWD = 2, VATTN_OP_DUAL_BWD = 3 };
+
+/* Raster -> tile-major row gather.  Tile-major position of raster token
+ * (t, y, x) is tile_id*s + local_id with
+ *   tile_id  = ((t/t_t)*N_h + y/t_h)*N_w + x/t_w,
+ *   local_id = ((t%t_t)*t_h + y%t_h)*t_w + x%t_w
+ * ("AtlasVid ..." abstract, reordered spatiotemporal windows; "Fast Video
+ * Generation with Sliding Tile Attention" abstract, tile-by-tile operation).
+ * src/dst: batch*heads*N rows of row_bytes bytes each (row_bytes a positive
+ * multiple of 4: 2*head_dim for Q/K/V/O, 4 for LSE).  src and dst must not
+ * overlap. */
+int vattn_tile_permute(const vattn_geom* geom, const void* src_raster, void* dst_tiled,
+                       int64_t row_bytes, void* stream);
+
+/* Inverse of vattn_tile_permute (tile-major -> raster). */
+int vattn_tile_unpermute(const vattn_geom* geom, const void* src_tiled, void* dst_raster,
+                         int64_t row_bytes, void* stream);
+
+/* Kept-tile list ("Fast Video Generation with Sliding Tile Attention",
+ * abstract: each query tile attends to the key tiles of a 3D window around
+ * it).  out: device int32 [n_tiles][kept], n_tiles = prod(grid/tile),
+ * kept = prod(min(window, tiles per dim)); row = query tile id (tile-major),
+ * entries = key tile ids ordered t outermost, w fastest. */
+int vattn_kept_tiles(const vattn_geom* geom, int32_t* out, void* stream);
+
+/* Sliding-tile attention forward (local branch).  For query i in tile a:
+ * S_ij = scale*q_i.k_j over the tokens j of a's kept tiles;
+ * LSE_i = ln sum_j exp(S_ij); O_i = sum_j exp(S_ij - LSE_i) v_j.
+ * q, k, v, o: tile-major bf16 [B,h,N,d]; lse: float32 [B,h,N] tile-major. */
+int vattn_sta_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale,
+                  void* o, float* lse, void* stream);
+
+/* Average pooling of K and V over p_t x p_h x p_w token blocks ("UltraGen ..."
+ * §4.2: latents downsampled before global attention).  Inputs tile-major
+ * [B,h,N,d]; outputs pooled-raster [B,h,N_p,d].  fp32 sum, exact divide by
+ * the block size, one round-to-nearest-even to bf16. */
+int vattn_pool_kv(const vattn_geom* geom, const void* k_tiled, const void* v_tiled, void* kp,
+                  void* vp, void* stream);
+
+/* Global branch forward: every query (tile-major, full resolution) attends to
+ * all N_p pooled keys, no mask ("UltraGen ..." §4.1-4.2).  o, lse as in
+ * vattn_sta_fwd. */
+int vattn_global_fwd(const vattn_geom* geom, const void* q, const void* kp, const void* vp,
+                     float scale, void* o, float* lse, void* stream);
+
+/* Dual-branch forward: pool, local branch, global branch, and the per-head
+ * blend O = g*O_l + (1-g)*O_g ("UltraGen ..." §4.1).  q/k/v/o tile-major.
+ * o_l/lse_l/o_g/lse_g/kp/vp: optional outputs that the backward needs; pass
+ * all six NULL for inference, or all six non-NULL.  When they are NULL the
+ * intermediates live in `workspace` (ws_bytes >= vattn_workspace_size
+ * (VATTN_OP_DUAL_FWD)); otherwise workspace may be NULL. */
+int vattn_dual_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                   const float* g, float scale, void* o, void* o_l, float* lse_l, void* o_g,
+                   float* lse_g, void* kp, void* vp, void* workspace, size_t ws_bytes, void* stream);
+
+/* Sliding-tile attention backward.  Given q, k, v, the forward's o and lse
+ * and the upstream gradient dout (all tile-major), writes dq, dk, dv (bf16,
+ * tile-major).  dV = P^T dO, dP = dO V^T, dS = P*(dP - rowsum(dO*O)),
+ * dQ = scale dS K, dK = scale dS^T Q over the kept pairs only.
+ * workspace >= vattn_workspace_size(VATTN_OP_STA_BWD). */
+int vattn_sta_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                  const void* o, const float* lse, const void* dout, float scale, void* dq,
+                  void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Dual-branch backward: the gradients of O = g*O_l + (1-g)*O_g w.r.t. q, k,
+ * v, including the path through the pooling (dK = dK_l + pool^T(dK_p), same
+ * for V), from the forward's saved o_l, lse_l, o_g, lse_g, kp, vp.
+ * dg (float32 [heads], optional, NULL = skip): sum over batch and tokens of
+ * dO . (O_l - O_g).  workspace >= vattn_workspace_size(VATTN_OP_DUAL_BWD). */
+int vattn_dual_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                   const float* g, const void* o_l, const float* lse_l, const void* o_g,
+                   const float* lse_g, const void* kp, const void* vp, const void* dout,
+                   float scale, void* dq, void* dk, void* dv, float* dg, void* workspace,
+                   size_t ws_bytes, void* stream);
+
+/* Scratch bytes that `op` needs for `geom` (0 if none). */
+int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes);
+
+/* Synchronises `stream`, reads and clears the library's device error word and
+ * the CUDA error state.  Returns VATTN_OK, VATTN_ERR_DEVICE_TIMEOUT or
+ * VATTN_ERR_CUDA. */
+int vattn_get_status(void* stream);
+
+/* Message for the last non-OK return on this thread ("" if none). */
+const char* vattn_last_error(void);
+
+/* Test hook.  flags bit 0: the attention kernels' load warp skips its first
+ * arrival, so the consumer's bounded wait runs out (no fault, no hang);
+ * timeout_ns: the device wait limit (<= 0 restores the default, 2 s).
+ * Affects calls made after it on any thread. */
+int vattn_debug_set(int flags, int64_t timeout_ns);
+
+/* Library version string. */
+const char* vattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VATTN_H */

@@ -369,3 +369,39 @@ def pairs_global(g: Geom, batch: int, heads: int) -> int:
 def ultragen_cost_ratio(K: int) -> float:
     """App. B of "UltraGen ...": (5/(4K^2) + 1/K^4) of full attention's cost."""
     return 5.0 / (4.0 * K * K) + 1.0 / K ** 4
+
+
+# ---------------------------------------------------------------------------
+# sampled evaluation (large grids): the same definitions restricted to a few
+# query tiles / rows of one (batch, head) slice
+# ---------------------------------------------------------------------------
+
+def tile_coords_of(g: Geom, tile_id: int) -> tuple:
+    nt, nh, nw = g.tiles_per_dim
+    return (tile_id // (nh * nw), (tile_id // nw) % nh, tile_id % nw)
+
+
+def sta_attention_tiles(q, k, v, g: Geom, scale: float, tile_ids):
+    """Local branch for the listed query tiles of one head ([N, d] raster
+    inputs).  Returns (raster query ids, O [n, d], LSE [n]) concatenated over
+    the tiles in the given order."""
+    nt, nh, nw = g.tiles_per_dim
+    ids, outs, lses = [], [], []
+    for tid in tile_ids:
+        at, ah, aw = tile_coords_of(g, int(tid))
+        qi = _tile_token_box(g, (at, ah, aw), (at + 1, ah + 1, aw + 1))
+        rt = window_range(at, g.window[0], nt)
+        rh = window_range(ah, g.window[1], nh)
+        rw = window_range(aw, g.window[2], nw)
+        kj = _tile_token_box(g, (rt.start, rh.start, rw.start), (rt.stop, rh.stop, rw.stop))
+        o, lse, _ = _softmax_attend(q[qi], k[kj], v[kj], scale)
+        ids.append(qi)
+        outs.append(o)
+        lses.append(lse)
+    return np.concatenate(ids), np.concatenate(outs), np.concatenate(lses)
+
+
+def global_attention_rows(q, kp, vp, scale: float, rows):
+    """Global branch for the listed raster query rows of one head."""
+    o, lse, _ = _softmax_attend(q[np.asarray(rows)], kp, vp, scale)
+    return o, lse

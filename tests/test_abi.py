@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every symbol include/vattn.h declares, and
+rejects bad arguments synchronously (CPU only: no call here launches work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "vattn.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(vattn_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def V():
+    import video_dit_local_b200 as V
+    return V
+
+
+def test_every_declared_symbol_is_exported(V):
+    names = _declared()
+    assert "vattn_sta_fwd" in names and "vattn_dual_bwd" in names
+    lib = ctypes.CDLL(V.binding.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    # the Python binding offers the same names
+    for n in names:
+        assert hasattr(V.binding, n), n
+
+
+def test_library_has_no_libcuda_link_dependency(V):
+    import subprocess
+    out = subprocess.run(["readelf", "-d", V.binding.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out
+
+
+def test_version(V):
+    assert "sm_100a" in V.vattn_version()
+
+
+def _geom(V, **kw):
+    a = dict(batch=1, heads=2, head_dim=64, grid=(4, 8, 8), tile=(2, 4, 4), window=(1, 2, 2), pool=(1, 2, 2))
+    a.update(kw)
+    return V.make_geom(a["batch"], a["heads"], a["head_dim"], a["grid"], a["tile"], a["window"], a["pool"])
+
+
+def test_argument_errors(V):
+    B = V.binding
+    g = _geom(V)
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd(g, 0, 16, 16, 0.1, 16)
+    assert e.value.code == B.VATTN_ERR_INVALID_ARG and "q is NULL" in str(e.value)
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd(g, 16, 24, 16, 0.1, 16)
+    assert e.value.code == B.VATTN_ERR_ALIGN
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd(_geom(V, grid=(5, 8, 8)), 16, 16, 16, 0.1, 16)
+    assert e.value.code == B.VATTN_ERR_SHAPE
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd(_geom(V, head_dim=96), 16, 16, 16, 0.1, 16)
+    assert e.value.code == B.VATTN_ERR_UNSUPPORTED
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd(_geom(V, tile=(1, 2, 4)), 16, 16, 16, 0.1, 16)   # tile volume 8
+    assert e.value.code == B.VATTN_ERR_UNSUPPORTED
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_pool_kv(_geom(V, pool=(1, 3, 2)), 16, 16, 16, 16)
+    assert e.value.code == B.VATTN_ERR_SHAPE
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_tile_permute(g, 16, 16, 6)
+    assert e.value.code == B.VATTN_ERR_INVALID_ARG
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_dual_fwd(g, 16, 16, 16, 16, 0.1, 16, o_l=16)   # partial set of saved outputs
+    assert e.value.code == B.VATTN_ERR_INVALID_ARG
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_dual_fwd(g, 16, 16, 16, 16, 0.1, 16, workspace=32, ws_bytes=8)
+    assert e.value.code == B.VATTN_ERR_WORKSPACE
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_workspace_size(99, g)
+    assert e.value.code == B.VATTN_ERR_INVALID_ARG
+
+
+def test_empty_batch_is_a_noop(V):
+    g = _geom(V, batch=0)
+    V.vattn_sta_fwd(g, 0, 0, 0, 0.1, 0)      # nothing to do: no pointer is touched
+    V.vattn_dual_fwd(g, 0, 0, 0, 0, 0.1, 0)
+
+
+def test_workspace_sizes(V):
+    g = _geom(V)
+    bh, n, npool, d = 2, 256, 64, 64
+
+    def a(x):
+        return (x + 255) // 256 * 256
+    assert V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, g) == a(bh * n * d * 2) + 2 * a(bh * npool * d * 2)
+    assert V.vattn_workspace_size(V.VATTN_OP_STA_BWD, g) == a(bh * n * 4)
+    assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == 2 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)
+
+
+def test_kernel_geometry_matches_oracle_inverse_ranges():
+    """The device code's window helpers (restated here from the header
+    comment: start = clamp(a - w/2, 0, max(n - w, 0))) agree with the oracle."""
+    from oracle import vattn_oracle as O
+    for n in range(1, 12):
+        for w in range(1, 14):
+            for a in range(n):
+                s = min(max(a - w // 2, 0), max(n - w, 0))
+                assert range(s, s + min(w, n)) == O.window_range(a, w, n)

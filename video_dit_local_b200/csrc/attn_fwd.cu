@@ -1,0 +1,482 @@
+// Attention forward on tcgen05 tensor cores, one kernel for both branches:
+//  - FWD_STA: sliding-tile attention ("Fast Video Generation with Sliding Tile
+//    Attention", abstract).  The query block lies inside one query tile; its
+//    key stream is the box of kept tiles, computed here from the tile
+//    coordinate, so masked tiles are never loaded.
+//  - FWD_GLOBAL: every query attends to all pooled keys ("UltraGen ..." §4.2),
+//    with an optional blend epilogue O = g*O_local + (1-g)*O_global (§4.1).
+//
+// CTA = 128 query rows, 11 warps:
+//   warps 0-3  softmax group 0 (even key blocks), warps 4-7 softmax group 1
+//   (odd key blocks); each group owns one S accumulator and one O
+//   accumulator in TMEM (S0 cols 0-127, S1 128-255, O0 256+, O1 384+), and
+//   the two partial results are merged in the epilogue;
+//   warp 8 loads Q and K, warp 9 loads V (TMA, 128-byte swizzle, no
+//   multicast); warp 10 issues the MMAs and owns the TMEM allocation.
+// P is written back over its own S columns as bf16 and read by the P*V MMA
+// straight from TMEM.  The running max is only moved (and O rescaled) when a
+// row's max grows by more than 2^8; otherwise P may reach 2^8, which bf16 and
+// the fp32 accumulators carry without loss of relative precision.
+#include "common.cuh"
+
+namespace vattn {
+
+namespace fwd {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NTHREADS = 352;
+constexpr int WARP_QK_LOAD = 8;
+constexpr int WARP_V_LOAD = 9;
+constexpr int WARP_MMA = 10;
+constexpr int NK = 3;  // K ring stages
+constexpr int NV = 2;  // V ring stages
+constexpr float RESCALE_LOG2_THRESHOLD = 8.0f;
+
+template <int D>
+struct Smem {
+  static constexpr int CHUNKS = D / 64;                 // 64-column (128-byte) swizzle boxes
+  static constexpr int BLOCK_BYTES = CHUNKS * 128 * 128; // 128 rows x D bf16
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + BLOCK_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * BLOCK_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NV * BLOCK_BYTES;
+  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_XCH = OFF_MISC + 16;
+  static constexpr int TOTAL = OFF_XCH + 2 * 128 * 2 * 4;
+  static constexpr int ALLOC = TOTAL + 1024;
+};
+
+struct Params {
+  DevGeom g;
+  int mode;
+  int G;             // rows per TMA sub-box of a key block (divides the tile volume)
+  int q_blocks_per_tile;
+  int Nk;            // key rows per batch*head in the K/V tensors
+  float scale_log2;  // scale * log2(e)
+  __nv_bfloat16* o;
+  float* lse;
+  const __nv_bfloat16* o_local;
+  const float* gvec;
+  __nv_bfloat16* blend_out;
+  DevCtl ctl;
+};
+
+// Key stream of one CTA: `runs` runs of `run_len` contiguous rows.
+struct Stream {
+  int runs, run_len, eh, t0, h0, w0;
+  __device__ __forceinline__ int length() const { return runs * run_len; }
+};
+
+__device__ __forceinline__ Stream make_stream(const Params& p, int q_tile) {
+  Stream s;
+  if (p.mode == FWD_STA) {
+    const DevGeom& g = p.g;
+    const int at = q_tile / (g.Nh * g.Nw), ah = (q_tile / g.Nw) % g.Nh, aw = q_tile % g.Nw;
+    s.t0 = win_start(at, g.wt, g.Nt);
+    s.h0 = win_start(ah, g.wh, g.Nh);
+    s.w0 = win_start(aw, g.ww, g.Nw);
+    const int et = win_extent(g.wt, g.Nt);
+    s.eh = win_extent(g.wh, g.Nh);
+    s.runs = et * s.eh;
+    s.run_len = win_extent(g.ww, g.Nw) * g.s;
+  } else {
+    s.runs = 1;
+    s.run_len = p.Nk;
+    s.eh = 1;
+    s.t0 = s.h0 = s.w0 = 0;
+  }
+  return s;
+}
+
+// Key row (within the batch*head slice) of stream position v < length().
+__device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int v) {
+  if (p.mode != FWD_STA) return v;
+  const int r = v / s.run_len, o = v - r * s.run_len;
+  const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
+  return ((kt * p.g.Nh + kh) * p.g.Nw + s.w0) * p.g.s + o;
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using L = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + NK;
+  uint64_t* v_full = k_empty + NK;
+  uint64_t* v_empty = v_full + NV;
+  uint64_t* s_full = v_empty + NV;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_final = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  float2* xch = reinterpret_cast<float2*>(smem + L::OFF_XCH);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int qblk = blockIdx.x;
+  WaitCtx wc;
+  wc.abort_flag = abort_flag;
+  wc.timeout_ns = p.ctl.timeout_ns;
+  wc.err_word = p.ctl.err_word;
+
+  // query block -> rows
+  int q_tile, q_row0, q_valid;
+  if (p.mode == FWD_STA) {
+    q_tile = qblk / p.q_blocks_per_tile;
+    const int sub = qblk - q_tile * p.q_blocks_per_tile;
+    q_row0 = q_tile * p.g.s + sub * BM;
+    q_valid = min(BM, p.g.s - sub * BM);
+  } else {
+    q_tile = 0;
+    q_row0 = qblk * BM;
+    q_valid = min(BM, p.g.N - q_row0);
+  }
+  const Stream st = make_stream(p, q_tile);
+  const int L_total = st.length();
+  const int nblk = (L_total + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(o_final, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == WARP_QK_LOAD && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  constexpr uint32_t BOX_BYTES = 128 * 128;   // one 128-row x 128-byte box
+  const uint32_t sub_bytes = (uint32_t)p.G * 128;
+  const int subs = BN / p.G;
+
+  if (warp == WARP_QK_LOAD) {
+    if (lane == 0) {
+      int issued_k = 0;
+      if (!(p.ctl.debug_flags & 1)) {
+        mbar_arrive_expect_tx(q_full, L::BLOCK_BYTES);
+        for (int c = 0; c < L::CHUNKS; ++c)
+          tma_load_3d(smem + L::OFF_Q + c * BOX_BYTES, &tm_q, q_full, c * 64, q_row0, bh);
+      }
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NK, r = j / NK;
+        if (!mbar_wait(&k_empty[s], (r & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&k_full[s], L::BLOCK_BYTES);
+        uint8_t* dst = smem + L::OFF_K + s * L::BLOCK_BYTES;
+        for (int u = 0; u < subs; ++u) {
+          const int v = j * BN + u * p.G;
+          const int row = v < L_total ? stream_row(p, st, v) : p.Nk;  // past the end: zero fill
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * 64, row, bh);
+        }
+        ++issued_k;
+      }
+      {  // every issued load has landed before the CTA can exit (a no-op unless aborted)
+        for (int j = issued_k - NK < 0 ? 0 : issued_k - NK; j < issued_k; ++j)
+          mbar_wait_drain(&k_full[j % NK], (j / NK) & 1, wc);
+      }
+    }
+  } else if (warp == WARP_V_LOAD) {
+    if (lane == 0) {
+      int issued_v = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NV, r = j / NV;
+        if (!mbar_wait(&v_empty[s], (r & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&v_full[s], L::BLOCK_BYTES);
+        uint8_t* dst = smem + L::OFF_V + s * L::BLOCK_BYTES;
+        for (int u = 0; u < subs; ++u) {
+          const int v = j * BN + u * p.G;
+          const int row = v < L_total ? stream_row(p, st, v) : p.Nk;
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * 64, row, bh);
+        }
+        ++issued_v;
+      }
+      {
+        for (int j = issued_v - NV < 0 ? 0 : issued_v - NV; j < issued_v; ++j)
+          mbar_wait_drain(&v_full[j % NV], (j / NV) & 1, wc);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
+      const uint32_t q_base = smem_u32(smem + L::OFF_Q);
+      const uint32_t k_base = smem_u32(smem + L::OFF_K);
+      const uint32_t v_base = smem_u32(smem + L::OFF_V);
+      bool ok = mbar_wait(q_full, 0, wc);
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j % NK;
+        if (!mbar_wait(&k_full[s], (j / NK) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t kb = k_base + s * L::BLOCK_BYTES;
+        const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 128);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
+                 kk > 0);
+        }
+        tc_commit(&k_empty[s]);
+        tc_commit(&s_full[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && nblk > 1) ok = issue_qk(1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int w = j & 1;
+        if (!mbar_wait(&p_full[w], (j >> 1) & 1, wc)) break;
+        const int s = j % NV;
+        if (!mbar_wait(&v_full[s], (j / NV) & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t vb = v_base + s * L::BLOCK_BYTES;
+        const uint32_t o_tmem = tmem + 256 + (uint32_t)(w * 128);
+        const uint32_t p_tmem = tmem + (uint32_t)(w * 128);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // B = V block (keys x d), MN-major: LBO = next 64-column box, SBO = next 8 keys
+          mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, BOX_BYTES, 1024), IDESC_PV,
+                 (j >= 2 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&v_empty[s]);
+        if (j + 2 < nblk) ok = issue_qk(j + 2);
+      }
+      tc_commit(o_final);
+      // every MMA this thread issued must be finished before TMEM is freed
+      mbar_wait_drain(o_final, 0, wc);
+    }
+  } else {
+    // ---------------- softmax groups ----------------
+    const int w = warp >> 2;            // group 0: warps 0-3, group 1: warps 4-7
+    const int quad = warp & 3;          // TMEM lane quarter
+    const int row = quad * 32 + lane;   // query row within the block
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 128);
+    const uint32_t tO = tmem + lane_addr + 256u + (uint32_t)(w * 128);
+    const float c2 = p.scale_log2;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int i = 0;; ++i) {
+      const int j = 2 * i + w;
+      if (j >= nblk) break;
+      ok = mbar_wait(&s_full[w], i & 1, wc);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, sr[q4]);
+      tmem_wait_ld();
+      const int valid = L_total - j * BN;
+      if (valid < BN) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (q4 * 32 + c >= valid) sr[q4][c] = __float_as_uint(-INFINITY);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[q4][c]));
+      const float mx2 = mx * c2;
+      bool need = false;
+      if (i == 0) {
+        m_ref = mx2;
+      } else if (mx2 > m_ref + RESCALE_LOG2_THRESHOLD) {
+        need = true;
+      }
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m_ref - mx2);
+        m_ref = mx2;
+        l_sum *= alpha;
+      }
+      const float neg_m = -m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[q4][2 * c]), c2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[q4][2 * c + 1]), c2, neg_m));
+          sum += p0 + p1;
+          pk[c] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tS + q4 * 16, pk);
+      }
+      l_sum += sum;
+      if (__any_sync(0xffffffffu, need)) {
+        // O of this group is quiescent: the commit that signalled this S also
+        // covers the previous P*V into it, and the next one waits for p_full.
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tO + c0, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[w]);
+    }
+    // ---------------- epilogue ----------------
+    if (ok && !*abort_flag) ok = mbar_wait(o_final, 0, wc);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    xch[w * 128 + row] = make_float2(m_ref, l_sum);
+    named_bar_sync(1, 256);
+    if (ok && !*abort_flag) {
+      const float2 other = xch[(1 - w) * 128 + row];
+      const float m = fmaxf(m_ref, other.x);
+      const float a_self = ex2(m_ref - m), a_other = ex2(other.x - m);
+      const float l = l_sum * a_self + other.y * a_other;
+      const float inv_l = 1.f / l;
+      const float a0 = (w == 0 ? a_self : a_other) * inv_l;
+      const float a1 = (w == 0 ? a_other : a_self) * inv_l;
+      const bool have1 = nblk >= 2;
+      const bool row_ok = row < q_valid;
+      const size_t grow = (size_t)bh * p.g.N + (size_t)(q_row0 + row);
+      const uint32_t tO0 = tmem + lane_addr + 256u, tO1 = tmem + lane_addr + 384u;
+      float gh = 0.f;
+      if (p.blend_out) gh = p.gvec[bh % p.g.heads];
+#pragma unroll
+      for (int c0 = (w * D) / 2; c0 < ((w + 1) * D) / 2; c0 += 32) {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tO0 + c0, x0);
+        if (have1) tmem_ld32(tO1 + c0, x1);
+        tmem_wait_ld();
+        float* o = reinterpret_cast<float*>(x0);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          o[c] = __uint_as_float(x0[c]) * a0 + (have1 ? __uint_as_float(x1[c]) * a1 : 0.f);
+        if (row_ok) {
+          if (p.o) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pack_bf16(o[8 * v4 + 0], o[8 * v4 + 1]), pack_bf16(o[8 * v4 + 2], o[8 * v4 + 3]),
+                                   pack_bf16(o[8 * v4 + 4], o[8 * v4 + 5]), pack_bf16(o[8 * v4 + 6], o[8 * v4 + 7]));
+          }
+          if (p.blend_out) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.o_local + grow * D + c0);
+            uint4* dst = reinterpret_cast<uint4*>(p.blend_out + grow * D + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              const uint4 ol = src[v4];
+              const uint32_t w4[4] = {ol.x, ol.y, ol.z, ol.w};
+              uint32_t r4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                r4[e] = pack_bf16(gh * bf16lo(w4[e]) + (1.f - gh) * o[8 * v4 + 2 * e],
+                                  gh * bf16hi(w4[e]) + (1.f - gh) * o[8 * v4 + 2 * e + 1]);
+              dst[v4] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+            }
+          }
+        }
+      }
+      if (w == 0 && row_ok && p.lse) p.lse[grow] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+
+bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
+                    const char** err);
+
+template <int D>
+static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
+  using namespace fwd;
+  Params p;
+  p.g = g;
+  p.mode = mode;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.o = (__nv_bfloat16*)a.o;
+  p.lse = a.lse;
+  p.o_local = (const __nv_bfloat16*)a.o_local;
+  p.gvec = a.g;
+  p.blend_out = a.o_local ? (__nv_bfloat16*)a.blend_out : nullptr;
+  p.ctl = current_ctl();
+  int qblocks;
+  if (mode == FWD_STA) {
+    int G = 1;
+    while (G < BN && g.s % (G * 2) == 0) G *= 2;
+    p.G = G;
+    p.q_blocks_per_tile = (g.s + BM - 1) / BM;
+    p.Nk = g.N;
+    qblocks = g.n_tiles * p.q_blocks_per_tile;
+  } else {
+    p.G = BN;
+    p.q_blocks_per_tile = 1;
+    p.Nk = g.Np;
+    qblocks = (g.N + BM - 1) / BM;
+  }
+  const long long bh = (long long)g.B * g.heads;
+  if (qblocks == 0 || bh == 0) return cudaSuccess;
+  CUtensorMap tq, tk, tv;
+  const char* err = nullptr;
+  if (!make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) || !make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err) ||
+      !make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err))
+    return cudaErrorInvalidValue;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Smem<D>::ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(qblocks, (unsigned)bh);
+  attn_fwd_kernel<D><<<grid, NTHREADS, Smem<D>::ALLOC, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
+  if (g.d == 128) return launch_fwd_d<128>(g, mode, a, st);
+  if (g.d == 64) return launch_fwd_d<64>(g, mode, a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vattn

@@ -1,0 +1,253 @@
+// HBM-bound kernels: raster <-> tile-major row gather, the kept-tile list, and
+// K/V average pooling.  All of them are grid-stride loops over 16-byte
+// vectors with 32-bit index math done by multiply-high division.
+#include "common.cuh"
+
+namespace vattn {
+
+// Unsigned 32-bit division by a runtime constant via a precomputed
+// multiplier (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994): q = (umulhi(n, m) + n) >> s  for n < 2^31.
+struct FastDiv {
+  uint32_t d, m, s;
+  FastDiv() = default;
+  explicit FastDiv(uint32_t div) : d(div) {
+    s = 0;
+    while ((1u << s) < div) ++s;  // s = ceil(log2(div))
+    const uint64_t one = 1;
+    m = static_cast<uint32_t>(((one << 32) * ((one << s) - div)) / div + 1);
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
+};
+
+struct ReorderParams {
+  FastDiv s, nhnw, nw, thtw, tw;      // tile-major -> raster
+  FastDiv W, H, tt, th, tww;          // raster -> tile-major
+  uint32_t T, Hh, Ww, ttt, tth, ttw, Nh, Nw, vol;
+};
+
+// tile-major position m -> raster token
+__device__ __forceinline__ uint32_t tiled_to_raster(const ReorderParams& p, uint32_t m) {
+  const uint32_t tile = p.s.div(m);
+  const uint32_t l = m - tile * p.vol;
+  const uint32_t at = p.nhnw.div(tile);
+  const uint32_t rem = tile - at * p.Nh * p.Nw;
+  const uint32_t ah = p.nw.div(rem);
+  const uint32_t aw = rem - ah * p.Nw;
+  const uint32_t lt = p.thtw.div(l);
+  const uint32_t rl = l - lt * p.tth * p.ttw;
+  const uint32_t lh = p.tw.div(rl);
+  const uint32_t lw = rl - lh * p.ttw;
+  return ((at * p.ttt + lt) * p.Hh + ah * p.tth + lh) * p.Ww + aw * p.ttw + lw;
+}
+
+// raster token (t, y, x) -> tile-major position
+__device__ __forceinline__ uint32_t coords_to_tiled(const ReorderParams& p, uint32_t t, uint32_t y, uint32_t x) {
+  const uint32_t at = p.tt.div(t), ah = p.th.div(y), aw = p.tww.div(x);
+  const uint32_t lt = t - at * p.ttt, lh = y - ah * p.tth, lw = x - aw * p.ttw;
+  return ((at * p.Nh + ah) * p.Nw + aw) * p.vol + (lt * p.tth + lh) * p.ttw + lw;
+}
+
+__device__ __forceinline__ uint32_t raster_to_tiled(const ReorderParams& p, uint32_t n) {
+  const uint32_t r = p.W.div(n);
+  const uint32_t x = n - r * p.Ww;
+  const uint32_t t = p.H.div(r);
+  const uint32_t y = r - t * p.Hh;
+  return coords_to_tiled(p, t, y, x);
+}
+
+static ReorderParams make_params(const DevGeom& g) {
+  ReorderParams p;
+  p.s = FastDiv(g.s);
+  p.nhnw = FastDiv(g.Nh * g.Nw);
+  p.nw = FastDiv(g.Nw);
+  p.thtw = FastDiv(g.th * g.tw);
+  p.tw = FastDiv(g.tw);
+  p.W = FastDiv(g.W);
+  p.H = FastDiv(g.H);
+  p.tt = FastDiv(g.tt);
+  p.th = FastDiv(g.th);
+  p.tww = FastDiv(g.tw);
+  p.T = g.T;
+  p.Hh = g.H;
+  p.Ww = g.W;
+  p.ttt = g.tt;
+  p.tth = g.th;
+  p.ttw = g.tw;
+  p.Nh = g.Nh;
+  p.Nw = g.Nw;
+  p.vol = g.s;
+  return p;
+}
+
+// Every destination row is written once.  A row is `units` words of UNIT
+// bytes (uint4 when the row is a multiple of 16 bytes, else uint32).  Indices
+// are 32-bit: the host splits the batch*head range so that every launch
+// covers fewer than 2^31 words.  TO_TILED: dst is tile-major, src raster.
+template <bool TO_TILED, typename U>
+__global__ void __launch_bounds__(256) permute_kernel(ReorderParams p, FastDiv per_row, FastDiv n_rows,
+                                                       const U* __restrict__ src, U* __restrict__ dst,
+                                                       uint32_t total) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t row = per_row.div(i);
+    const uint32_t c = i - row * per_row.d;
+    const uint32_t bh = n_rows.div(row);
+    const uint32_t r = row - bh * n_rows.d;
+    const uint32_t sr = TO_TILED ? tiled_to_raster(p, r) : raster_to_tiled(p, r);
+    const U v = __ldg(src + ((size_t)bh * n_rows.d + sr) * per_row.d + c);
+    __stcs(dst + i, v);
+  }
+}
+
+static int grid_for(long long work, int threads) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long blocks = (work + threads - 1) / threads;
+  long long cap = (long long)sms * 8;  // 8 resident 256-thread blocks per SM
+  if (blocks > cap) blocks = cap;
+  return (int)(blocks < 1 ? 1 : blocks);
+}
+
+template <typename U>
+static cudaError_t permute_typed(const DevGeom& g, const void* src, void* dst, uint32_t units, bool to_tiled,
+                                 cudaStream_t st) {
+  const ReorderParams p = make_params(g);
+  const long long per_bh = (long long)g.N * units;
+  const long long bh_total = (long long)g.B * g.heads;
+  long long chunk = ((1ll << 31) - 1) / per_bh;
+  if (chunk < 1) return cudaErrorInvalidValue;
+  for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
+    const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
+    const uint32_t total = (uint32_t)(nb * per_bh);
+    const U* s = (const U*)src + b0 * per_bh;
+    U* d = (U*)dst + b0 * per_bh;
+    const int grid = grid_for(total, 256);
+    if (to_tiled)
+      permute_kernel<true, U><<<grid, 256, 0, st>>>(p, FastDiv(units), FastDiv(g.N), s, d, total);
+    else
+      permute_kernel<false, U><<<grid, 256, 0, st>>>(p, FastDiv(units), FastDiv(g.N), s, d, total);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const DevGeom& g, const void* src, void* dst, int64_t row_bytes, bool to_tiled,
+                           cudaStream_t st) {
+  if ((long long)g.B * g.heads * g.N == 0) return cudaSuccess;
+  if (row_bytes % 16 == 0) return permute_typed<uint4>(g, src, dst, (uint32_t)(row_bytes / 16), to_tiled, st);
+  return permute_typed<uint32_t>(g, src, dst, (uint32_t)(row_bytes / 4), to_tiled, st);
+}
+
+// ---------------------------------------------------------------------------
+// kept-tile list
+// ---------------------------------------------------------------------------
+__global__ void kept_tiles_kernel(DevGeom g, int32_t* __restrict__ out) {
+  const int total = g.n_tiles * g.kept;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int qt = i / g.kept, j = i - qt * g.kept;
+    const int at = qt / (g.Nh * g.Nw), ah = (qt / g.Nw) % g.Nh, aw = qt % g.Nw;
+    const int et = win_extent(g.wt, g.Nt), eh = win_extent(g.wh, g.Nh), ew = win_extent(g.ww, g.Nw);
+    (void)et;
+    const int jt = j / (eh * ew), jh = (j / ew) % eh, jw = j % ew;
+    const int kt = win_start(at, g.wt, g.Nt) + jt;
+    const int kh = win_start(ah, g.wh, g.Nh) + jh;
+    const int kw = win_start(aw, g.ww, g.Nw) + jw;
+    out[i] = (kt * g.Nh + kh) * g.Nw + kw;
+  }
+}
+
+cudaError_t launch_kept_tiles(const DevGeom& g, int32_t* out, cudaStream_t st) {
+  const int total = g.n_tiles * g.kept;
+  kept_tiles_kernel<<<grid_for(total, 256), 256, 0, st>>>(g, out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K/V average pooling: tile-major input -> pooled-raster output
+// ("UltraGen ..." §4.2, spatially compressed global attention)
+// ---------------------------------------------------------------------------
+struct PoolParams {
+  ReorderParams rp;
+  FastDiv PW, PH;      // pooled grid divisions
+  uint32_t pt, ph, pw, PWv, PHv, N, Np, vpr;
+  float inv_cnt;
+};
+
+// One thread produces one 16-byte vector (8 bf16) of one pooled row: the fp32
+// sum of the block's tokens in (t, y, x) order, times 1/count (exact: count is
+// a product of the pool sizes; a power of two at every shipped geometry),
+// one round-to-nearest-even to bf16.
+__global__ void __launch_bounds__(256) pool_kv_kernel(PoolParams p, FastDiv per_row, FastDiv n_prow,
+                                                       const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                       uint4* __restrict__ kp, uint4* __restrict__ vp,
+                                                       uint32_t rows_per_tensor) {
+  const uint32_t total = 2 * rows_per_tensor * p.vpr;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t row2 = per_row.div(i);
+    const uint32_t c = i - row2 * p.vpr;
+    const bool is_v = row2 >= rows_per_tensor;
+    const uint32_t row = is_v ? row2 - rows_per_tensor : row2;
+    const uint32_t bh = n_prow.div(row);
+    const uint32_t u = row - bh * p.Np;
+    const uint32_t r = p.PW.div(u);
+    const uint32_t ux = u - r * p.PWv;
+    const uint32_t ut = p.PH.div(r);
+    const uint32_t uy = r - ut * p.PHv;
+    const uint4* src = (is_v ? v : k) + (size_t)bh * p.N * p.vpr + c;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (uint32_t a = 0; a < p.pt; ++a)
+      for (uint32_t b = 0; b < p.ph; ++b)
+        for (uint32_t x = 0; x < p.pw; ++x) {
+          const uint32_t m = coords_to_tiled(p.rp, ut * p.pt + a, uy * p.ph + b, ux * p.pw + x);
+          const uint4 w = __ldg(src + (size_t)m * p.vpr);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += bf16lo(ww[e]);
+            acc[2 * e + 1] += bf16hi(ww[e]);
+          }
+        }
+    uint4 o;
+    o.x = pack_bf16(acc[0] * p.inv_cnt, acc[1] * p.inv_cnt);
+    o.y = pack_bf16(acc[2] * p.inv_cnt, acc[3] * p.inv_cnt);
+    o.z = pack_bf16(acc[4] * p.inv_cnt, acc[5] * p.inv_cnt);
+    o.w = pack_bf16(acc[6] * p.inv_cnt, acc[7] * p.inv_cnt);
+    (is_v ? vp : kp)[(size_t)row * p.vpr + c] = o;
+  }
+}
+
+cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void* kp, void* vp, cudaStream_t st) {
+  PoolParams p;
+  p.rp = make_params(g);
+  p.PW = FastDiv(g.PW);
+  p.PH = FastDiv(g.PH);
+  p.pt = g.pt;
+  p.ph = g.ph;
+  p.pw = g.pw;
+  p.PWv = g.PW;
+  p.PHv = g.PH;
+  p.N = g.N;
+  p.Np = g.Np;
+  p.vpr = g.d / 8;
+  p.inv_cnt = 1.0f / (float)(g.pt * g.ph * g.pw);
+  const long long per_bh = (long long)g.Np * p.vpr;
+  const long long bh_total = (long long)g.B * g.heads;
+  if (per_bh * bh_total == 0) return cudaSuccess;
+  const long long chunk = ((1ll << 30) - 1) / per_bh;  // 2 tensors per launch: stay below 2^31 vectors
+  if (chunk < 1) return cudaErrorInvalidValue;
+  for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
+    const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
+    const uint32_t rows = (uint32_t)(nb * g.Np);
+    const size_t in_off = (size_t)b0 * g.N * p.vpr, out_off = (size_t)b0 * g.Np * p.vpr;
+    pool_kv_kernel<<<grid_for(2ll * rows * p.vpr, 256), 256, 0, st>>>(
+        p, FastDiv(p.vpr), FastDiv(g.Np), (const uint4*)k + in_off, (const uint4*)v + in_off,
+        (uint4*)kp + out_off, (uint4*)vp + out_off, rows);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace vattn

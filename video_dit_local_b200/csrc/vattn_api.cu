@@ -1,0 +1,500 @@
+// C-ABI entry points: argument validation, workspace carving, TMA descriptor
+// encoding and kernel launches on the caller's stream.  No device memory is
+// allocated here.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+
+namespace vattn {
+
+__device__ int g_error_word = 0;
+
+static thread_local std::string t_last_error;
+static std::atomic<int> s_debug_flags{0};
+static std::atomic<long long> s_timeout_ns{2000000000ll};
+
+// Address of this device's status word (cached per device).
+static int* error_word_ptr() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) cache[dev] = (int*)p;
+  }
+  return cache[dev];
+}
+
+DevCtl current_ctl() {
+  DevCtl c;
+  c.timeout_ns = (unsigned long long)s_timeout_ns.load();
+  c.err_word = error_word_ptr();
+  c.debug_flags = s_debug_flags.load();
+  return c;
+}
+
+static int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+static int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return code;
+}
+
+static int ok() {
+  t_last_error.clear();
+  return VATTN_OK;
+}
+
+static int cuda_fail(cudaError_t e, const char* what) {
+  return fail(VATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no link-time
+// dependency on libcuda)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::atomic<bool> tried{false};
+  if (!fn && !tried.exchange(true)) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
+                    const char** err) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows_per_bh, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows_per_bh * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed";
+    return false;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+enum Need { NEED_TILE = 1, NEED_POOL = 2, NEED_ATTN = 4 };
+
+static int build_geom(const vattn_geom* in, int need, DevGeom* g) {
+  if (!in) return fail(VATTN_ERR_INVALID_ARG, "geom is NULL");
+  if (in->batch < 0 || in->heads < 0) return fail(VATTN_ERR_INVALID_ARG, "batch/heads must be >= 0");
+  if (in->T <= 0 || in->H <= 0 || in->W <= 0) return fail(VATTN_ERR_INVALID_ARG, "T, H, W must be > 0");
+  for (int i = 0; i < 3; ++i) {
+    if (in->tile[i] <= 0 || in->window[i] <= 0) return fail(VATTN_ERR_INVALID_ARG, "tile/window must be > 0");
+    if ((need & NEED_POOL) && in->pool[i] <= 0) return fail(VATTN_ERR_INVALID_ARG, "pool must be > 0");
+  }
+  if (in->T % in->tile[0] || in->H % in->tile[1] || in->W % in->tile[2])
+    return fail(VATTN_ERR_SHAPE, "grid %dx%dx%d not divisible by tile %dx%dx%d", in->T, in->H, in->W, in->tile[0],
+                in->tile[1], in->tile[2]);
+  if ((need & NEED_POOL) && (in->T % in->pool[0] || in->H % in->pool[1] || in->W % in->pool[2]))
+    return fail(VATTN_ERR_SHAPE, "grid %dx%dx%d not divisible by pool %dx%dx%d", in->T, in->H, in->W, in->pool[0],
+                in->pool[1], in->pool[2]);
+  const long long N = (long long)in->T * in->H * in->W;
+  if (N >= (1ll << 31)) return fail(VATTN_ERR_UNSUPPORTED, "N = T*H*W must be < 2^31");
+  if ((need & NEED_ATTN) && in->head_dim != 64 && in->head_dim != 128)
+    return fail(VATTN_ERR_UNSUPPORTED, "head_dim %lld not supported (64 or 128)", (long long)in->head_dim);
+  if (in->head_dim <= 0 || in->head_dim > 4096) return fail(VATTN_ERR_INVALID_ARG, "head_dim out of range");
+  if (in->batch * in->heads >= 65536) return fail(VATTN_ERR_UNSUPPORTED, "batch*heads must be < 65536");
+  g->B = (int)in->batch;
+  g->heads = (int)in->heads;
+  g->d = (int)in->head_dim;
+  g->N = (int)N;
+  g->T = in->T;
+  g->H = in->H;
+  g->W = in->W;
+  g->tt = in->tile[0];
+  g->th = in->tile[1];
+  g->tw = in->tile[2];
+  g->wt = in->window[0];
+  g->wh = in->window[1];
+  g->ww = in->window[2];
+  g->pt = (need & NEED_POOL) ? in->pool[0] : 1;
+  g->ph = (need & NEED_POOL) ? in->pool[1] : 1;
+  g->pw = (need & NEED_POOL) ? in->pool[2] : 1;
+  g->Nt = g->T / g->tt;
+  g->Nh = g->H / g->th;
+  g->Nw = g->W / g->tw;
+  g->s = g->tt * g->th * g->tw;
+  g->n_tiles = g->Nt * g->Nh * g->Nw;
+  g->kept = win_extent(g->wt, g->Nt) * win_extent(g->wh, g->Nh) * win_extent(g->ww, g->Nw);
+  g->PT = g->T / g->pt;
+  g->PH = g->H / g->ph;
+  g->PW = g->W / g->pw;
+  g->Np = g->PT * g->PH * g->PW;
+  if ((need & NEED_ATTN) && g->s % 16 != 0)
+    return fail(VATTN_ERR_UNSUPPORTED, "tile volume %d must be a multiple of 16", g->s);
+  return VATTN_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE_PTR(p)                                                                  \
+  do {                                                                                  \
+    if (!(p)) return fail(VATTN_ERR_INVALID_ARG, "%s is NULL", #p);                     \
+    if (!aligned16(p)) return fail(VATTN_ERR_ALIGN, "%s is not 16-byte aligned", #p);   \
+  } while (0)
+
+#define CHECK_LAUNCH(expr, what)                 \
+  do {                                           \
+    cudaError_t e_ = (expr);                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+static inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static bool empty_geom(const DevGeom& g) { return (long long)g.B * g.heads == 0; }
+
+struct DualFwdWs {
+  size_t o_l, kp, vp, total;
+};
+static DualFwdWs dual_fwd_ws(const DevGeom& g) {
+  DualFwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  w.o_l = 0;
+  w.kp = align256(bh * g.N * g.d * 2);
+  w.vp = w.kp + align256(bh * g.Np * g.d * 2);
+  w.total = w.vp + align256(bh * g.Np * g.d * 2);
+  return w;
+}
+struct BwdWs {
+  size_t delta_l, delta_g, dkp, dvp, total;
+};
+static BwdWs bwd_ws(const DevGeom& g, bool dual) {
+  BwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  w.delta_l = 0;
+  w.delta_g = align256(bh * g.N * 4);
+  if (!dual) {
+    w.dkp = w.dvp = w.total = w.delta_g;
+    return w;
+  }
+  w.dkp = w.delta_g + align256(bh * g.N * 4);
+  w.dvp = w.dkp + align256(bh * g.Np * g.d * 4);
+  w.total = w.dvp + align256(bh * g.Np * g.d * 4);
+  return w;
+}
+
+}  // namespace vattn
+
+using namespace vattn;
+
+extern "C" {
+
+const char* vattn_version(void) { return "vattn 0.1.0 (sm_100a)"; }
+
+const char* vattn_last_error(void) { return t_last_error.c_str(); }
+
+int vattn_debug_set(int flags, int64_t timeout_ns) {
+  s_debug_flags.store(flags);
+  s_timeout_ns.store(timeout_ns > 0 ? (long long)timeout_ns : 2000000000ll);
+  return ok();
+}
+
+int vattn_get_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending CUDA error");
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (word != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    return fail(word, "device reported status %d (a bounded wait ran out)", word);
+  }
+  return ok();
+}
+
+int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
+  if (!bytes) return fail(VATTN_ERR_INVALID_ARG, "bytes is NULL");
+  DevGeom g;
+  int need = NEED_TILE | NEED_ATTN | (op == VATTN_OP_STA_BWD ? 0 : NEED_POOL);
+  int r = build_geom(geom, need, &g);
+  if (r) return r;
+  switch (op) {
+    case VATTN_OP_DUAL_FWD: *bytes = dual_fwd_ws(g).total; break;
+    case VATTN_OP_STA_BWD: *bytes = bwd_ws(g, false).total; break;
+    case VATTN_OP_DUAL_BWD: *bytes = bwd_ws(g, true).total; break;
+    default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
+  }
+  return ok();
+}
+
+int vattn_tile_permute(const vattn_geom* geom, const void* src, void* dst, int64_t row_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE, &g);
+  if (r) return r;
+  if (row_bytes <= 0 || row_bytes % 4) return fail(VATTN_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 4");
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(src);
+  REQUIRE_PTR(dst);
+  if (src == dst) return fail(VATTN_ERR_INVALID_ARG, "src and dst must not overlap");
+  CHECK_LAUNCH(launch_permute(g, src, dst, row_bytes, true, (cudaStream_t)stream), "tile_permute launch");
+  return ok();
+}
+
+int vattn_tile_unpermute(const vattn_geom* geom, const void* src, void* dst, int64_t row_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE, &g);
+  if (r) return r;
+  if (row_bytes <= 0 || row_bytes % 4) return fail(VATTN_ERR_INVALID_ARG, "row_bytes must be a positive multiple of 4");
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(src);
+  REQUIRE_PTR(dst);
+  if (src == dst) return fail(VATTN_ERR_INVALID_ARG, "src and dst must not overlap");
+  CHECK_LAUNCH(launch_permute(g, src, dst, row_bytes, false, (cudaStream_t)stream), "tile_unpermute launch");
+  return ok();
+}
+
+int vattn_kept_tiles(const vattn_geom* geom, int32_t* out, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE, &g);
+  if (r) return r;
+  REQUIRE_PTR(out);
+  CHECK_LAUNCH(launch_kept_tiles(g, out, (cudaStream_t)stream), "kept_tiles launch");
+  return ok();
+}
+
+int vattn_sta_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                  float* lse, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  if (lse && !aligned16(lse)) return fail(VATTN_ERR_ALIGN, "lse is not 16-byte aligned");
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, (cudaStream_t)stream), "sta_fwd launch");
+  return ok();
+}
+
+int vattn_pool_kv(const vattn_geom* geom, const void* k, const void* v, void* kp, void* vp, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL, &g);
+  if (r) return r;
+  if (g.d % 8) return fail(VATTN_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(kp);
+  REQUIRE_PTR(vp);
+  CHECK_LAUNCH(launch_pool_kv(g, k, v, kp, vp, (cudaStream_t)stream), "pool_kv launch");
+  return ok();
+}
+
+int vattn_global_fwd(const vattn_geom* geom, const void* q, const void* kp, const void* vp, float scale, void* o,
+                     float* lse, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kp);
+  REQUIRE_PTR(vp);
+  REQUIRE_PTR(o);
+  if (lse && !aligned16(lse)) return fail(VATTN_ERR_ALIGN, "lse is not 16-byte aligned");
+  FwdArgs a{};
+  a.q = q;
+  a.k = kp;
+  a.v = vp;
+  a.o = o;
+  a.lse = lse;
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_GLOBAL, a, (cudaStream_t)stream), "global_fwd launch");
+  return ok();
+}
+
+int vattn_dual_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* gvec,
+                   float scale, void* o, void* o_l, float* lse_l, void* o_g, float* lse_g, void* kp, void* vp,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(gvec);
+  REQUIRE_PTR(o);
+  const int n_saved = (o_l != nullptr) + (lse_l != nullptr) + (o_g != nullptr) + (lse_g != nullptr) +
+                      (kp != nullptr) + (vp != nullptr);
+  if (n_saved != 0 && n_saved != 6)
+    return fail(VATTN_ERR_INVALID_ARG, "o_l, lse_l, o_g, lse_g, kp, vp must be all NULL or all non-NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (n_saved == 0) {
+    const DualFwdWs w = dual_fwd_ws(g);
+    if (!workspace || ws_bytes < w.total)
+      return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+    if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+    uint8_t* ws = (uint8_t*)workspace;
+    o_l = ws + w.o_l;
+    kp = ws + w.kp;
+    vp = ws + w.vp;
+  } else {
+    REQUIRE_PTR(o_l);
+    REQUIRE_PTR(lse_l);
+    REQUIRE_PTR(o_g);
+    REQUIRE_PTR(lse_g);
+    REQUIRE_PTR(kp);
+    REQUIRE_PTR(vp);
+  }
+  CHECK_LAUNCH(launch_pool_kv(g, k, v, kp, vp, st), "dual_fwd pool launch");
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o_l;
+  a.lse = lse_l;
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "dual_fwd local launch");
+  FwdArgs b{};
+  b.q = q;
+  b.k = kp;
+  b.v = vp;
+  b.o = o_g;  // NULL at inference: only the blended output is written
+  b.lse = lse_g;
+  b.scale = scale;
+  b.o_local = o_l;
+  b.g = gvec;
+  b.blend_out = o;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_GLOBAL, b, st), "dual_fwd global launch");
+  return ok();
+}
+
+int vattn_sta_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const void* o,
+                  const float* lse, const void* dout, float scale, void* dq, void* dk, void* dv, void* workspace,
+                  size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(lse);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  const BwdWs w = bwd_ws(g, false);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.o_l = o;
+  a.lse_l = lse;
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.delta_l = (float*)((uint8_t*)workspace + w.delta_l);
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_bwd_preprocess(g, a, false, st), "sta_bwd preprocess launch");
+  CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, false, st), "sta_bwd dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dq(g, a, false, st), "sta_bwd dq launch");
+  return ok();
+}
+
+int vattn_dual_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* gvec,
+                   const void* o_l, const float* lse_l, const void* o_g, const float* lse_g, const void* kp,
+                   const void* vp, const void* dout, float scale, void* dq, void* dk, void* dv, float* dg,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(gvec);
+  REQUIRE_PTR(o_l);
+  REQUIRE_PTR(lse_l);
+  REQUIRE_PTR(o_g);
+  REQUIRE_PTR(lse_g);
+  REQUIRE_PTR(kp);
+  REQUIRE_PTR(vp);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  if (dg && !aligned16(dg)) return fail(VATTN_ERR_ALIGN, "dg is not 16-byte aligned");
+  const BwdWs w = bwd_ws(g, true);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.kp = kp;
+  a.vp = vp;
+  a.dout = dout;
+  a.o_l = o_l;
+  a.lse_l = lse_l;
+  a.o_g = o_g;
+  a.lse_g = lse_g;
+  a.g = gvec;
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.dg = dg;
+  uint8_t* ws = (uint8_t*)workspace;
+  a.delta_l = (float*)(ws + w.delta_l);
+  a.delta_g = (float*)(ws + w.delta_g);
+  a.dkp = (float*)(ws + w.dkp);
+  a.dvp = (float*)(ws + w.dvp);
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_bwd_preprocess(g, a, true, st), "dual_bwd preprocess launch");
+  CHECK_LAUNCH(launch_bwd_dkdv_global(g, a, st), "dual_bwd global dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, true, st), "dual_bwd local dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dq(g, a, true, st), "dual_bwd dq launch");
+  return ok();
+}
+
+}  // extern "C"

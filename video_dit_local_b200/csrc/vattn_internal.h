@@ -1,0 +1,93 @@
+// Internal declarations shared by the host entry points and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/vattn.h"
+
+namespace vattn {
+
+// Flattened, validated geometry handed to every kernel by value.
+struct DevGeom {
+  int B, heads, d;          // batch, heads, head_dim
+  int N, Np;                // tokens, pooled tokens
+  int T, H, W;
+  int tt, th, tw;           // tile
+  int wt, wh, ww;           // window (tiles)
+  int pt, ph, pw;           // pool
+  int Nt, Nh, Nw;           // tiles per dim
+  int s;                    // tile volume
+  int n_tiles, kept;        // tiles, kept tiles per query tile
+  int PT, PH, PW;           // pooled grid
+};
+
+// Runtime knobs shared by the attention kernels.
+struct DevCtl {
+  unsigned long long timeout_ns;
+  int* err_word;            // device status word (first writer wins)
+  int debug_flags;          // bit 0: skip the first producer arrival
+};
+
+DevCtl current_ctl();
+
+// -- reorder / pooling (reorder.cu) --
+cudaError_t launch_permute(const DevGeom& g, const void* src, void* dst, int64_t row_bytes, bool to_tiled,
+                           cudaStream_t st);
+cudaError_t launch_kept_tiles(const DevGeom& g, int32_t* out, cudaStream_t st);
+cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void* kp, void* vp, cudaStream_t st);
+
+// -- attention forward (attn_fwd.cu) --
+enum FwdMode { FWD_STA = 0, FWD_GLOBAL = 1 };
+struct FwdArgs {
+  const void* q;
+  const void* k;        // STA: K (tile-major, N rows); GLOBAL: K_p (Np rows)
+  const void* v;
+  void* o;              // bf16 out (may be NULL when blend_out is set and o_branch is not wanted)
+  float* lse;           // may be NULL
+  float scale;
+  // blend epilogue (GLOBAL only): out = g*o_local + (1-g)*this_branch
+  const void* o_local;  // NULL = no blend
+  const float* g;
+  void* blend_out;
+};
+cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
+
+// -- attention backward (attn_bwd.cu) --
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* kp;         // pooled K/V (dual only)
+  const void* vp;
+  const void* dout;
+  const void* o_l;        // local-branch output (or the STA output)
+  const float* lse_l;
+  const void* o_g;        // global-branch output (dual only)
+  const float* lse_g;
+  const float* g;         // blend factor per head, NULL = STA only (g = 1)
+  float scale;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dg;              // optional
+  // workspace pieces
+  float* delta_l;         // [B,h,N] rowsum(dO*O_l)
+  float* delta_g;         // [B,h,N] rowsum(dO*O_g)
+  float* dkp;             // [B,h,Np,d] fp32
+  float* dvp;
+};
+cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
+cudaError_t launch_bwd_dq(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
+cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
+cudaError_t launch_bwd_dkdv_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st);
+
+// TMA descriptor for a [rows_per_bh x bh] stack of rows of `d` bf16 elements,
+// box = 64 elements x box_rows rows x 1, 128-byte swizzle.  Returns false and
+// fills *err on failure.
+bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
+                    const char** err);
+
+}  // namespace vattn
