@@ -129,6 +129,31 @@ int vattn_dual_fwd(const vattn_geom* geom, const void* q, const void* k, const v
                    const float* g, float scale, void* o, void* o_l, float* lse_l, void* o_g,
                    float* lse_g, void* kp, void* vp, void* workspace, size_t ws_bytes, void* stream);
 
+/* Scratch held by the library for vattn_dual_fwd_noalloc (bytes). */
+#define VATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* Dual-branch inference forward that allocates nothing.  The pages have no
+ * counterpart: this entry point exists for callers that cannot call
+ * cudaMalloc (a plug-in inside a host framework whose memory pool has already
+ * reserved the device and offers no allocation hook; a latency-critical path
+ * that forbids allocation after start-up).  It computes what vattn_dual_fwd
+ * computes with all six saved outputs NULL, but takes the workspace from a
+ * static device array of VATTN_NOALLOC_SCRATCH_BYTES that every GPU which
+ * loads the library holds until the process exits.
+ *  - Geometries whose dual-forward workspace (vattn_workspace_size
+ *    (VATTN_OP_DUAL_FWD)) exceeds VATTN_NOALLOC_SCRATCH_BYTES are rejected
+ *    with VATTN_ERR_WORKSPACE before anything is launched.
+ *  - The first call on each device resolves the scratch's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one scratch array and it keeps the last
+ *    call's contents (nothing in it has to start at zero).  Calls whose work
+ *    overlaps on the GPU (other streams, other host threads) race on it:
+ *    serialise them.
+ * Arguments, layouts and errors are otherwise those of vattn_dual_fwd. */
+int vattn_dual_fwd_noalloc(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                           const float* g, float scale, void* o, void* stream);
+
 /* Sliding-tile attention backward.  Given q, k, v, the forward's o and lse
  * and the upstream gradient dout (all tile-major), writes dq, dk, dv (bf16,
  * tile-major).  dV = P^T dO, dP = dO V^T, dS = P*(dP - rowsum(dO*O)),

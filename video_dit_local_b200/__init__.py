@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     vattn_debug_set,
     vattn_dual_bwd,
     vattn_dual_fwd,
+    vattn_dual_fwd_noalloc,
     vattn_get_status,
     vattn_global_fwd,
     vattn_kept_tiles,

@@ -27,6 +27,7 @@ VATTN_ERR_WORKSPACE = -7
 VATTN_OP_DUAL_FWD = 1
 VATTN_OP_STA_BWD = 2
 VATTN_OP_DUAL_BWD = 3
+VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 class VattnError(RuntimeError):
@@ -77,6 +78,7 @@ _SIGS = {
     "vattn_dual_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_sta_bwd": [_GP, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
+    "vattn_dual_fwd_noalloc": [_GP, _P, _P, _P, _P, _F, _P, _P],
     "vattn_workspace_size": [_INT, _GP, ctypes.POINTER(_SZ)],
     "vattn_get_status": [_P],
     "vattn_last_error": [],
@@ -87,7 +89,7 @@ _SIGS = {
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m video_dit_local_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python video_dit_local_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for name, args in _SIGS.items():
         fn = getattr(lib, name)
@@ -160,6 +162,13 @@ def vattn_dual_fwd(geom: Geom, q, k, v, g, scale: float, o, o_l=None, lse_l=None
     _check(lib.vattn_dual_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), scale, _ptr(o), _ptr(o_l),
                               _ptr(lse_l), _ptr(o_g), _ptr(lse_g), _ptr(kp), _ptr(vp), _ptr(workspace), ws_bytes,
                               _stream(stream)))
+
+
+def vattn_dual_fwd_noalloc(geom: Geom, q, k, v, g, scale: float, o, stream=None) -> None:
+    """vattn_dual_fwd for callers that cannot allocate: the workspace is the
+    library's own static device scratch (VATTN_NOALLOC_SCRATCH_BYTES)."""
+    _check(lib.vattn_dual_fwd_noalloc(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), scale, _ptr(o),
+                                      _stream(stream)))
 
 
 def vattn_sta_bwd(geom: Geom, q, k, v, o, lse, dout, scale: float, dq, dk, dv, workspace, ws_bytes: int = 0,

@@ -48,6 +48,11 @@ static int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+int record_error(int code, const char* msg) {
+  t_last_error = msg ? msg : "";
+  return code;
+}
+
 static int ok() {
   t_last_error.clear();
   return VATTN_OK;

@@ -33,6 +33,9 @@ struct DevCtl {
 
 DevCtl current_ctl();
 
+// Records `msg` as this thread's last error and returns `code`.
+int record_error(int code, const char* msg);
+
 // -- reorder / pooling (reorder.cu) --
 cudaError_t launch_permute(const DevGeom& g, const void* src, void* dst, int64_t row_bytes, bool to_tiled,
                            cudaStream_t st);
