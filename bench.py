@@ -170,6 +170,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = S.WORKLOADS["720p"]
+    if args.heads and args.heads != w.heads:   # reduced case for profiling only
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads)
     geom = _geom(V, w)
     scale = 1.0 / math.sqrt(w.head_dim)
     flops_local, _ = _flops_fwd(w)
@@ -277,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, per-head U(0.5,2) scale)",
-        "config": {"workload": "720p sliding-tile fwd: B1 h24 d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
+        "config": {"workload": f"720p sliding-tile fwd: B1 h{w.heads} d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
                    "global_batch": w.batch * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (2.1 GB Q/K/V), no flush",
                    "step": "permute Q,K,V + sta_fwd + unpermute O,LSE"},
@@ -406,7 +409,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) bf16, per-head U(0.5,2) scale)",
-            "config": {"workload": "720p sliding-tile fwd: B1 h24 d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
+            "config": {"workload": f"720p sliding-tile fwd: B1 h{w.heads} d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
                        "sample": sample},
             "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -422,6 +425,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=0, help="profiling only: fewer heads than the workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -1,6 +1,6 @@
 """Builds libvattn.so (sm_100a) in-tree with nvcc.
 
-    python -m video_dit_local_b200.build [--debug]
+    python video_dit_local_b200/build.py [-v]
 
 Each .cu file under csrc/ is compiled to an object in parallel, then linked
 into video_dit_local_b200/libvattn.so (cudart linked statically, no libcuda
