@@ -338,7 +338,64 @@ def run_extras(V, dev):
                                    "status": V.vattn_get_status()}
         del q, k, v, o, ws
         torch.cuda.empty_cache()
+    out["train_fwd_bwd"] = _bench_train(V, dev, peaks)
     return out
+
+
+def _bench_train(V, dev, peaks):
+    """Training workload (B2 h24 d128, 1080p grid): dual forward with saved
+    outputs, then the dual backward; effective FLOPs 4d (fwd) + 10d (bwd) per
+    computed pair."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["train"]
+    geom = _geom(V, w)
+    T, H, W = w.grid
+    npool = (T // w.pool[0]) * (H // w.pool[1]) * (W // w.pool[2])
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 400 + i) for i in range(3))
+    do = _device_randn(shape, 404, std=0.1)
+    gvec = torch.rand(w.heads, device=dev)
+    scale = 1 / math.sqrt(w.head_dim)
+    o, o_l, o_g, dq, dk, dv = (torch.empty_like(q) for _ in range(6))
+    lse_l = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    lse_g = torch.empty_like(lse_l)
+    kp = torch.empty((w.batch, w.heads, npool, w.head_dim), dtype=torch.bfloat16, device=dev)
+    vp = torch.empty_like(kp)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, geom), dtype=torch.uint8, device=dev)
+    fl, fg = _flops_fwd(w)
+    bwd_flops = 2.5 * (fl + fg)
+
+    def fwd():
+        V.vattn_dual_fwd(geom, q, k, v, gvec, scale, o, o_l, lse_l, o_g, lse_g, kp, vp)
+
+    def bwd():
+        V.vattn_dual_bwd(geom, q, k, v, gvec, o_l, lse_l, o_g, lse_g, kp, vp, do, scale, dq, dk, dv, None, ws)
+    for _ in range(2):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    n = 3
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    tf = tb = 0.0
+    for _ in range(n):
+        ev[0].record()
+        fwd()
+        ev[1].record()
+        bwd()
+        ev[2].record()
+        torch.cuda.synchronize()
+        tf += ev[0].elapsed_time(ev[1])
+        tb += ev[1].elapsed_time(ev[2])
+    tf, tb = tf / n, tb / n
+    res = {"fwd_ms": round(tf, 3), "bwd_ms": round(tb, 3),
+           "fwd_eff_tflops": round((fl + fg) / tf / 1e9, 1), "bwd_eff_tflops": round(bwd_flops / tb / 1e9, 1),
+           "step_eff_tflops": round((fl + fg + bwd_flops) / (tf + tb) / 1e9, 1),
+           "step_frac": round((fl + fg + bwd_flops) / (tf + tb) / 1e9 / peaks["bf16_tflops"], 4),
+           "status": V.vattn_get_status()}
+    del q, k, v, do, o, o_l, o_g, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def cpu_baseline(budget_s: float):

@@ -405,3 +405,77 @@ def global_attention_rows(q, kp, vp, scale: float, rows):
     """Global branch for the listed raster query rows of one head."""
     o, lse, _ = _softmax_attend(q[np.asarray(rows)], kp, vp, scale)
     return o, lse
+
+
+def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_tiles, k_tiles, chunk: int = 8192):
+    """dual_backward for one head ([N, d] raster inputs) restricted to the
+    tokens of `q_tiles` (dQ) and of `k_tiles` (dK, dV).  Every softmax row it
+    uses is the full row of the definition; only the outputs are restricted.
+
+    Returns dict(q_ids, dQ, k_ids, dK, dV) with rows in the order of the ids.
+    """
+    nt, nh, nw = g.tiles_per_dim
+    gl, gg = float(gval), 1.0 - float(gval)
+
+    def window_ids(tid):
+        at, ah, aw = tile_coords_of(g, int(tid))
+        rt = window_range(at, g.window[0], nt)
+        rh = window_range(ah, g.window[1], nh)
+        rw = window_range(aw, g.window[2], nw)
+        qi = _tile_token_box(g, (at, ah, aw), (at + 1, ah + 1, aw + 1))
+        kj = _tile_token_box(g, (rt.start, rh.start, rw.start), (rt.stop, rh.stop, rw.stop))
+        return qi, kj
+
+    kp, vp = pool(k, g), pool(v, g)
+    # dQ rows: local branch of the query tile, global branch of the same rows
+    q_ids, dq_rows = [], []
+    for tid in q_tiles:
+        qi, kj = window_ids(tid)
+        dq_l, _, _ = _softmax_attend_bwd(q[qi], k[kj], v[kj], gl * do[qi], scale)
+        dq_g, _, _ = _softmax_attend_bwd(q[qi], kp, vp, gg * do[qi], scale)
+        q_ids.append(qi)
+        dq_rows.append(dq_l + dq_g)
+    # dK/dV rows, local branch: every query tile whose window holds the key tile
+    k_ids = [_tile_token_box(g, tile_coords_of(g, int(t)), tuple(c + 1 for c in tile_coords_of(g, int(t))))
+             for t in k_tiles]
+    want = np.concatenate(k_ids)
+    pos = {int(t): i for i, t in enumerate(want)}
+    dk = np.zeros((len(want), q.shape[1]))
+    dv = np.zeros_like(dk)
+    kept = kept_tiles(g)
+    wanted_tiles = set(int(t) for t in k_tiles)
+    for a in range(kept.shape[0]):
+        if not wanted_tiles.intersection(int(x) for x in kept[a]):
+            continue
+        qi, kj = window_ids(a)
+        _, dk_a, dv_a = _softmax_attend_bwd(q[qi], k[kj], v[kj], gl * do[qi], scale)
+        for col, tok in enumerate(kj):
+            r = pos.get(int(tok))
+            if r is not None:
+                dk[r] += dk_a[col]
+                dv[r] += dv_a[col]
+    # pooled branch: dK_p, dV_p at the pool blocks of the wanted tokens, summed
+    # over every query (row chunks of the full softmax)
+    u_all = pooled_index(g)
+    cols = np.unique(u_all[want])
+    dkp = np.zeros((len(cols), q.shape[1]))
+    dvp = np.zeros_like(dkp)
+    for r0 in range(0, g.n, chunk):
+        qc, doc = q[r0:r0 + chunk], gg * do[r0:r0 + chunk]
+        s = (qc @ kp.T) * scale
+        mx = s.max(axis=1, keepdims=True)
+        e = np.exp(s - mx)
+        p = e / e.sum(axis=1, keepdims=True)
+        dp = doc @ vp.T
+        row = (p * dp).sum(axis=1, keepdims=True)
+        pc = p[:, cols]
+        ds = pc * (dp[:, cols] - row)
+        dvp += pc.T @ doc
+        dkp += scale * (ds.T @ qc)
+    cidx = {int(c): i for i, c in enumerate(cols)}
+    cnt = g.pool[0] * g.pool[1] * g.pool[2]
+    for r, tok in enumerate(want):
+        c = cidx[int(u_all[tok])]
+        dk[r] += dkp[c] / cnt
+        dv[r] += dvp[c] / cnt
+    return dict(q_ids=np.concatenate(q_ids), dQ=np.concatenate(dq_rows), k_ids=want, dK=dk, dV=dv)

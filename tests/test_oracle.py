@@ -331,3 +331,22 @@ def test_pins_catch_transposed_tile_order(monkeypatch):
     with pytest.raises(AssertionError):
         test_permutation_matches_reshape_formulation(ODD)
     monkeypatch.setattr(O, "tile_major_index", orig)
+
+
+def test_sampled_evaluators_equal_full_definitions():
+    """The row-restricted helpers used for large grids agree with the full
+    definitions on a grid where both run."""
+    g = ODD
+    rng = np.random.default_rng(33)
+    q, k, v = (rng.standard_normal((1, 1, g.n, 8)) for _ in range(3))
+    do = rng.standard_normal((1, 1, g.n, 8))
+    full = O.dual_backward(q, k, v, [0.35], do, g, 0.4)
+    s = O.dual_backward_sampled(q[0, 0], k[0, 0], v[0, 0], 0.35, do[0, 0], g, 0.4, [0, 7, 44], [0, 13, 44], chunk=97)
+    assert np.abs(s["dQ"] - full["dQ"][0, 0][s["q_ids"]]).max() < 1e-12
+    assert np.abs(s["dK"] - full["dK"][0, 0][s["k_ids"]]).max() < 1e-12
+    assert np.abs(s["dV"] - full["dV"][0, 0][s["k_ids"]]).max() < 1e-12
+    fwd = O.dual_forward(q, k, v, [0.35], g, 0.4)
+    ids, ol, lsel = O.sta_attention_tiles(q[0, 0], k[0, 0], v[0, 0], g, 0.4, [3, 20])
+    assert np.abs(ol - fwd["O_l"][0, 0][ids]).max() < 1e-12 and np.abs(lsel - fwd["LSE_l"][0, 0][ids]).max() < 1e-12
+    og, lseg = O.global_attention_rows(q[0, 0], fwd["K_p"][0, 0], fwd["V_p"][0, 0], 0.4, ids)
+    assert np.abs(og - fwd["O_g"][0, 0][ids]).max() < 1e-12

@@ -1,11 +1,902 @@
-// Attention backward (placeholder until the tcgen05 backward kernels land).
+// Attention backward on tcgen05 tensor cores.
+//
+// Gradients of O = g*O_l + (1-g)*O_g ("UltraGen ..." §4.1) with the softmax
+// attention of each branch restated per branch b with weight gamma_b
+// (gamma_l = g, gamma_g = 1 - g; gamma = 1 for the sliding-tile backward):
+//   D_b   = rowsum(dO * O_b)
+//   P_b   = exp(S_b - LSE_b),  dP_b = dO V_b^T
+//   dS_b  = gamma_b * P_b * (dP_b - D_b)
+//   dV_b  = gamma_b * P_b^T dO,  dK_b = scale * dS_b^T Q,  dQ = scale * sum_b dS_b K_b
+// and the pooled branch's dK_p/dV_p flow back to every token of their pool
+// block divided by its size.
+//
+// Kernels:
+//   bwd_preprocess_kernel  D_l, D_g (and dg) from dO, O_l, O_g        HBM-bound
+//   dkdv_kernel<D>         one CTA per 128 keys; streams 64-query blocks:
+//                          GLOBAL  -> all queries vs pooled keys, fp32 dK_p/dV_p
+//                          LOCAL   -> the query tiles whose window holds the key
+//                                     tile ("inverse window"), pool-backward
+//                                     fused into the epilogue
+//   dq_kernel<D>           one CTA per 128 queries; streams 64-key blocks of the
+//                          kept window, then (dual) of all pooled keys
+// TMEM holds S/dP double-buffered per softmax group plus the accumulators;
+// P and dS are written back as bf16 over their own S/dP columns and read by
+// the next MMAs as the A operand.  No atomics: dQ, dK and dV are
+// deterministic.
 #include "common.cuh"
 
 namespace vattn {
 
-cudaError_t launch_bwd_preprocess(const DevGeom&, const BwdArgs&, bool, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_bwd_dq(const DevGeom&, const BwdArgs&, bool, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_bwd_dkdv_local(const DevGeom&, const BwdArgs&, bool, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_bwd_dkdv_global(const DevGeom&, const BwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace bwd {
+
+constexpr int NTHREADS = 352;
+constexpr int WARP_LOAD_A = 8;
+constexpr int WARP_LOAD_B = 9;
+constexpr int WARP_MMA = 10;
+constexpr float LOG2E = 1.4426950408889634f;
+
+// A row stream over a box of tiles (see TileBox) or a flat range.
+struct RowStream {
+  int runs, run_len, eh, t0, h0, w0;
+  bool tiled;
+  __device__ __forceinline__ int length() const { return runs * run_len; }
+  __device__ __forceinline__ int row(const DevGeom& g, int v) const {
+    if (!tiled) return v;
+    const int r = v / run_len, o = v - r * run_len;
+    const int kt = t0 + r / eh, kh = h0 + r % eh;
+    return ((kt * g.Nh + kh) * g.Nw + w0) * g.s + o;
+  }
+};
+
+__device__ __forceinline__ RowStream flat_stream(int n) {
+  RowStream s;
+  s.runs = 1;
+  s.run_len = n;
+  s.eh = 1;
+  s.t0 = s.h0 = s.w0 = 0;
+  s.tiled = false;
+  return s;
+}
+
+// key tiles kept by query tile q (its window)
+__device__ __forceinline__ RowStream window_stream(const DevGeom& g, int q) {
+  const int at = q / (g.Nh * g.Nw), ah = (q / g.Nw) % g.Nh, aw = q % g.Nw;
+  RowStream s;
+  s.t0 = win_start(at, g.wt, g.Nt);
+  s.h0 = win_start(ah, g.wh, g.Nh);
+  s.w0 = win_start(aw, g.ww, g.Nw);
+  s.eh = win_extent(g.wh, g.Nh);
+  s.runs = win_extent(g.wt, g.Nt) * s.eh;
+  s.run_len = win_extent(g.ww, g.Nw) * g.s;
+  s.tiled = true;
+  return s;
+}
+
+// query tiles whose window holds key tile k (the inverse window): per dim a
+// contiguous range, so again a box of tiles
+__device__ __forceinline__ RowStream inverse_stream(const DevGeom& g, int k) {
+  const int kt = k / (g.Nh * g.Nw), kh = (k / g.Nw) % g.Nh, kw = k % g.Nw;
+  int lt, ht, lh, hh, lw, hw;
+  inverse_range(kt, g.wt, g.Nt, &lt, &ht);
+  inverse_range(kh, g.wh, g.Nh, &lh, &hh);
+  inverse_range(kw, g.ww, g.Nw, &lw, &hw);
+  RowStream s;
+  s.t0 = lt;
+  s.h0 = lh;
+  s.w0 = lw;
+  s.eh = hh - lh + 1;
+  s.runs = (ht - lt + 1) * s.eh;
+  s.run_len = (hw - lw + 1) * g.s;
+  s.tiled = true;
+  return s;
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// pooled-raster index of the pool block holding tile-major token `tok`
+__device__ __forceinline__ int pooled_of_tiled(const DevGeom& g, int tok) {
+  const int tile = tok / g.s, l = tok - tile * g.s;
+  const int at = tile / (g.Nh * g.Nw), ah = (tile / g.Nw) % g.Nh, aw = tile % g.Nw;
+  const int lt = l / (g.th * g.tw), lh = (l / g.tw) % g.th, lw = l % g.tw;
+  const int t = at * g.tt + lt, y = ah * g.th + lh, x = aw * g.tw + lw;
+  return ((t / g.pt) * g.PH + y / g.ph) * g.PW + x / g.pw;
+}
+
+__device__ __forceinline__ float gamma_of(int mode, const float* gvec, int h) {
+  if (mode == 0) return 1.f;
+  const float gv = gvec[h];
+  return mode == 1 ? gv : 1.f - gv;
+}
+
+// ---------------------------------------------------------------------------
+// preprocess: D_l, D_g, dg
+// ---------------------------------------------------------------------------
+// grid (blocks_per_bh, B*heads); every group of vpr = d/8 lanes handles one row
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint4* __restrict__ dout,
+                                                              const uint4* __restrict__ o_l,
+                                                              const uint4* __restrict__ o_g,
+                                                              float* __restrict__ delta_l, float* __restrict__ delta_g,
+                                                              float* __restrict__ dg, int vpr, int N, int heads) {
+  const int bh = blockIdx.y;
+  const int groups = blockDim.x / vpr;
+  const int grp = threadIdx.x / vpr, lane_in = threadIdx.x % vpr;
+  float dg_acc = 0.f;
+  // the loop bound is uniform across the block, so every lane reaches the
+  // shuffles; rows past the end contribute zero
+  for (int rb = blockIdx.x * groups; rb < N; rb += gridDim.x * groups) {
+    const int r = rb + grp;
+    const bool in = r < N;
+    float sl = 0.f, sg = 0.f;
+    if (in) {
+      const size_t base = ((size_t)bh * N + r) * vpr + lane_in;
+      const uint4 a = __ldg(dout + base);
+      const uint4 b = __ldg(o_l + base);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sl += bf16lo(av[e]) * bf16lo(bv[e]) + bf16hi(av[e]) * bf16hi(bv[e]);
+      if (o_g) {
+        const uint4 c = __ldg(o_g + base);
+        const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sg += bf16lo(av[e]) * bf16lo(cv[e]) + bf16hi(av[e]) * bf16hi(cv[e]);
+      }
+    }
+    for (int o = vpr / 2; o > 0; o >>= 1) {
+      sl += __shfl_xor_sync(0xffffffffu, sl, o);
+      sg += __shfl_xor_sync(0xffffffffu, sg, o);
+    }
+    if (in && lane_in == 0) {
+      delta_l[(size_t)bh * N + r] = sl;
+      if (o_g) delta_g[(size_t)bh * N + r] = sg;
+      dg_acc += sl - sg;
+    }
+  }
+  if (dg) {
+    __shared__ float red[32];
+    for (int o = 16; o > 0; o >>= 1) dg_acc += __shfl_xor_sync(0xffffffffu, dg_acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dg_acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float t = 0.f;
+      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+      atomicAdd(&dg[bh % heads], t);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK / dV
+// ---------------------------------------------------------------------------
+enum { DKDV_LOCAL = 0, DKDV_GLOBAL = 1 };
+
+template <int D>
+struct DkdvSmem {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int KV_BYTES = CHUNKS * 128 * 128;  // 128 key rows
+  static constexpr int QB_BYTES = CHUNKS * 64 * 128;   // 64 query rows
+  static constexpr int NQ = 3;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = KV_BYTES;
+  static constexpr int OFF_Q = 2 * KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + NQ * QB_BYTES;
+  static constexpr int OFF_LSE = OFF_DO + NQ * QB_BYTES;
+  static constexpr int OFF_DEL = OFF_LSE + NQ * 256;
+  static constexpr int OFF_BAR = OFF_DEL + NQ * 256;
+  static constexpr int NBAR = 1 + 4 * NQ + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int TOTAL = OFF_MISC + 16;
+  static constexpr int ALLOC = TOTAL + 1024;
+};
+
+struct DkdvParams {
+  DevGeom g;
+  int mode;          // DKDV_LOCAL / DKDV_GLOBAL
+  int Gq;            // query sub-box rows (divides the tile volume, <= 64)
+  int kv_blocks_per_tile;
+  int Nk;            // key rows per batch*head (N or Np)
+  float c2;          // scale * log2(e)
+  float scale;
+  const float* lse;
+  const float* delta;
+  const float* gvec;
+  int gamma_mode;    // 0: 1, 1: g, 2: 1-g
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dkp_out;
+  float* dvp_out;
+  const float* dkp_in;   // pool-backward addend for LOCAL (NULL = none), already scaled
+  const float* dvp_in;
+  DevCtl ctl;
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                const DkdvParams p) {
+  using L = DkdvSmem<D>;
+  constexpr int NQ = L::NQ;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = q_full + NQ;
+  uint64_t* do_full = q_empty + NQ;
+  uint64_t* do_empty = do_full + NQ;
+  uint64_t* sdp_full = do_empty + NQ;
+  uint64_t* p_full = sdp_full + 2;
+  uint64_t* acc_done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  float* lse_s = reinterpret_cast<float*>(smem + L::OFF_LSE);
+  float* del_s = reinterpret_cast<float*>(smem + L::OFF_DEL);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int h = bh % p.g.heads;
+  const DevGeom& g = p.g;
+  WaitCtx wc;
+  wc.abort_flag = abort_flag;
+  wc.timeout_ns = p.ctl.timeout_ns;
+  wc.err_word = p.ctl.err_word;
+
+  int key_row0, key_valid;
+  RowStream qs;
+  if (p.mode == DKDV_LOCAL) {
+    const int kt = blockIdx.x / p.kv_blocks_per_tile;
+    const int sb = blockIdx.x - kt * p.kv_blocks_per_tile;
+    key_row0 = kt * g.s + sb * 128;
+    key_valid = min(128, g.s - sb * 128);
+    qs = inverse_stream(g, kt);
+  } else {
+    key_row0 = blockIdx.x * 128;
+    key_valid = min(128, p.Nk - key_row0);
+    qs = flat_stream(g.N);
+  }
+  const int Lq = qs.length();
+  const int nblk = (Lq + 63) / 64;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&do_full[i], 1);
+      mbar_init(&do_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sdp_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  constexpr uint32_t KBOX = 128 * 128;  // 128 rows x 128 bytes
+  constexpr uint32_t QBOX = 64 * 128;   // 64 rows x 128 bytes
+  const int subs = 64 / p.Gq;
+
+  if (warp == WARP_LOAD_A || warp == WARP_LOAD_B) {
+    if (lane == 0) {
+      const bool is_a = warp == WARP_LOAD_A;  // A: K, V tiles, Q and LSE; B: dO and D
+      if (is_a) {
+        mbar_arrive_expect_tx(kv_full, 2 * L::KV_BYTES);
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          tma_load_3d(smem + L::OFF_K + c * KBOX, &tm_k, kv_full, c * 64, key_row0, bh);
+          tma_load_3d(smem + L::OFF_V + c * KBOX, &tm_v, kv_full, c * 64, key_row0, bh);
+        }
+      }
+      uint64_t* full = is_a ? q_full : do_full;
+      uint64_t* empty = is_a ? q_empty : do_empty;
+      const CUtensorMap* tm = is_a ? &tm_q : &tm_do;
+      const float* vec = is_a ? p.lse : p.delta;
+      float* vec_s = is_a ? lse_s : del_s;
+      const uint32_t off_x = is_a ? L::OFF_Q : L::OFF_DO;
+      int issued = 0;
+      for (int i = 0; i < nblk; ++i) {
+        const int s = i % NQ, r = i / NQ;
+        if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
+        // LSE / D rows: whole 16-byte groups by bulk copy, a ragged tail of
+        // fewer than 4 rows (only at the end of a flat query stream) by plain
+        // loads, written before the arrival that publishes the stage
+        uint32_t tx = L::QB_BYTES;
+        for (int u = 0; u < subs; ++u) {
+          const int v = i * 64 + u * p.Gq;
+          if (v >= Lq) break;
+          const int n = min(p.Gq, Lq - v), nb = n & ~3;
+          tx += nb * 4;
+          if (nb < n) {
+            const int row = qs.row(g, v);
+            for (int t = nb; t < n; ++t) vec_s[s * 64 + u * p.Gq + t] = vec[(size_t)bh * g.N + row + t];
+          }
+        }
+        mbar_arrive_expect_tx(&full[s], tx);
+        for (int u = 0; u < subs; ++u) {
+          const int v = i * 64 + u * p.Gq;
+          const bool ok = v < Lq;
+          const int row = ok ? qs.row(g, v) : g.N;
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_3d(smem + off_x + s * L::QB_BYTES + c * QBOX + u * p.Gq * 128, tm, &full[s], c * 64, row, bh);
+          if (ok) {
+            const int nb = min(p.Gq, Lq - v) & ~3;
+            if (nb > 0) bulk_load(vec_s + s * 64 + u * p.Gq, vec + (size_t)bh * g.N + row, nb * 4, &full[s]);
+          }
+        }
+        ++issued;
+      }
+      for (int i = issued - NQ < 0 ? 0 : issued - NQ; i < issued; ++i) mbar_wait_drain(&full[i % NQ], (i / NQ) & 1, wc);
+      if (is_a) mbar_wait_drain(kv_full, 0, wc);
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t k_base = smem_u32(smem + L::OFF_K), v_base = smem_u32(smem + L::OFF_V);
+      const uint32_t q_base = smem_u32(smem + L::OFF_Q), do_base = smem_u32(smem + L::OFF_DO);
+      bool ok = mbar_wait(kv_full, 0, wc);
+      auto issue_sdp = [&](int i) -> bool {
+        const int s = i % NQ, w = i & 1;
+        if (!mbar_wait(&q_full[s], (i / NQ) & 1, wc)) return false;
+        if (!mbar_wait(&do_full[s], (i / NQ) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t qb = q_base + s * L::QB_BYTES, db = do_base + s * L::QB_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2) * KBOX + (kk & 3) * 32, qo = (kk >> 2) * QBOX + (kk & 3) * 32;
+          mma_ss(tmem + w * 64, smem_desc_sw128(k_base + ko, 16, 1024), smem_desc_sw128(qb + qo, 16, 1024), IDESC_S,
+                 kk > 0);
+          mma_ss(tmem + 128 + w * 64, smem_desc_sw128(v_base + ko, 16, 1024), smem_desc_sw128(db + qo, 16, 1024),
+                 IDESC_S, kk > 0);
+        }
+        tc_commit(&sdp_full[w]);
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      if (ok && nblk > 1) ok = issue_sdp(1);
+      for (int i = 0; ok && i < nblk; ++i) {
+        const int w = i & 1, s = i % NQ;
+        if (!mbar_wait(&p_full[w], (i >> 1) & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t qb = q_base + s * L::QB_BYTES, db = do_base + s * L::QB_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // dV += P^T dO ; dK += dS^T Q   (B operands MN-major: LBO = next 64-column box)
+          mma_ts(tmem + 256, tmem + w * 64 + kk * 8, smem_desc_sw128(db + kk * 2048, QBOX, 1024), IDESC_ACC,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + 384, tmem + 128 + w * 64 + kk * 8, smem_desc_sw128(qb + kk * 2048, QBOX, 1024), IDESC_ACC,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&q_empty[s]);
+        tc_commit(&do_empty[s]);
+        if (i + 2 < nblk) ok = issue_sdp(i + 2);
+      }
+      tc_commit(acc_done);
+      mbar_wait_drain(acc_done, 0, wc);
+    }
+  } else {
+    // ---------------- softmax groups: row = key ----------------
+    const int w = warp >> 2, quad = warp & 3, row = quad * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 64);
+    const uint32_t tP = tmem + lane_addr + 128u + (uint32_t)(w * 64);
+    const float gam = gamma_of(p.gamma_mode, p.gvec, h);
+    bool ok = true;
+    for (int i = w; i < nblk; i += 2) {
+      const int it = i >> 1, s = i % NQ;
+      ok = mbar_wait(&sdp_full[w], it & 1, wc);
+      ok = ok && mbar_wait(&q_full[s], (i / NQ) & 1, wc);    // LSE rows in shared memory
+      ok = ok && mbar_wait(&do_full[s], (i / NQ) & 1, wc);   // D rows in shared memory
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[2][32], dv[2][32];
+      tmem_ld32(tS, sv[0]);
+      tmem_ld32(tS + 32, sv[1]);
+      tmem_ld32(tP, dv[0]);
+      tmem_ld32(tP + 32, dv[1]);
+      tmem_wait_ld();
+      const float* ls = lse_s + s * 64;
+      const float* ds_ = del_s + s * 64;
+      const int valid = Lq - i * 64;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int c0 = hh * 32 + 2 * c;
+          float pp[2], dd[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int cc = c0 + e;
+            const float pe = ex2(fmaf(__uint_as_float(sv[hh][2 * c + e]), p.c2, -ls[cc] * LOG2E));
+            const float de = pe * (__uint_as_float(dv[hh][2 * c + e]) - ds_[cc]);
+            const bool in = cc < valid;
+            pp[e] = in ? gam * pe : 0.f;
+            dd[e] = in ? gam * de : 0.f;
+          }
+          pk[c] = pack_bf16(pp[0], pp[1]);
+          dk[c] = pack_bf16(dd[0], dd[1]);
+        }
+        tmem_st16(tS + hh * 16, pk);
+        tmem_st16(tP + hh * 16, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[w]);
+    }
+    // ---------------- epilogue: group 0 writes dV, group 1 writes dK ----------------
+    if (ok && !*abort_flag) ok = mbar_wait(acc_done, 0, wc);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const bool row_ok = row < key_valid;
+      const uint32_t tAcc = tmem + lane_addr + (w == 0 ? 256u : 384u);
+      const float mul = (w == 0) ? 1.f : p.scale;
+      const size_t tok = (size_t)key_row0 + row;
+      if (p.mode == DKDV_GLOBAL) {
+        float* dst = (w == 0 ? p.dvp_out : p.dkp_out) + ((size_t)bh * p.Nk + tok) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t x[32];
+          tmem_ld32(tAcc + c0, x);
+          tmem_wait_ld();
+          if (row_ok) {
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              reinterpret_cast<float4*>(dst + c0)[v4] =
+                  make_float4(__uint_as_float(x[4 * v4]) * mul, __uint_as_float(x[4 * v4 + 1]) * mul,
+                              __uint_as_float(x[4 * v4 + 2]) * mul, __uint_as_float(x[4 * v4 + 3]) * mul);
+          }
+        }
+      } else {
+        const float* add = (w == 0) ? p.dvp_in : p.dkp_in;
+        const float* add_row = nullptr;
+        float inv_cnt = 0.f;
+        if (add && row_ok) {
+          add_row = add + ((size_t)bh * g.Np + pooled_of_tiled(g, (int)tok)) * D;
+          inv_cnt = 1.f / (float)(g.pt * g.ph * g.pw);
+        }
+        __nv_bfloat16* dst = (w == 0 ? p.dv : p.dk) + ((size_t)bh * g.N + tok) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t x[32];
+          tmem_ld32(tAcc + c0, x);
+          tmem_wait_ld();
+          if (row_ok) {
+            float f[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(x[c]) * mul;
+            if (add_row) {
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(add_row + c0) + v4);
+                f[4 * v4] += a.x * inv_cnt;
+                f[4 * v4 + 1] += a.y * inv_cnt;
+                f[4 * v4 + 2] += a.z * inv_cnt;
+                f[4 * v4 + 3] += a.w * inv_cnt;
+              }
+            }
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              reinterpret_cast<uint4*>(dst + c0)[v4] =
+                  make_uint4(pack_bf16(f[8 * v4], f[8 * v4 + 1]), pack_bf16(f[8 * v4 + 2], f[8 * v4 + 3]),
+                             pack_bf16(f[8 * v4 + 4], f[8 * v4 + 5]), pack_bf16(f[8 * v4 + 6], f[8 * v4 + 7]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+template <int D>
+struct DqSmem {
+  static constexpr int CHUNKS = D / 64;
+  static constexpr int QB_BYTES = CHUNKS * 128 * 128;  // 128 query rows
+  static constexpr int KB_BYTES = CHUNKS * 64 * 128;   // 64 key rows
+  static constexpr int NK = 4;
+  static constexpr int NV = 4;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = QB_BYTES;
+  static constexpr int OFF_K = 2 * QB_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * KB_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NV * KB_BYTES;
+  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int TOTAL = OFF_MISC + 16;
+  static constexpr int ALLOC = TOTAL + 1024;
+};
+
+struct DqParams {
+  DevGeom g;
+  int dual;          // 0: local phase only (gamma = 1), 1: local (g) then global (1-g)
+  int G0;            // key sub-box rows of the local phase
+  int q_blocks_per_tile;
+  float c2;
+  float scale;
+  const float* lse_l;
+  const float* delta_l;
+  const float* lse_g;
+  const float* delta_g;
+  const float* gvec;
+  __nv_bfloat16* dq;
+  DevCtl ctl;
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ CUtensorMap tm_kp, const __grid_constant__ CUtensorMap tm_vp,
+              const DqParams p) {
+  using L = DqSmem<D>;
+  constexpr int NK = L::NK, NV = L::NV;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* qdo_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + NK;
+  uint64_t* v_full = k_empty + NK;
+  uint64_t* v_empty = v_full + NV;
+  uint64_t* sdp_full = v_empty + NV;
+  uint64_t* p_full = sdp_full + 2;
+  uint64_t* acc_done = p_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int h = bh % p.g.heads;
+  const DevGeom& g = p.g;
+  WaitCtx wc;
+  wc.abort_flag = abort_flag;
+  wc.timeout_ns = p.ctl.timeout_ns;
+  wc.err_word = p.ctl.err_word;
+
+  const int q_tile = blockIdx.x / p.q_blocks_per_tile;
+  const int sub = blockIdx.x - q_tile * p.q_blocks_per_tile;
+  const int q_row0 = q_tile * g.s + sub * 128;
+  const int q_valid = min(128, g.s - sub * 128);
+  const RowStream s0 = window_stream(g, q_tile);
+  const RowStream s1 = flat_stream(g.Np);
+  const int L0 = s0.length(), L1 = p.dual ? s1.length() : 0;
+  const int nb0 = (L0 + 63) / 64, nb1 = (L1 + 63) / 64;
+  const int nblk = nb0 + nb1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qdo_full, 1);
+    for (int i = 0; i < NK; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sdp_full[i], 1);
+      mbar_init(&p_full[i], 128);
+    }
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  constexpr uint32_t QBOX = 128 * 128;
+  constexpr uint32_t KBOX = 64 * 128;
+
+  if (warp == WARP_LOAD_A || warp == WARP_LOAD_B) {
+    if (lane == 0) {
+      const bool is_k = warp == WARP_LOAD_A;
+      if (is_k) {
+        mbar_arrive_expect_tx(qdo_full, 2 * L::QB_BYTES);
+        for (int c = 0; c < L::CHUNKS; ++c) {
+          tma_load_3d(smem + L::OFF_Q + c * QBOX, &tm_q, qdo_full, c * 64, q_row0, bh);
+          tma_load_3d(smem + L::OFF_DO + c * QBOX, &tm_do, qdo_full, c * 64, q_row0, bh);
+        }
+      }
+      const int NS = is_k ? NK : NV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const uint32_t off = is_k ? L::OFF_K : L::OFF_V;
+      int issued = 0;
+      for (int j = 0; j < nblk; ++j) {
+        const int s = j % NS, r = j / NS;
+        if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
+        mbar_arrive_expect_tx(&full[s], L::KB_BYTES);
+        const bool ph1 = j >= nb0;
+        const int jj = ph1 ? j - nb0 : j;
+        const int G = ph1 ? 64 : p.G0;
+        const int Lp = ph1 ? L1 : L0;
+        const CUtensorMap* tm = ph1 ? (is_k ? &tm_kp : &tm_vp) : (is_k ? &tm_k : &tm_v);
+        const int oob = ph1 ? g.Np : g.N;
+        for (int u = 0; u < 64 / G; ++u) {
+          const int v = jj * 64 + u * G;
+          const int row = v < Lp ? (ph1 ? s1.row(g, v) : s0.row(g, v)) : oob;
+          for (int c = 0; c < L::CHUNKS; ++c)
+            tma_load_3d(smem + off + s * L::KB_BYTES + c * KBOX + u * G * 128, tm, &full[s], c * 64, row, bh);
+        }
+        ++issued;
+      }
+      for (int j = issued - NS < 0 ? 0 : issued - NS; j < issued; ++j) mbar_wait_drain(&full[j % NS], (j / NS) & 1, wc);
+      if (is_k) mbar_wait_drain(qdo_full, 0, wc);
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q_base = smem_u32(smem + L::OFF_Q), do_base = smem_u32(smem + L::OFF_DO);
+      const uint32_t k_base = smem_u32(smem + L::OFF_K), v_base = smem_u32(smem + L::OFF_V);
+      bool ok = mbar_wait(qdo_full, 0, wc);
+      auto issue_sdp = [&](int j) -> bool {
+        const int w = j & 1, sk = j % NK, sv = j % NV;
+        if (!mbar_wait(&k_full[sk], (j / NK) & 1, wc)) return false;
+        if (!mbar_wait(&v_full[sv], (j / NV) & 1, wc)) return false;
+        tc_fence_after();
+        const uint32_t kb = k_base + sk * L::KB_BYTES, vb = v_base + sv * L::KB_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = (kk >> 2) * QBOX + (kk & 3) * 32, ko = (kk >> 2) * KBOX + (kk & 3) * 32;
+          mma_ss(tmem + w * 64, smem_desc_sw128(q_base + qo, 16, 1024), smem_desc_sw128(kb + ko, 16, 1024), IDESC_S,
+                 kk > 0);
+          mma_ss(tmem + 128 + w * 64, smem_desc_sw128(do_base + qo, 16, 1024), smem_desc_sw128(vb + ko, 16, 1024),
+                 IDESC_S, kk > 0);
+        }
+        tc_commit(&v_empty[sv]);
+        tc_commit(&sdp_full[w]);
+        return true;
+      };
+      if (ok && nblk > 0) ok = issue_sdp(0);
+      if (ok && nblk > 1) ok = issue_sdp(1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int w = j & 1, sk = j % NK;
+        if (!mbar_wait(&p_full[w], (j >> 1) & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t kb = k_base + sk * L::KB_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + 256, tmem + 128 + w * 64 + kk * 8, smem_desc_sw128(kb + kk * 2048, KBOX, 1024), IDESC_ACC,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&k_empty[sk]);
+        if (j + 2 < nblk) ok = issue_sdp(j + 2);
+      }
+      tc_commit(acc_done);
+      mbar_wait_drain(acc_done, 0, wc);
+    }
+  } else {
+    const int w = warp >> 2, quad = warp & 3, row = quad * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 64);
+    const uint32_t tP = tmem + lane_addr + 128u + (uint32_t)(w * 64);
+    const int qrow = min(q_row0 + row, g.N - 1);  // padding rows read a valid entry and are never stored
+    const size_t qi = (size_t)bh * g.N + qrow;
+    const float l2_l = p.lse_l[qi] * LOG2E, d_l = p.delta_l[qi];
+    const float l2_g = p.dual ? p.lse_g[qi] * LOG2E : 0.f, d_g = p.dual ? p.delta_g[qi] : 0.f;
+    const float gam_l = p.dual ? p.gvec[h] : 1.f, gam_g = 1.f - gam_l;
+    bool ok = true;
+    for (int j = w; j < nblk; j += 2) {
+      const int it = j >> 1;
+      ok = mbar_wait(&sdp_full[w], it & 1, wc);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[2][32], dv[2][32];
+      tmem_ld32(tS, sv[0]);
+      tmem_ld32(tS + 32, sv[1]);
+      tmem_ld32(tP, dv[0]);
+      tmem_ld32(tP + 32, dv[1]);
+      tmem_wait_ld();
+      const bool ph1 = j >= nb0;
+      const float l2 = ph1 ? l2_g : l2_l, dd = ph1 ? d_g : d_l, gam = ph1 ? gam_g : gam_l;
+      const int valid = ph1 ? L1 - (j - nb0) * 64 : L0 - j * 64;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t dk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float o2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int cc = hh * 32 + 2 * c + e;
+            const float pe = ex2(fmaf(__uint_as_float(sv[hh][2 * c + e]), p.c2, -l2));
+            const float de = gam * pe * (__uint_as_float(dv[hh][2 * c + e]) - dd);
+            o2[e] = cc < valid ? de : 0.f;
+          }
+          dk[c] = pack_bf16(o2[0], o2[1]);
+        }
+        tmem_st16(tP + hh * 16, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[w]);
+    }
+    if (ok && !*abort_flag) ok = mbar_wait(acc_done, 0, wc);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const bool row_ok = row < q_valid;
+      const uint32_t tAcc = tmem + lane_addr + 256u;
+      __nv_bfloat16* dst = p.dq + ((size_t)bh * g.N + q_row0 + row) * D;
+#pragma unroll 1
+      for (int c0 = (w * D) / 2; c0 < ((w + 1) * D) / 2; c0 += 32) {
+        uint32_t x[32];
+        tmem_ld32(tAcc + c0, x);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            reinterpret_cast<uint4*>(dst + c0)[v4] = make_uint4(
+                pack_bf16(__uint_as_float(x[8 * v4]) * p.scale, __uint_as_float(x[8 * v4 + 1]) * p.scale),
+                pack_bf16(__uint_as_float(x[8 * v4 + 2]) * p.scale, __uint_as_float(x[8 * v4 + 3]) * p.scale),
+                pack_bf16(__uint_as_float(x[8 * v4 + 4]) * p.scale, __uint_as_float(x[8 * v4 + 5]) * p.scale),
+                pack_bf16(__uint_as_float(x[8 * v4 + 6]) * p.scale, __uint_as_float(x[8 * v4 + 7]) * p.scale));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+static int pow2_rows(int s, int cap) {
+  int G = 1;
+  while (G < cap && s % (G * 2) == 0) G *= 2;
+  return G;
+}
+
+template <typename K>
+static cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D>
+static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global, bool dual, cudaStream_t st) {
+  DkdvParams p;
+  p.g = g;
+  p.mode = global ? DKDV_GLOBAL : DKDV_LOCAL;
+  p.Gq = global ? 64 : pow2_rows(g.s, 64);
+  p.kv_blocks_per_tile = (g.s + 127) / 128;
+  p.Nk = global ? g.Np : g.N;
+  p.scale = a.scale;
+  p.c2 = a.scale * LOG2E;
+  p.lse = global ? a.lse_g : a.lse_l;
+  p.delta = global ? a.delta_g : a.delta_l;
+  p.gvec = a.g;
+  p.gamma_mode = dual ? (global ? 2 : 1) : 0;
+  p.dk = (__nv_bfloat16*)a.dk;
+  p.dv = (__nv_bfloat16*)a.dv;
+  p.dkp_out = global ? a.dkp : nullptr;
+  p.dvp_out = global ? a.dvp : nullptr;
+  p.dkp_in = (!global && dual) ? a.dkp : nullptr;
+  p.dvp_in = (!global && dual) ? a.dvp : nullptr;
+  p.ctl = current_ctl();
+  const long long bh = (long long)g.B * g.heads;
+  const int blocks = global ? (g.Np + 127) / 128 : g.n_tiles * p.kv_blocks_per_tile;
+  if (bh == 0 || blocks == 0) return cudaSuccess;
+  CUtensorMap tk, tv, tq, tdo;
+  const char* err = nullptr;
+  const void* kp = global ? a.kp : a.k;
+  const void* vp = global ? a.vp : a.v;
+  if (!make_tmap_rows(&tk, kp, D, p.Nk, bh, 128, &err) || !make_tmap_rows(&tv, vp, D, p.Nk, bh, 128, &err) ||
+      !make_tmap_rows(&tq, a.q, D, g.N, bh, p.Gq, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, p.Gq, &err))
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_smem(dkdv_kernel<D>, DkdvSmem<D>::ALLOC);
+  if (e != cudaSuccess) return e;
+  dkdv_kernel<D><<<dim3(blocks, (unsigned)bh), NTHREADS, DkdvSmem<D>::ALLOC, st>>>(tk, tv, tq, tdo, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
+  DqParams p;
+  p.g = g;
+  p.dual = dual ? 1 : 0;
+  p.G0 = pow2_rows(g.s, 64);
+  p.q_blocks_per_tile = (g.s + 127) / 128;
+  p.scale = a.scale;
+  p.c2 = a.scale * LOG2E;
+  p.lse_l = a.lse_l;
+  p.delta_l = a.delta_l;
+  p.lse_g = a.lse_g;
+  p.delta_g = a.delta_g;
+  p.gvec = a.g;
+  p.dq = (__nv_bfloat16*)a.dq;
+  p.ctl = current_ctl();
+  const long long bh = (long long)g.B * g.heads;
+  const int blocks = g.n_tiles * p.q_blocks_per_tile;
+  if (bh == 0 || blocks == 0) return cudaSuccess;
+  CUtensorMap tq, tdo, tk, tv, tkp, tvp;
+  const char* err = nullptr;
+  if (!make_tmap_rows(&tq, a.q, D, g.N, bh, 128, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, 128, &err) ||
+      !make_tmap_rows(&tk, a.k, D, g.N, bh, p.G0, &err) || !make_tmap_rows(&tv, a.v, D, g.N, bh, p.G0, &err))
+    return cudaErrorInvalidValue;
+  if (dual) {
+    if (!make_tmap_rows(&tkp, a.kp, D, g.Np, bh, 64, &err) || !make_tmap_rows(&tvp, a.vp, D, g.Np, bh, 64, &err))
+      return cudaErrorInvalidValue;
+  } else {
+    tkp = tk;
+    tvp = tv;
+  }
+  cudaError_t e = set_smem(dq_kernel<D>, DqSmem<D>::ALLOC);
+  if (e != cudaSuccess) return e;
+  dq_kernel<D><<<dim3(blocks, (unsigned)bh), NTHREADS, DqSmem<D>::ALLOC, st>>>(tq, tdo, tk, tv, tkp, tvp, p);
+  return cudaGetLastError();
+}
+
+}  // namespace bwd
+
+cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
+  const long long bh = (long long)g.B * g.heads;
+  if (bh == 0 || g.N == 0) return cudaSuccess;
+  if (dual && a.dg) {
+    cudaError_t e = cudaMemsetAsync(a.dg, 0, sizeof(float) * g.heads, st);
+    if (e != cudaSuccess) return e;
+  }
+  const int vpr = g.d / 8;
+  const int rows_per_block = 256 / vpr;
+  int blocks = (g.N + rows_per_block - 1) / rows_per_block;
+  if (blocks > 64) blocks = 64;
+  bwd::bwd_preprocess_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>(
+      (const uint4*)a.dout, (const uint4*)a.o_l, dual ? (const uint4*)a.o_g : nullptr, a.delta_l,
+      dual ? a.delta_g : nullptr, dual ? a.dg : nullptr, vpr, g.N, g.heads);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st) {
+  if (g.d == 128) return bwd::launch_dkdv_d<128>(g, a, true, true, st);
+  if (g.d == 64) return bwd::launch_dkdv_d<64>(g, a, true, true, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
+  if (g.d == 128) return bwd::launch_dkdv_d<128>(g, a, false, dual, st);
+  if (g.d == 64) return bwd::launch_dkdv_d<64>(g, a, false, dual, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_dq(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
+  if (g.d == 128) return bwd::launch_dq_d<128>(g, a, dual, st);
+  if (g.d == 64) return bwd::launch_dq_d<64>(g, a, dual, st);
+  return cudaErrorInvalidValue;
+}
 
 }  // namespace vattn
