@@ -160,6 +160,29 @@ def _device_randn(shape, seed, std=1.0, scales=None):
     return x.to(torch.bfloat16)
 
 
+def run_train_only(args, rank, world, local_rank):
+    """Profiling mode: the training workload's fwd+bwd step alone (optionally
+    with fewer heads), timed with CUDA events."""
+    import dataclasses
+
+    import torch
+
+    import video_dit_local_b200 as V
+    from synth import inputs as S
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = S.WORKLOADS["train"]
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads)
+    peaks, _ = _peaks()
+    res = _bench_train(V, dev, peaks, w=w, n=args.steps, warm=args.warmup)
+    return {"metric": METRIC, "value": res["step_eff_tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["fwd_ms"] + res["bwd_ms"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch N(0,1))",
+            "config": {"workload": f"train dual fwd+bwd: B{w.batch} h{w.heads} d128, grid 21x72x120, tile 3x8x8, "
+                                   "window 3x3x3, pool 1x4x4"}, "train": res}
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -296,7 +319,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_extras:
+    if rank == 0 and world == 1 and not args.no_extras and args.workload == "720p":
         result["extras"] = run_extras(V, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
@@ -342,13 +365,13 @@ def run_extras(V, dev):
     return out
 
 
-def _bench_train(V, dev, peaks):
+def _bench_train(V, dev, peaks, w=None, n=3, warm=2):
     """Training workload (B2 h24 d128, 1080p grid): dual forward with saved
     outputs, then the dual backward; effective FLOPs 4d (fwd) + 10d (bwd) per
     computed pair."""
     import torch
     from synth import inputs as S
-    w = S.WORKLOADS["train"]
+    w = w or S.WORKLOADS["train"]
     geom = _geom(V, w)
     T, H, W = w.grid
     npool = (T // w.pool[0]) * (H // w.pool[1]) * (W // w.pool[2])
@@ -371,11 +394,10 @@ def _bench_train(V, dev, peaks):
 
     def bwd():
         V.vattn_dual_bwd(geom, q, k, v, gvec, o_l, lse_l, o_g, lse_g, kp, vp, do, scale, dq, dk, dv, None, ws)
-    for _ in range(2):
+    for _ in range(warm):
         fwd()
         bwd()
     torch.cuda.synchronize()
-    n = 3
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     tf = tb = 0.0
     for _ in range(n):
@@ -483,6 +505,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--heads", type=int, default=0, help="profiling only: fewer heads than the workload")
+    ap.add_argument("--workload", choices=["720p", "train"], default="720p",
+                    help="720p: the benchmark line; train: profiling of the training step alone")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -503,7 +527,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        result = run_ours(args, rank, world, local_rank)
+        if args.workload == "train":
+            result = run_train_only(args, rank, world, local_rank)
+        else:
+            result = run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:
