@@ -191,6 +191,11 @@ const char* vattn_last_error(void);
  * Affects calls made after it on any thread. */
 int vattn_debug_set(int flags, int64_t timeout_ns);
 
+/* Test hook: y[i] = the library's polynomial 2^x[i] (the one the attention
+ * forward uses for a quarter of its exponentials), for checking against
+ * CUDA's exp2f.  x, y: device float32 [n]. */
+int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream);
+
 /* Library version string. */
 const char* vattn_version(void);
 

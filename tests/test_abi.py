@@ -95,8 +95,9 @@ def test_workspace_sizes(V):
     def a(x):
         return (x + 255) // 256 * 256
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, g) == a(bh * n * d * 2) + 2 * a(bh * npool * d * 2)
-    assert V.vattn_workspace_size(V.VATTN_OP_STA_BWD, g) == a(bh * n * 4)
-    assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == 2 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)
+    assert V.vattn_workspace_size(V.VATTN_OP_STA_BWD, g) == 2 * a(bh * n * 4)
+    assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == (4 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)
+                                                              + a(bh * n * d * 4))
 
 
 def test_kernel_geometry_matches_oracle_inverse_ranges():

@@ -289,3 +289,21 @@ def test_device_timeout_is_reported_and_context_survives(V):
     check = [(0, 0), (0, 1)]
     o_r, lse_r = _sta_gpu(V, w, check)
     _check_sta(w, o_r, lse_r, check, range(8))
+
+
+def test_polynomial_exp2_against_cuda_exp2f(V):
+    """The FMA-pipe 2^x used for a quarter of the forward's exponentials
+    against CUDA's exp2f (torch.exp2): relative error <= 1e-4 on the range the
+    forward feeds it (x <= 8); at or below the clamp the result is tiny."""
+    import torch
+    x = torch.cat([torch.linspace(-124.0, 8.0, 1 << 20, device="cuda"),
+                   torch.rand(1 << 20, device="cuda") * 16 - 8]).contiguous()
+    y = torch.empty_like(x)
+    V.vattn_debug_exp2(x, y)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel <= 1e-4, rel
+    z = torch.tensor([-float("inf"), -1e30, -300.0, -126.0], device="cuda")
+    yz = torch.empty_like(z)
+    V.vattn_debug_exp2(z, yz)
+    assert (yz >= 0).all() and (yz <= 2.0 ** -124).all()

@@ -6,6 +6,7 @@ from .binding import (  # noqa: F401
     Geom,
     VattnError,
     make_geom,
+    vattn_debug_exp2,
     vattn_debug_set,
     vattn_dual_bwd,
     vattn_dual_fwd,

@@ -83,6 +83,7 @@ _SIGS = {
     "vattn_get_status": [_P],
     "vattn_last_error": [],
     "vattn_debug_set": [_INT, _I64],
+    "vattn_debug_exp2": [_P, _P, _I64, _P],
     "vattn_version": [],
 }
 
@@ -205,6 +206,10 @@ def vattn_last_error() -> str:
 
 def vattn_debug_set(flags: int, timeout_ns: int = 0) -> None:
     _check(lib.vattn_debug_set(flags, timeout_ns))
+
+
+def vattn_debug_exp2(x, y, n: Optional[int] = None, stream=None) -> None:
+    _check(lib.vattn_debug_exp2(_ptr(x), _ptr(y), x.numel() if n is None else n, _stream(stream)))
 
 
 def vattn_version() -> str:

@@ -108,56 +108,74 @@ __device__ __forceinline__ int pooled_of_tiled(const DevGeom& g, int tok) {
   return ((t / g.pt) * g.PH + y / g.ph) * g.PW + x / g.pw;
 }
 
-__device__ __forceinline__ float gamma_of(int mode, const float* gvec, int h) {
-  if (mode == 0) return 1.f;
-  const float gv = gvec[h];
-  return mode == 1 ? gv : 1.f - gv;
-}
-
 // ---------------------------------------------------------------------------
 // preprocess: D_l, D_g, dg
 // ---------------------------------------------------------------------------
-// grid (blocks_per_bh, B*heads); every group of vpr = d/8 lanes handles one row
-__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint4* __restrict__ dout,
-                                                              const uint4* __restrict__ o_l,
-                                                              const uint4* __restrict__ o_g,
-                                                              float* __restrict__ delta_l, float* __restrict__ delta_g,
-                                                              float* __restrict__ dg, int vpr, int N, int heads) {
+// grid (blocks_per_bh, B*heads); every group of vpr = d/8 lanes handles one row.
+// It writes the negated row terms -D_b and -L_b with
+// L_b = LSE_b*log2(e) - log2(gamma_b), so that the kernels form
+// gamma_b*P_b = exp2(S*scale*log2(e) - L_b) with one FMA and one ex2 and
+// dS_b = gamma_b*P_b*(dP_b - D_b) with one add and one multiply (gamma_b = 0
+// gives L_b = +inf and gamma_b*P_b = 0).
+struct PreArgs {
+  const uint4* dout;
+  const uint4* o_l;
+  const uint4* o_g;       // NULL: single branch
+  const float* lse_l;
+  const float* lse_g;
+  float* ndelta_l;
+  float* ndelta_g;
+  float* nlse2_l;
+  float* nlse2_g;
+  float* dg;              // NULL: skip
+  const float* gvec;      // NULL: gamma_l = 1
+  int vpr, N, heads;
+};
+
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const PreArgs a) {
   const int bh = blockIdx.y;
-  const int groups = blockDim.x / vpr;
-  const int grp = threadIdx.x / vpr, lane_in = threadIdx.x % vpr;
+  const int h = bh % a.heads;
+  const int groups = blockDim.x / a.vpr;
+  const int grp = threadIdx.x / a.vpr, lane_in = threadIdx.x % a.vpr;
+  const float gl = a.gvec ? a.gvec[h] : 1.f, gg = 1.f - gl;
+  const float off_l = __log2f(gl), off_g = __log2f(gg);
   float dg_acc = 0.f;
   // the loop bound is uniform across the block, so every lane reaches the
   // shuffles; rows past the end contribute zero
-  for (int rb = blockIdx.x * groups; rb < N; rb += gridDim.x * groups) {
+  for (int rb = blockIdx.x * groups; rb < a.N; rb += gridDim.x * groups) {
     const int r = rb + grp;
-    const bool in = r < N;
+    const bool in = r < a.N;
     float sl = 0.f, sg = 0.f;
     if (in) {
-      const size_t base = ((size_t)bh * N + r) * vpr + lane_in;
-      const uint4 a = __ldg(dout + base);
-      const uint4 b = __ldg(o_l + base);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+      const size_t base = ((size_t)bh * a.N + r) * a.vpr + lane_in;
+      const uint4 x = __ldg(a.dout + base);
+      const uint4 y = __ldg(a.o_l + base);
+      const uint32_t xv[4] = {x.x, x.y, x.z, x.w}, yv[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sl += bf16lo(av[e]) * bf16lo(bv[e]) + bf16hi(av[e]) * bf16hi(bv[e]);
-      if (o_g) {
-        const uint4 c = __ldg(o_g + base);
-        const uint32_t cv[4] = {c.x, c.y, c.z, c.w};
+      for (int e = 0; e < 4; ++e) sl += bf16lo(xv[e]) * bf16lo(yv[e]) + bf16hi(xv[e]) * bf16hi(yv[e]);
+      if (a.o_g) {
+        const uint4 z = __ldg(a.o_g + base);
+        const uint32_t zv[4] = {z.x, z.y, z.z, z.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sg += bf16lo(av[e]) * bf16lo(cv[e]) + bf16hi(av[e]) * bf16hi(cv[e]);
+        for (int e = 0; e < 4; ++e) sg += bf16lo(xv[e]) * bf16lo(zv[e]) + bf16hi(xv[e]) * bf16hi(zv[e]);
       }
     }
-    for (int o = vpr / 2; o > 0; o >>= 1) {
+    for (int o = a.vpr / 2; o > 0; o >>= 1) {
       sl += __shfl_xor_sync(0xffffffffu, sl, o);
       sg += __shfl_xor_sync(0xffffffffu, sg, o);
     }
     if (in && lane_in == 0) {
-      delta_l[(size_t)bh * N + r] = sl;
-      if (o_g) delta_g[(size_t)bh * N + r] = sg;
+      const size_t i = (size_t)bh * a.N + r;
+      a.ndelta_l[i] = -sl;
+      a.nlse2_l[i] = off_l - a.lse_l[i] * LOG2E;
+      if (a.o_g) {
+        a.ndelta_g[i] = -sg;
+        a.nlse2_g[i] = off_g - a.lse_g[i] * LOG2E;
+      }
       dg_acc += sl - sg;
     }
   }
-  if (dg) {
+  if (a.dg) {
     __shared__ float red[32];
     for (int o = 16; o > 0; o >>= 1) dg_acc += __shfl_xor_sync(0xffffffffu, dg_acc, o);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = dg_acc;
@@ -165,7 +183,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint4* __rest
     if (threadIdx.x == 0) {
       float t = 0.f;
       for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
-      atomicAdd(&dg[bh % heads], t);
+      atomicAdd(&a.dg[h], t);
     }
   }
 }
@@ -202,10 +220,8 @@ struct DkdvParams {
   int Nk;            // key rows per batch*head (N or Np)
   float c2;          // scale * log2(e)
   float scale;
-  const float* lse;
-  const float* delta;
-  const float* gvec;
-  int gamma_mode;    // 0: 1, 1: g, 2: 1-g
+  const float* nlse2;    // log2(gamma) - LSE*log2(e) per query row
+  const float* ndelta;   // -rowsum(dO*O)
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   float* dkp_out;
@@ -240,7 +256,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const int h = bh % p.g.heads;
   const DevGeom& g = p.g;
   WaitCtx wc;
   wc.abort_flag = abort_flag;
@@ -273,7 +288,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sdp_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
     }
     mbar_init(acc_done, 1);
     *abort_flag = 0;
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint64_t* full = is_a ? q_full : do_full;
       uint64_t* empty = is_a ? q_empty : do_empty;
       const CUtensorMap* tm = is_a ? &tm_q : &tm_do;
-      const float* vec = is_a ? p.lse : p.delta;
+      const float* vec = is_a ? p.nlse2 : p.ndelta;
       float* vec_s = is_a ? lse_s : del_s;
       const uint32_t off_x = is_a ? L::OFF_Q : L::OFF_DO;
       int issued = 0;
@@ -395,50 +410,55 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 64);
     const uint32_t tP = tmem + lane_addr + 128u + (uint32_t)(w * 64);
-    const float gam = gamma_of(p.gamma_mode, p.gvec, h);
     bool ok = true;
     for (int i = w; i < nblk; i += 2) {
       const int it = i >> 1, s = i % NQ;
       ok = mbar_wait(&sdp_full[w], it & 1, wc);
-      ok = ok && mbar_wait(&q_full[s], (i / NQ) & 1, wc);    // LSE rows in shared memory
+      ok = ok && mbar_wait(&q_full[s], (i / NQ) & 1, wc);    // L rows in shared memory
       ok = ok && mbar_wait(&do_full[s], (i / NQ) & 1, wc);   // D rows in shared memory
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[2][32], dv[2][32];
-      tmem_ld32(tS, sv[0]);
-      tmem_ld32(tS + 32, sv[1]);
-      tmem_ld32(tP, dv[0]);
-      tmem_ld32(tP + 32, dv[1]);
-      tmem_wait_ld();
-      const float* ls = lse_s + s * 64;
-      const float* ds_ = del_s + s * 64;
+      const float2 c2x2 = make_float2(p.c2, p.c2);
+      const float4* ls4 = reinterpret_cast<const float4*>(lse_s + s * 64);
+      const float4* ds4 = reinterpret_cast<const float4*>(del_s + s * 64);
+      const bool full_blk = Lq - i * 64 >= 64;   // uniform: only the last block is ragged
       const int valid = Lq - i * 64;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
+        // one 32-column half at a time keeps S, dP and the packed outputs in registers
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + hh * 32, sv);
+        tmem_ld32(tP + hh * 32, dv);
+        tmem_wait_ld();
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = hh * 32 + 2 * c;
-          float pp[2], dd[2];
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 l4 = ls4[hh * 8 + c4], d4 = ds4[hh * 8 + c4];  // -L, -D of four query columns
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int cc = c0 + e;
-            const float pe = ex2(fmaf(__uint_as_float(sv[hh][2 * c + e]), p.c2, -ls[cc] * LOG2E));
-            const float de = pe * (__uint_as_float(dv[hh][2 * c + e]) - ds_[cc]);
-            const bool in = cc < valid;
-            pp[e] = in ? gam * pe : 0.f;
-            dd[e] = in ? gam * de : 0.f;
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int c = c4 * 4 + e2 * 2;
+            const float2 nl = e2 ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
+            const float2 nd = e2 ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+            const float2 x = ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), c2x2, nl);
+            float2 pp = make_float2(ex2(x.x), ex2(x.y));
+            float2 dd = fmul2(pp, fadd2(make_float2(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])), nd));
+            if (!full_blk) {
+              const int cc = hh * 32 + c;
+              if (cc >= valid) pp.x = dd.x = 0.f;
+              if (cc + 1 >= valid) pp.y = dd.y = 0.f;
+            }
+            pk[c4 * 2 + e2] = pack_bf16(pp.x, pp.y);
+            dk[c4 * 2 + e2] = pack_bf16(dd.x, dd.y);
           }
-          pk[c] = pack_bf16(pp[0], pp[1]);
-          dk[c] = pack_bf16(dd[0], dd[1]);
         }
         tmem_st16(tS + hh * 16, pk);
         tmem_st16(tP + hh * 16, dk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[w]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[w]);
     }
     // ---------------- epilogue: group 0 writes dV, group 1 writes dK ----------------
     if (ok && !*abort_flag) ok = mbar_wait(acc_done, 0, wc);
@@ -532,19 +552,23 @@ struct DqSmem {
   static constexpr int ALLOC = TOTAL + 1024;
 };
 
+// Two launches make dQ: GLOBAL (dense 128-row query blocks against all pooled
+// keys, fp32 result to a workspace) and LOCAL (query blocks inside one query
+// tile against its kept window; adds the GLOBAL part and writes bf16 dQ).
+enum { DQ_LOCAL = 0, DQ_GLOBAL = 1 };
+
 struct DqParams {
   DevGeom g;
-  int dual;          // 0: local phase only (gamma = 1), 1: local (g) then global (1-g)
-  int G0;            // key sub-box rows of the local phase
+  int mode;          // DQ_LOCAL / DQ_GLOBAL
+  int G0;            // key sub-box rows of the local stream
   int q_blocks_per_tile;
   float c2;
   float scale;
-  const float* lse_l;
-  const float* delta_l;
-  const float* lse_g;
-  const float* delta_g;
-  const float* gvec;
-  __nv_bfloat16* dq;
+  const float* nlse2;    // log2(gamma) - LSE*log2(e) of this branch
+  const float* ndelta;   // -rowsum(dO*O)
+  const float* acc_in;   // LOCAL: fp32 global-branch dQ to add (NULL = none)
+  float* acc_out;        // GLOBAL: fp32 output
+  __nv_bfloat16* dq;     // LOCAL: bf16 output
   DevCtl ctl;
 };
 
@@ -552,7 +576,6 @@ template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-              const __grid_constant__ CUtensorMap tm_kp, const __grid_constant__ CUtensorMap tm_vp,
               const DqParams p) {
   using L = DqSmem<D>;
   constexpr int NK = L::NK, NV = L::NV;
@@ -572,22 +595,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
-  const int h = bh % p.g.heads;
   const DevGeom& g = p.g;
   WaitCtx wc;
   wc.abort_flag = abort_flag;
   wc.timeout_ns = p.ctl.timeout_ns;
   wc.err_word = p.ctl.err_word;
 
-  const int q_tile = blockIdx.x / p.q_blocks_per_tile;
-  const int sub = blockIdx.x - q_tile * p.q_blocks_per_tile;
-  const int q_row0 = q_tile * g.s + sub * 128;
-  const int q_valid = min(128, g.s - sub * 128);
-  const RowStream s0 = window_stream(g, q_tile);
-  const RowStream s1 = flat_stream(g.Np);
-  const int L0 = s0.length(), L1 = p.dual ? s1.length() : 0;
-  const int nb0 = (L0 + 63) / 64, nb1 = (L1 + 63) / 64;
-  const int nblk = nb0 + nb1;
+  const bool glob = p.mode == DQ_GLOBAL;
+  int q_row0, q_valid, q_tile = 0;
+  if (glob) {
+    q_row0 = blockIdx.x * 128;
+    q_valid = min(128, g.N - q_row0);
+  } else {
+    q_tile = blockIdx.x / p.q_blocks_per_tile;
+    const int sub = blockIdx.x - q_tile * p.q_blocks_per_tile;
+    q_row0 = q_tile * g.s + sub * 128;
+    q_valid = min(128, g.s - sub * 128);
+  }
+  const RowStream ks = glob ? flat_stream(g.Np) : window_stream(g, q_tile);
+  const int Lk = ks.length();
+  const int nblk = (Lk + 63) / 64;
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
@@ -601,7 +628,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sdp_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
     }
     mbar_init(acc_done, 1);
     *abort_flag = 0;
@@ -638,15 +665,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = j % NS, r = j / NS;
         if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
         mbar_arrive_expect_tx(&full[s], L::KB_BYTES);
-        const bool ph1 = j >= nb0;
-        const int jj = ph1 ? j - nb0 : j;
-        const int G = ph1 ? 64 : p.G0;
-        const int Lp = ph1 ? L1 : L0;
-        const CUtensorMap* tm = ph1 ? (is_k ? &tm_kp : &tm_vp) : (is_k ? &tm_k : &tm_v);
-        const int oob = ph1 ? g.Np : g.N;
+        const int G = glob ? 64 : p.G0;
+        const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+        const int oob = glob ? g.Np : g.N;
         for (int u = 0; u < 64 / G; ++u) {
-          const int v = jj * 64 + u * G;
-          const int row = v < Lp ? (ph1 ? s1.row(g, v) : s0.row(g, v)) : oob;
+          const int v = j * 64 + u * G;
+          const int row = v < Lk ? ks.row(g, v) : oob;
           for (int c = 0; c < L::CHUNKS; ++c)
             tma_load_3d(smem + off + s * L::KB_BYTES + c * KBOX + u * G * 128, tm, &full[s], c * 64, row, bh);
         }
@@ -704,9 +728,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tP = tmem + lane_addr + 128u + (uint32_t)(w * 64);
     const int qrow = min(q_row0 + row, g.N - 1);  // padding rows read a valid entry and are never stored
     const size_t qi = (size_t)bh * g.N + qrow;
-    const float l2_l = p.lse_l[qi] * LOG2E, d_l = p.delta_l[qi];
-    const float l2_g = p.dual ? p.lse_g[qi] * LOG2E : 0.f, d_g = p.dual ? p.delta_g[qi] : 0.f;
-    const float gam_l = p.dual ? p.gvec[h] : 1.f, gam_g = 1.f - gam_l;
+    const float2 nl2 = make_float2(p.nlse2[qi], p.nlse2[qi]), nd2 = make_float2(p.ndelta[qi], p.ndelta[qi]);
+    const float2 c2x2 = make_float2(p.c2, p.c2);
     bool ok = true;
     for (int j = w; j < nblk; j += 2) {
       const int it = j >> 1;
@@ -720,29 +743,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_ld32(tP, dv[0]);
       tmem_ld32(tP + 32, dv[1]);
       tmem_wait_ld();
-      const bool ph1 = j >= nb0;
-      const float l2 = ph1 ? l2_g : l2_l, dd = ph1 ? d_g : d_l, gam = ph1 ? gam_g : gam_l;
-      const int valid = ph1 ? L1 - (j - nb0) * 64 : L0 - j * 64;
+      const int valid = Lk - j * 64;
+      const bool full_blk = valid >= 64;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t dk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float o2[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int cc = hh * 32 + 2 * c + e;
-            const float pe = ex2(fmaf(__uint_as_float(sv[hh][2 * c + e]), p.c2, -l2));
-            const float de = gam * pe * (__uint_as_float(dv[hh][2 * c + e]) - dd);
-            o2[e] = cc < valid ? de : 0.f;
+          const float2 x =
+              ffma2(make_float2(__uint_as_float(sv[hh][2 * c]), __uint_as_float(sv[hh][2 * c + 1])), c2x2, nl2);
+          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+          float2 o2 =
+              fmul2(pp, fadd2(make_float2(__uint_as_float(dv[hh][2 * c]), __uint_as_float(dv[hh][2 * c + 1])), nd2));
+          if (!full_blk) {
+            const int cc = hh * 32 + 2 * c;
+            if (cc >= valid) o2.x = 0.f;
+            if (cc + 1 >= valid) o2.y = 0.f;
           }
-          dk[c] = pack_bf16(o2[0], o2[1]);
+          dk[c] = pack_bf16(o2.x, o2.y);
         }
         tmem_st16(tP + hh * 16, dk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[w]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[w]);
     }
     if (ok && !*abort_flag) ok = mbar_wait(acc_done, 0, wc);
     ok = __all_sync(0xffffffffu, ok);
@@ -750,20 +775,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok && !*abort_flag) {
       const bool row_ok = row < q_valid;
       const uint32_t tAcc = tmem + lane_addr + 256u;
-      __nv_bfloat16* dst = p.dq + ((size_t)bh * g.N + q_row0 + row) * D;
+      const size_t grow = (size_t)bh * g.N + q_row0 + row;
 #pragma unroll 1
       for (int c0 = (w * D) / 2; c0 < ((w + 1) * D) / 2; c0 += 32) {
         uint32_t x[32];
         tmem_ld32(tAcc + c0, x);
         tmem_wait_ld();
         if (row_ok) {
+          float f[32];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            reinterpret_cast<uint4*>(dst + c0)[v4] = make_uint4(
-                pack_bf16(__uint_as_float(x[8 * v4]) * p.scale, __uint_as_float(x[8 * v4 + 1]) * p.scale),
-                pack_bf16(__uint_as_float(x[8 * v4 + 2]) * p.scale, __uint_as_float(x[8 * v4 + 3]) * p.scale),
-                pack_bf16(__uint_as_float(x[8 * v4 + 4]) * p.scale, __uint_as_float(x[8 * v4 + 5]) * p.scale),
-                pack_bf16(__uint_as_float(x[8 * v4 + 6]) * p.scale, __uint_as_float(x[8 * v4 + 7]) * p.scale));
+          for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(x[c]) * p.scale;
+          if (glob) {
+            float4* dst = reinterpret_cast<float4*>(p.acc_out + grow * D + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(f[4 * v4], f[4 * v4 + 1], f[4 * v4 + 2], f[4 * v4 + 3]);
+          } else {
+            if (p.acc_in) {
+              const float4* src = reinterpret_cast<const float4*>(p.acc_in + grow * D + c0);
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4) {
+                const float4 a4 = __ldg(src + v4);
+                f[4 * v4] += a4.x;
+                f[4 * v4 + 1] += a4.y;
+                f[4 * v4 + 2] += a4.z;
+                f[4 * v4 + 3] += a4.w;
+              }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * D + c0);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pack_bf16(f[8 * v4], f[8 * v4 + 1]), pack_bf16(f[8 * v4 + 2], f[8 * v4 + 3]),
+                                   pack_bf16(f[8 * v4 + 4], f[8 * v4 + 5]), pack_bf16(f[8 * v4 + 6], f[8 * v4 + 7]));
+          }
         }
       }
     }
@@ -798,10 +841,8 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   p.Nk = global ? g.Np : g.N;
   p.scale = a.scale;
   p.c2 = a.scale * LOG2E;
-  p.lse = global ? a.lse_g : a.lse_l;
-  p.delta = global ? a.delta_g : a.delta_l;
-  p.gvec = a.g;
-  p.gamma_mode = dual ? (global ? 2 : 1) : 0;
+  p.nlse2 = global ? a.nlse2_g : a.nlse2_l;
+  p.ndelta = global ? a.ndelta_g : a.ndelta_l;
   p.dk = (__nv_bfloat16*)a.dk;
   p.dv = (__nv_bfloat16*)a.dv;
   p.dkp_out = global ? a.dkp : nullptr;
@@ -826,39 +867,35 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
 }
 
 template <int D>
-static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
+static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, bool add_acc, cudaStream_t st) {
   DqParams p;
   p.g = g;
-  p.dual = dual ? 1 : 0;
+  p.mode = global ? DQ_GLOBAL : DQ_LOCAL;
   p.G0 = pow2_rows(g.s, 64);
   p.q_blocks_per_tile = (g.s + 127) / 128;
   p.scale = a.scale;
   p.c2 = a.scale * LOG2E;
-  p.lse_l = a.lse_l;
-  p.delta_l = a.delta_l;
-  p.lse_g = a.lse_g;
-  p.delta_g = a.delta_g;
-  p.gvec = a.g;
+  p.nlse2 = global ? a.nlse2_g : a.nlse2_l;
+  p.ndelta = global ? a.ndelta_g : a.ndelta_l;
+  p.acc_in = (!global && add_acc) ? a.dq_acc : nullptr;
+  p.acc_out = global ? a.dq_acc : nullptr;
   p.dq = (__nv_bfloat16*)a.dq;
   p.ctl = current_ctl();
   const long long bh = (long long)g.B * g.heads;
-  const int blocks = g.n_tiles * p.q_blocks_per_tile;
+  const int blocks = global ? (g.N + 127) / 128 : g.n_tiles * p.q_blocks_per_tile;
   if (bh == 0 || blocks == 0) return cudaSuccess;
-  CUtensorMap tq, tdo, tk, tv, tkp, tvp;
+  CUtensorMap tq, tdo, tk, tv;
   const char* err = nullptr;
+  const void* kk = global ? a.kp : a.k;
+  const void* vv = global ? a.vp : a.v;
+  const long long nk = global ? g.Np : g.N;
+  const int G = global ? 64 : p.G0;
   if (!make_tmap_rows(&tq, a.q, D, g.N, bh, 128, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, 128, &err) ||
-      !make_tmap_rows(&tk, a.k, D, g.N, bh, p.G0, &err) || !make_tmap_rows(&tv, a.v, D, g.N, bh, p.G0, &err))
+      !make_tmap_rows(&tk, kk, D, nk, bh, G, &err) || !make_tmap_rows(&tv, vv, D, nk, bh, G, &err))
     return cudaErrorInvalidValue;
-  if (dual) {
-    if (!make_tmap_rows(&tkp, a.kp, D, g.Np, bh, 64, &err) || !make_tmap_rows(&tvp, a.vp, D, g.Np, bh, 64, &err))
-      return cudaErrorInvalidValue;
-  } else {
-    tkp = tk;
-    tvp = tv;
-  }
   cudaError_t e = set_smem(dq_kernel<D>, DqSmem<D>::ALLOC);
   if (e != cudaSuccess) return e;
-  dq_kernel<D><<<dim3(blocks, (unsigned)bh), NTHREADS, DqSmem<D>::ALLOC, st>>>(tq, tdo, tk, tv, tkp, tvp, p);
+  dq_kernel<D><<<dim3(blocks, (unsigned)bh), NTHREADS, DqSmem<D>::ALLOC, st>>>(tq, tdo, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -871,13 +908,25 @@ cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual,
     cudaError_t e = cudaMemsetAsync(a.dg, 0, sizeof(float) * g.heads, st);
     if (e != cudaSuccess) return e;
   }
-  const int vpr = g.d / 8;
-  const int rows_per_block = 256 / vpr;
+  bwd::PreArgs pa;
+  pa.dout = (const uint4*)a.dout;
+  pa.o_l = (const uint4*)a.o_l;
+  pa.o_g = dual ? (const uint4*)a.o_g : nullptr;
+  pa.lse_l = a.lse_l;
+  pa.lse_g = dual ? a.lse_g : nullptr;
+  pa.ndelta_l = a.ndelta_l;
+  pa.ndelta_g = dual ? a.ndelta_g : nullptr;
+  pa.nlse2_l = a.nlse2_l;
+  pa.nlse2_g = dual ? a.nlse2_g : nullptr;
+  pa.dg = dual ? a.dg : nullptr;
+  pa.gvec = dual ? a.g : nullptr;
+  pa.vpr = g.d / 8;
+  pa.N = g.N;
+  pa.heads = g.heads;
+  const int rows_per_block = 256 / pa.vpr;
   int blocks = (g.N + rows_per_block - 1) / rows_per_block;
   if (blocks > 64) blocks = 64;
-  bwd::bwd_preprocess_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>(
-      (const uint4*)a.dout, (const uint4*)a.o_l, dual ? (const uint4*)a.o_g : nullptr, a.delta_l,
-      dual ? a.delta_g : nullptr, dual ? a.dg : nullptr, vpr, g.N, g.heads);
+  bwd::bwd_preprocess_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>(pa);
   return cudaGetLastError();
 }
 
@@ -893,9 +942,15 @@ cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual,
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_bwd_dq_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st) {
+  if (g.d == 128) return bwd::launch_dq_d<128>(g, a, true, false, st);
+  if (g.d == 64) return bwd::launch_dq_d<64>(g, a, true, false, st);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_bwd_dq(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
-  if (g.d == 128) return bwd::launch_dq_d<128>(g, a, dual, st);
-  if (g.d == 64) return bwd::launch_dq_d<64>(g, a, dual, st);
+  if (g.d == 128) return bwd::launch_dq_d<128>(g, a, false, dual, st);
+  if (g.d == 64) return bwd::launch_dq_d<64>(g, a, false, dual, st);
   return cudaErrorInvalidValue;
 }
 

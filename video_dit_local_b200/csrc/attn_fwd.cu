@@ -32,6 +32,14 @@ constexpr int WARP_MMA = 10;
 constexpr int NK = 3;  // K ring stages
 constexpr int NV = 2;  // V ring stages
 constexpr float RESCALE_LOG2_THRESHOLD = 8.0f;
+// 32-column chunk (of 4) whose exp2 runs on the FMA pipe (exp2_poly) instead
+// of the MUFU unit; -1 = none.  Measured on B200 at 720p: the MUFU unit is
+// not the limiter of this kernel (removing every ex2 leaves the time
+// unchanged), so the default keeps all exponentials on the MUFU unit.
+#ifndef VATTN_POLY_CHUNK
+#define VATTN_POLY_CHUNK -1
+#endif
+constexpr int POLY_CHUNK = VATTN_POLY_CHUNK;
 
 template <int D>
 struct Smem {
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
     }
     mbar_init(o_final, 1);
     *abort_flag = 0;
@@ -305,11 +313,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int c = 0; c < 32; ++c)
             if (q4 * 32 + c >= valid) sr[q4][c] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // row max: four independent chains of three-input max
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sr[q4][c]));
+        for (int c = 0; c < 32; c += 2)
+          m4[(c >> 1) & 3] = fmax3(m4[(c >> 1) & 3], __uint_as_float(sr[q4][c]), __uint_as_float(sr[q4][c + 1]));
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mx2 = mx * c2;
       bool need = false;
       if (i == 0) {
@@ -323,21 +334,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         m_ref = mx2;
         l_sum *= alpha;
       }
-      const float neg_m = -m_ref;
-      float sum = 0.f;
+      // P = 2^(S*scale*log2(e) - m) two lanes at a time (packed fp32x2)
+      const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(-m_ref, -m_ref);
+      float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[q4][2 * c]), c2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[q4][2 * c + 1]), c2, neg_m));
-          sum += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(sr[q4][2 * c]), __uint_as_float(sr[q4][2 * c + 1])),
+                                 c2x2, negm2);
+          float2 pp;
+          if (q4 == POLY_CHUNK) {  // FMA-pipe exponentials for this chunk (see POLY_CHUNK)
+            pp.x = exp2_poly(x.x);
+            pp.y = exp2_poly(x.y);
+          } else {
+            pp.x = ex2(x.x);
+            pp.y = ex2(x.y);
+          }
+          s2[c & 1] = fadd2(s2[c & 1], pp);
+          pk[c] = pack_bf16(pp.x, pp.y);
         }
         tmem_st16(tS + q4 * 16, pk);
       }
-      l_sum += sum;
+      l_sum += (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
       if (__any_sync(0xffffffffu, need)) {
         // O of this group is quiescent: the commit that signalled this S also
         // covers the previous P*V into it, and the next one waits for p_full.
@@ -353,7 +373,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[w]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[w]);
     }
     // ---------------- epilogue ----------------
     if (ok && !*abort_flag) ok = mbar_wait(o_final, 0, wc);
@@ -461,15 +482,24 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   if (!make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) || !make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err) ||
       !make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err))
     return cudaErrorInvalidValue;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Smem<D>::ALLOC);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Smem<D>::ALLOC);
+  if (e != cudaSuccess) return e;
   dim3 grid(qblocks, (unsigned)bh);
   attn_fwd_kernel<D><<<grid, NTHREADS, Smem<D>::ALLOC, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    y[i] = exp2_poly(x[i]);
+}
+
+cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  exp2_poly_kernel<<<(int)blocks, 256, 0, st>>>(x, y, n);
   return cudaGetLastError();
 }
 

@@ -190,21 +190,27 @@ static DualFwdWs dual_fwd_ws(const DevGeom& g) {
   w.total = w.vp + align256(bh * g.Np * g.d * 2);
   return w;
 }
+// Backward workspace: per-row D and prescaled LSE for each branch, the pooled
+// branch's fp32 dK_p/dV_p, and the fp32 global-branch part of dQ.
 struct BwdWs {
-  size_t delta_l, delta_g, dkp, dvp, total;
+  size_t ndelta_l, nlse2_l, ndelta_g, nlse2_g, dkp, dvp, dq_acc, total;
 };
 static BwdWs bwd_ws(const DevGeom& g, bool dual) {
   BwdWs w;
   const size_t bh = (size_t)g.B * g.heads;
-  w.delta_l = 0;
-  w.delta_g = align256(bh * g.N * 4);
+  const size_t row = align256(bh * g.N * 4);
+  w.ndelta_l = 0;
+  w.nlse2_l = row;
   if (!dual) {
-    w.dkp = w.dvp = w.total = w.delta_g;
+    w.ndelta_g = w.nlse2_g = w.dkp = w.dvp = w.dq_acc = w.total = 2 * row;
     return w;
   }
-  w.dkp = w.delta_g + align256(bh * g.N * 4);
+  w.ndelta_g = 2 * row;
+  w.nlse2_g = 3 * row;
+  w.dkp = 4 * row;
   w.dvp = w.dkp + align256(bh * g.Np * g.d * 4);
-  w.total = w.dvp + align256(bh * g.Np * g.d * 4);
+  w.dq_acc = w.dvp + align256(bh * g.Np * g.d * 4);
+  w.total = w.dq_acc + align256(bh * g.N * g.d * 4);
   return w;
 }
 
@@ -221,6 +227,15 @@ const char* vattn_last_error(void) { return t_last_error.c_str(); }
 int vattn_debug_set(int flags, int64_t timeout_ns) {
   s_debug_flags.store(flags);
   s_timeout_ns.store(timeout_ns > 0 ? (long long)timeout_ns : 2000000000ll);
+  return ok();
+}
+
+int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return fail(VATTN_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return ok();
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(y);
+  CHECK_LAUNCH(launch_exp2_poly(x, y, n, (cudaStream_t)stream), "debug_exp2 launch");
   return ok();
 }
 
@@ -437,7 +452,8 @@ int vattn_sta_bwd(const vattn_geom* geom, const void* q, const void* k, const vo
   a.dq = dq;
   a.dk = dk;
   a.dv = dv;
-  a.delta_l = (float*)((uint8_t*)workspace + w.delta_l);
+  a.ndelta_l = (float*)((uint8_t*)workspace + w.ndelta_l);
+  a.nlse2_l = (float*)((uint8_t*)workspace + w.nlse2_l);
   cudaStream_t st = (cudaStream_t)stream;
   CHECK_LAUNCH(launch_bwd_preprocess(g, a, false, st), "sta_bwd preprocess launch");
   CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, false, st), "sta_bwd dk/dv launch");
@@ -490,14 +506,18 @@ int vattn_dual_bwd(const vattn_geom* geom, const void* q, const void* k, const v
   a.dv = dv;
   a.dg = dg;
   uint8_t* ws = (uint8_t*)workspace;
-  a.delta_l = (float*)(ws + w.delta_l);
-  a.delta_g = (float*)(ws + w.delta_g);
+  a.ndelta_l = (float*)(ws + w.ndelta_l);
+  a.ndelta_g = (float*)(ws + w.ndelta_g);
+  a.nlse2_l = (float*)(ws + w.nlse2_l);
+  a.nlse2_g = (float*)(ws + w.nlse2_g);
   a.dkp = (float*)(ws + w.dkp);
   a.dvp = (float*)(ws + w.dvp);
+  a.dq_acc = (float*)(ws + w.dq_acc);
   cudaStream_t st = (cudaStream_t)stream;
   CHECK_LAUNCH(launch_bwd_preprocess(g, a, true, st), "dual_bwd preprocess launch");
   CHECK_LAUNCH(launch_bwd_dkdv_global(g, a, st), "dual_bwd global dk/dv launch");
   CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, true, st), "dual_bwd local dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dq_global(g, a, st), "dual_bwd global dq launch");
   CHECK_LAUNCH(launch_bwd_dq(g, a, true, st), "dual_bwd dq launch");
   return ok();
 }

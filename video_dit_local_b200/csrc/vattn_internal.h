@@ -57,6 +57,7 @@ struct FwdArgs {
   void* blend_out;
 };
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st);
 
 // -- attention backward (attn_bwd.cu) --
 struct BwdArgs {
@@ -77,13 +78,17 @@ struct BwdArgs {
   void* dv;
   float* dg;              // optional
   // workspace pieces
-  float* delta_l;         // [B,h,N] rowsum(dO*O_l)
-  float* delta_g;         // [B,h,N] rowsum(dO*O_g)
+  float* ndelta_l;        // [B,h,N] -rowsum(dO*O_l)
+  float* ndelta_g;        // [B,h,N] -rowsum(dO*O_g)
+  float* nlse2_l;         // [B,h,N] log2(gamma_l) - LSE_l*log2(e)
+  float* nlse2_g;         // [B,h,N] log2(gamma_g) - LSE_g*log2(e)
   float* dkp;             // [B,h,Np,d] fp32
   float* dvp;
+  float* dq_acc;          // [B,h,N,d] fp32 global-branch part of dQ (dual only)
 };
 cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
 cudaError_t launch_bwd_dq(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
+cudaError_t launch_bwd_dq_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st);
 
