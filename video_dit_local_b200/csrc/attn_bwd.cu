@@ -534,13 +534,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // ---------------------------------------------------------------------------
 // dQ
 // ---------------------------------------------------------------------------
+// dQ key block: 96 keys.  TMEM holds S0 [0,96), S1 [96,192), dP0 [192,288),
+// dP1 [288,384) and the dQ accumulator [384,384+D); a 96-wide block puts 50%
+// more work into every S / dP instruction than a 64-wide one.
+constexpr int DQ_BN = 96;
+constexpr uint32_t DQ_S0 = 0, DQ_S1 = 96, DQ_P0 = 192, DQ_P1 = 288, DQ_ACC = 384;
+
 template <int D>
 struct DqSmem {
   static constexpr int CHUNKS = D / 64;
-  static constexpr int QB_BYTES = CHUNKS * 128 * 128;  // 128 query rows
-  static constexpr int KB_BYTES = CHUNKS * 64 * 128;   // 64 key rows
-  static constexpr int NK = 4;
-  static constexpr int NV = 4;
+  static constexpr int QB_BYTES = CHUNKS * 128 * 128;    // 128 query rows
+  static constexpr int KB_BYTES = CHUNKS * DQ_BN * 128;  // DQ_BN key rows
+  static constexpr int NK = 3;
+  static constexpr int NV = 3;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = QB_BYTES;
   static constexpr int OFF_K = 2 * QB_BYTES;
@@ -614,7 +620,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   const RowStream ks = glob ? flat_stream(g.Np) : window_stream(g, q_tile);
   const int Lk = ks.length();
-  const int nblk = (Lk + 63) / 64;
+  const int nblk = (Lk + DQ_BN - 1) / DQ_BN;
 
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
@@ -644,7 +650,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   constexpr uint32_t QBOX = 128 * 128;
-  constexpr uint32_t KBOX = 64 * 128;
+  constexpr uint32_t KBOX = DQ_BN * 128;
 
   if (warp == WARP_LOAD_A || warp == WARP_LOAD_B) {
     if (lane == 0) {
@@ -665,11 +671,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = j % NS, r = j / NS;
         if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
         mbar_arrive_expect_tx(&full[s], L::KB_BYTES);
-        const int G = glob ? 64 : p.G0;
+        const int G = glob ? DQ_BN : p.G0;
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
         const int oob = glob ? g.Np : g.N;
-        for (int u = 0; u < 64 / G; ++u) {
-          const int v = j * 64 + u * G;
+        for (int u = 0; u < DQ_BN / G; ++u) {
+          const int v = j * DQ_BN + u * G;
           const int row = v < Lk ? ks.row(g, v) : oob;
           for (int c = 0; c < L::CHUNKS; ++c)
             tma_load_3d(smem + off + s * L::KB_BYTES + c * KBOX + u * G * 128, tm, &full[s], c * 64, row, bh);
@@ -681,7 +687,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, DQ_BN, 0, 0);
       constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_base = smem_u32(smem + L::OFF_Q), do_base = smem_u32(smem + L::OFF_DO);
       const uint32_t k_base = smem_u32(smem + L::OFF_K), v_base = smem_u32(smem + L::OFF_V);
@@ -695,10 +701,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t qo = (kk >> 2) * QBOX + (kk & 3) * 32, ko = (kk >> 2) * KBOX + (kk & 3) * 32;
-          mma_ss(tmem + w * 64, smem_desc_sw128(q_base + qo, 16, 1024), smem_desc_sw128(kb + ko, 16, 1024), IDESC_S,
-                 kk > 0);
-          mma_ss(tmem + 128 + w * 64, smem_desc_sw128(do_base + qo, 16, 1024), smem_desc_sw128(vb + ko, 16, 1024),
+          mma_ss(tmem + (w ? DQ_S1 : DQ_S0), smem_desc_sw128(q_base + qo, 16, 1024), smem_desc_sw128(kb + ko, 16, 1024),
                  IDESC_S, kk > 0);
+          mma_ss(tmem + (w ? DQ_P1 : DQ_P0), smem_desc_sw128(do_base + qo, 16, 1024),
+                 smem_desc_sw128(vb + ko, 16, 1024), IDESC_S, kk > 0);
         }
         tc_commit(&v_empty[sv]);
         tc_commit(&sdp_full[w]);
@@ -712,9 +718,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
         const uint32_t kb = k_base + sk * L::KB_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + 256, tmem + 128 + w * 64 + kk * 8, smem_desc_sw128(kb + kk * 2048, KBOX, 1024), IDESC_ACC,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < DQ_BN / 16; ++kk)
+          mma_ts(tmem + DQ_ACC, tmem + (w ? DQ_P1 : DQ_P0) + kk * 8, smem_desc_sw128(kb + kk * 2048, KBOX, 1024),
+                 IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&k_empty[sk]);
         if (j + 2 < nblk) ok = issue_sdp(j + 2);
       }
@@ -724,8 +730,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     const int w = warp >> 2, quad = warp & 3, row = quad * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 64);
-    const uint32_t tP = tmem + lane_addr + 128u + (uint32_t)(w * 64);
+    const uint32_t tS = tmem + lane_addr + (w ? DQ_S1 : DQ_S0);
+    const uint32_t tP = tmem + lane_addr + (w ? DQ_P1 : DQ_P0);
     const int qrow = min(q_row0 + row, g.N - 1);  // padding rows read a valid entry and are never stored
     const size_t qi = (size_t)bh * g.N + qrow;
     const float2 nl2 = make_float2(p.nlse2[qi], p.nlse2[qi]), nd2 = make_float2(p.ndelta[qi], p.ndelta[qi]);
@@ -737,24 +743,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[2][32], dv[2][32];
-      tmem_ld32(tS, sv[0]);
-      tmem_ld32(tS + 32, sv[1]);
-      tmem_ld32(tP, dv[0]);
-      tmem_ld32(tP + 32, dv[1]);
-      tmem_wait_ld();
-      const int valid = Lk - j * 64;
-      const bool full_blk = valid >= 64;
+      const int valid = Lk - j * DQ_BN;
+      const bool full_blk = valid >= DQ_BN;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int hh = 0; hh < DQ_BN / 32; ++hh) {
+        // one 32-column chunk at a time: S, dP and the packed dS stay in registers
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tS + hh * 32, sv);
+        tmem_ld32(tP + hh * 32, dv);
+        tmem_wait_ld();
         uint32_t dk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float2 x =
-              ffma2(make_float2(__uint_as_float(sv[hh][2 * c]), __uint_as_float(sv[hh][2 * c + 1])), c2x2, nl2);
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])), c2x2, nl2);
           const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-          float2 o2 =
-              fmul2(pp, fadd2(make_float2(__uint_as_float(dv[hh][2 * c]), __uint_as_float(dv[hh][2 * c + 1])), nd2));
+          float2 o2 = fmul2(pp, fadd2(make_float2(__uint_as_float(dv[2 * c]), __uint_as_float(dv[2 * c + 1])), nd2));
           if (!full_blk) {
             const int cc = hh * 32 + 2 * c;
             if (cc >= valid) o2.x = 0.f;
@@ -774,7 +777,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     if (ok && !*abort_flag) {
       const bool row_ok = row < q_valid;
-      const uint32_t tAcc = tmem + lane_addr + 256u;
+      const uint32_t tAcc = tmem + lane_addr + DQ_ACC;
       const size_t grow = (size_t)bh * g.N + q_row0 + row;
 #pragma unroll 1
       for (int c0 = (w * D) / 2; c0 < ((w + 1) * D) / 2; c0 += 32) {
@@ -871,7 +874,9 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   DqParams p;
   p.g = g;
   p.mode = global ? DQ_GLOBAL : DQ_LOCAL;
-  p.G0 = pow2_rows(g.s, 64);
+  int G0 = DQ_BN;  // largest multiple of 8 dividing both the key block and the tile volume
+  while (G0 > 8 && (DQ_BN % G0 != 0 || g.s % G0 != 0)) G0 -= 8;
+  p.G0 = G0;
   p.q_blocks_per_tile = (g.s + 127) / 128;
   p.scale = a.scale;
   p.c2 = a.scale * LOG2E;
@@ -889,7 +894,7 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   const void* kk = global ? a.kp : a.k;
   const void* vv = global ? a.vp : a.v;
   const long long nk = global ? g.Np : g.N;
-  const int G = global ? 64 : p.G0;
+  const int G = global ? DQ_BN : p.G0;
   if (!make_tmap_rows(&tq, a.q, D, g.N, bh, 128, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, 128, &err) ||
       !make_tmap_rows(&tk, kk, D, nk, bh, G, &err) || !make_tmap_rows(&tv, vv, D, nk, bh, G, &err))
     return cudaErrorInvalidValue;
