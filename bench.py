@@ -43,6 +43,23 @@ STA_FWD_TRAFFIC = 2683000000  # bytes per launch, from profiles/sta_fwd_720p.md 
 STA_FWD_TRAFFIC_SRC_SHA = "b36fa1d8cdbf443f"
 
 
+def reduce_max(values, world: int, device=None):
+    """Max over ranks of a list of floats (the timing rule: every multi-GPU
+    number is the slowest rank's); a no-op on one process."""
+    if world <= 1:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(flops_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job throughput: every rank runs its own full workload (weak
+    scaling), so the job's work is world x per-rank work over the max time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def _src_sha() -> str:
     h = hashlib.sha256()
     for f in ("attn_fwd.cu", "common.cuh"):
@@ -253,10 +270,7 @@ def run_ours(args, rank, world, local_rank):
     if V.vattn_get_status() != 0:
         raise RuntimeError("device status after timing: " + V.vattn_last_error())
     ms_step = ms_total / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step, ms_kernel], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step, ms_kernel = t.tolist()
+    ms_step, ms_kernel = reduce_max([ms_step, ms_kernel], world, dev)
 
     # end to end through the C ABI from pinned host buffers
     o_host = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
@@ -280,10 +294,7 @@ def run_ours(args, rank, world, local_rank):
     a1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = a0.elapsed_time(a1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = t.item()
+    ms_e2e = reduce_max([ms_e2e], world, dev)[0]
     h2d = sum(p.numel() * p.element_size() for p in pinned)
     d2h = o_host.numel() * 2 + lse_host.numel() * 4
 
@@ -292,7 +303,7 @@ def run_ours(args, rank, world, local_rank):
     traffic = STA_FWD_TRAFFIC if STA_FWD_TRAFFIC_SRC_SHA == _src_sha() else None
     result = {
         "metric": METRIC,
-        "value": round(world * flops_local / (ms_step * 1e-3) / 1e12, 2),
+        "value": round(whole_job_tflops(flops_local, ms_step, world), 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -314,7 +325,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{peak_src} bf16 (burst)", "traffic": traffic,
                      "kernel": "attn_fwd_kernel<128> (sliding tile)", "kernel_ms": round(ms_kernel, 4),
                      "algorithmic_flop_per_launch": flops_local},
-        "e2e": {"value": round(world * flops_local / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(whole_job_tflops(flops_local, ms_e2e, world), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
