@@ -479,3 +479,64 @@ def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_til
         dk[r] += dkp[c] / cnt
         dv[r] += dvp[c] / cnt
     return dict(q_ids=np.concatenate(q_ids), dQ=np.concatenate(dq_rows), k_ids=want, dK=dk, dV=dv)
+
+
+# ---------------------------------------------------------------------------
+# cross-window local attention ("UltraGen ..." §4.3: window partitions that
+# alternate between adjacent layers, K x K windows and shifted (K+1) x (K+1)
+# partitions).  Reading taken: along each dim the tile grid is cut into
+# consecutive blocks; mode "partition" uses blocks of `window` tiles starting
+# at tile 0, mode "shifted" uses blocks of `window + 1` tiles whose cuts are
+# moved by floor((window + 1) / 2); blocks at the grid edge are truncated.  A
+# query tile attends to every tile of its own block (in all three dims).
+# ---------------------------------------------------------------------------
+
+def partition_range(a: int, w: int, n: int, shifted: bool) -> range:
+    """Tiles of the block holding tile a along one dim."""
+    size = w + 1 if shifted else w
+    off = (w + 1) // 2 if shifted else 0
+    b = (a + off) // size
+    lo = max(b * size - off, 0)
+    hi = min((b + 1) * size - off, n)
+    return range(lo, hi)
+
+
+def xwin_query_tiles(g: Geom, shifted: bool):
+    """Yield (query token ids, key token ids) per query tile, both raster."""
+    nt, nh, nw = g.tiles_per_dim
+    for at in range(nt):
+        for ah in range(nh):
+            for aw in range(nw):
+                qi = _tile_token_box(g, (at, ah, aw), (at + 1, ah + 1, aw + 1))
+                rt = partition_range(at, g.window[0], nt, shifted)
+                rh = partition_range(ah, g.window[1], nh, shifted)
+                rw = partition_range(aw, g.window[2], nw, shifted)
+                kj = _tile_token_box(g, (rt.start, rh.start, rw.start), (rt.stop, rh.stop, rw.stop))
+                yield qi, kj
+
+
+def xwin_attention(q, k, v, g: Geom, scale: float, shifted: bool):
+    """Cross-window local attention: raster in, raster out (O, LSE)."""
+    B, nh, n, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, nh, n))
+    for b in range(B):
+        for h in range(nh):
+            for qi, kj in xwin_query_tiles(g, shifted):
+                o[b, h, qi], lse[b, h, qi], _ = _softmax_attend(q[b, h, qi], k[b, h, kj], v[b, h, kj], scale)
+    return o, lse
+
+
+def xwin_backward(q, k, v, do, g: Geom, scale: float, shifted: bool):
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    B, nh = q.shape[:2]
+    for b in range(B):
+        for h in range(nh):
+            for qi, kj in xwin_query_tiles(g, shifted):
+                a, bk, c = _softmax_attend_bwd(q[b, h, qi], k[b, h, kj], v[b, h, kj], do[b, h, qi], scale)
+                dq[b, h, qi] += a
+                dk[b, h, kj] += bk
+                dv[b, h, kj] += c
+    return dq, dk, dv

@@ -350,3 +350,101 @@ def test_sampled_evaluators_equal_full_definitions():
     assert np.abs(ol - fwd["O_l"][0, 0][ids]).max() < 1e-12 and np.abs(lsel - fwd["LSE_l"][0, 0][ids]).max() < 1e-12
     og, lseg = O.global_attention_rows(q[0, 0], fwd["K_p"][0, 0], fwd["V_p"][0, 0], 0.4, ids)
     assert np.abs(og - fwd["O_g"][0, 0][ids]).max() < 1e-12
+
+
+# ---------------------------------------------------------------- cross-window local attention
+
+def _brute_blocks(n, w, shifted):
+    """Independent construction of the partition: walk the dim and start a new
+    block at every cut (cuts at positions p with (p + off) % size == 0)."""
+    size = w + 1 if shifted else w
+    off = (w + 1) // 2 if shifted else 0
+    blocks, cur = [], []
+    for p in range(n):
+        if cur and (p + off) % size == 0:
+            blocks.append(cur)
+            cur = []
+        cur.append(p)
+    blocks.append(cur)
+    return blocks
+
+
+@pytest.mark.parametrize("shifted", [False, True])
+def test_partition_blocks_tile_the_dim_and_match_walk(shifted):
+    for n in range(1, 17):
+        for w in range(1, 9):
+            blocks = _brute_blocks(n, w, shifted)
+            assert sorted(x for b in blocks for x in b) == list(range(n))
+            for b in blocks:
+                for a in b:
+                    assert list(O.partition_range(a, w, n, shifted)) == b
+
+
+def test_shifted_blocks_straddle_unshifted_cuts():
+    # every interior cut of the K-partition lies strictly inside a shifted block
+    for n in (9, 15, 30):
+        for w in (2, 3, 4):
+            cuts = [b[0] for b in _brute_blocks(n, w, False)][1:]
+            for c in cuts:
+                r = O.partition_range(c, w, n, True)
+                if r.start != c:
+                    continue
+                # a cut shared by both partitions is allowed only where the periods realign
+                assert (c + (w + 1) // 2) % (w + 1) == 0 and c % w == 0
+
+
+def _xwin_mask(g, shifted):
+    c = O.token_coords(g)
+    tc = c // np.asarray(g.tile)
+    dims = g.tiles_per_dim
+    lab = []
+    for ax in range(3):
+        blocks = _brute_blocks(dims[ax], g.window[ax], shifted)
+        label = np.empty(dims[ax], dtype=int)
+        for i, b in enumerate(blocks):
+            label[b] = i
+        lab.append(label[tc[:, ax]])
+    same = np.ones((g.n, g.n), dtype=bool)
+    for ax in range(3):
+        same &= lab[ax][:, None] == lab[ax][None, :]
+    return same
+
+
+@pytest.mark.parametrize("shifted", [False, True])
+def test_xwin_equals_masked_softmax(shifted):
+    g = O.Geom(4, 16, 24, (2, 4, 4), (1, 2, 3))
+    q, k, v = (_rand((1, 2, g.n, 8), s) for s in (40, 41, 42))
+    mask = _xwin_mask(g, shifted)
+    assert np.array_equal(mask, mask.T)        # symmetric relation
+    o, _ = O.xwin_attention(q, k, v, g, 0.3, shifted)
+    assert np.abs(o - _sdpa(q, k, v, 0.3, mask)).max() < 1e-12
+
+
+def test_xwin_window_covering_grid_is_full_attention():
+    g = O.Geom(4, 8, 8, (2, 4, 4), (2, 2, 2))
+    q, k, v = (_rand((1, 1, g.n, 8), s) for s in (43, 44, 45))
+    o, _ = O.xwin_attention(q, k, v, g, 0.3, False)
+    assert np.abs(o - _sdpa(q, k, v, 0.3)).max() < 1e-12
+
+
+@pytest.mark.parametrize("shifted", [False, True])
+def test_xwin_backward_finite_differences(shifted):
+    g = O.Geom(4, 16, 24, (2, 4, 4), (1, 2, 3))
+    rng = np.random.default_rng(46)
+    q, k, v = (rng.standard_normal((1, 1, g.n, 4)) for _ in range(3))
+    do = rng.standard_normal((1, 1, g.n, 4))
+    dq, dk, dv = O.xwin_backward(q, k, v, do, g, 0.4, shifted)
+
+    def loss():
+        return float((O.xwin_attention(q, k, v, g, 0.4, shifted)[0] * do).sum())
+    eps = 1e-5
+    for arr, grad in ((q, dq), (k, dk), (v, dv)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            old = arr[idx]
+            arr[idx] = old + eps
+            lp = loss()
+            arr[idx] = old - eps
+            lm = loss()
+            arr[idx] = old
+            assert abs((lp - lm) / (2 * eps) - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx]))
