@@ -373,7 +373,56 @@ def run_extras(V, dev):
         del q, k, v, o, ws
         torch.cuda.empty_cache()
     out["train_fwd_bwd"] = _bench_train(V, dev, peaks)
+    out.update(_bench_xwin(V, dev, peaks))
     return out
+
+
+def _xwin_pairs(w, shifted: bool) -> int:
+    """Query-key pairs of cross-window attention: the block extents are
+    separable per dim, so the sum over query tiles factorises."""
+    sizes = 1
+    for n_t, win in zip([a // b for a, b in zip(w.grid, w.tile)], w.window):
+        size = win + 1 if shifted else win
+        off = (win + 1) // 2 if shifted else 0
+        tot = 0
+        for a in range(n_t):
+            b = (a + off) // size
+            tot += min((b + 1) * size - off, n_t) - max(b * size - off, 0)
+        sizes *= tot
+    s = math.prod(w.tile)
+    return w.batch * w.heads * s * s * sizes
+
+
+def _bench_xwin(V, dev, peaks):
+    """Cross-window local attention at the 1080p grid (window 3x3x3), both
+    partitions, forward kernel timed alone."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["1080p"]
+    geom = _geom(V, w)
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 500 + i) for i in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    res = {}
+    for shifted in (0, 1):
+        fl = 4 * w.head_dim * _xwin_pairs(w, bool(shifted))
+        for _ in range(2):
+            V.vattn_xwin_fwd(geom, shifted, q, k, v, 1 / math.sqrt(w.head_dim), o, lse)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            V.vattn_xwin_fwd(geom, shifted, q, k, v, 1 / math.sqrt(w.head_dim), o, lse)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 5
+        res[f"1080p_xwin_fwd_{'shifted' if shifted else 'partition'}"] = {
+            "ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
+            "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status()}
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return res
 
 
 def _bench_train(V, dev, peaks, w=None, n=3, warm=2):

@@ -106,6 +106,23 @@ int vattn_kept_tiles(const vattn_geom* geom, int32_t* out, void* stream);
 int vattn_sta_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale,
                   void* o, float* lse, void* stream);
 
+/* Cross-window local attention forward ("UltraGen ..." §4.3: window
+ * partitions alternating between adjacent layers, K x K windows and shifted
+ * (K+1) x (K+1) partitions).  Along every dim the tile grid is cut into
+ * consecutive blocks: shifted = 0 uses blocks of window[d] tiles starting at
+ * tile 0; shifted = 1 uses blocks of window[d] + 1 tiles whose cuts are moved
+ * by floor((window[d] + 1) / 2); blocks at the grid edge are truncated.  Each
+ * query tile attends to all tiles of its block.  Arguments and layouts as in
+ * vattn_sta_fwd. */
+int vattn_xwin_fwd(const vattn_geom* geom, int shifted, const void* q, const void* k, const void* v,
+                   float scale, void* o, float* lse, void* stream);
+
+/* Backward of vattn_xwin_fwd (same contract as vattn_sta_bwd; workspace size
+ * vattn_workspace_size(VATTN_OP_STA_BWD)). */
+int vattn_xwin_bwd(const vattn_geom* geom, int shifted, const void* q, const void* k, const void* v,
+                   const void* o, const float* lse, const void* dout, float scale, void* dq, void* dk,
+                   void* dv, void* workspace, size_t ws_bytes, void* stream);
+
 /* Average pooling of K and V over p_t x p_h x p_w token blocks ("UltraGen ..."
  * §4.2: latents downsampled before global attention).  Inputs tile-major
  * [B,h,N,d]; outputs pooled-raster [B,h,N_p,d].  fp32 sum, exact divide by

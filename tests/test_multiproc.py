@@ -63,3 +63,15 @@ def test_reference_arm_prints_once_under_torchrun():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["value"] > 0
+
+
+def test_bench_xwin_pair_count_matches_oracle_tiles():
+    sys.path.insert(0, ROOT)
+    import bench
+    from oracle import vattn_oracle as O
+    from synth import inputs as S
+    w = S.small_workload("x", 1, 1, 2, 64, (6, 24, 40), (3, 8, 8), (2, 2, 2), (1, 1, 1))
+    g = O.geom_of(w)
+    for shifted in (False, True):
+        brute = sum(len(qi) * len(kj) for qi, kj in O.xwin_query_tiles(g, shifted)) * w.batch * w.heads
+        assert bench._xwin_pairs(w, shifted) == brute

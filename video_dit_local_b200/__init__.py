@@ -22,6 +22,8 @@ from .binding import (  # noqa: F401
     vattn_tile_unpermute,
     vattn_version,
     vattn_workspace_size,
+    vattn_xwin_bwd,
+    vattn_xwin_fwd,
     VATTN_OP_DUAL_FWD,
     VATTN_OP_STA_BWD,
     VATTN_OP_DUAL_BWD,

@@ -79,6 +79,8 @@ _SIGS = {
     "vattn_sta_bwd": [_GP, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_fwd_noalloc": [_GP, _P, _P, _P, _P, _F, _P, _P],
+    "vattn_xwin_fwd": [_GP, _INT, _P, _P, _P, _F, _P, _P, _P],
+    "vattn_xwin_bwd": [_GP, _INT, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_workspace_size": [_INT, _GP, ctypes.POINTER(_SZ)],
     "vattn_get_status": [_P],
     "vattn_last_error": [],
@@ -145,6 +147,20 @@ def vattn_kept_tiles(geom: Geom, out, stream=None) -> None:
 def vattn_sta_fwd(geom: Geom, q, k, v, scale: float, o, lse=None, stream=None) -> None:
     _check(lib.vattn_sta_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
                              _stream(stream)))
+
+
+def vattn_xwin_fwd(geom: Geom, shifted: int, q, k, v, scale: float, o, lse=None, stream=None) -> None:
+    _check(lib.vattn_xwin_fwd(ctypes.byref(geom), int(shifted), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
+                              _stream(stream)))
+
+
+def vattn_xwin_bwd(geom: Geom, shifted: int, q, k, v, o, lse, dout, scale: float, dq, dk, dv, workspace,
+                   ws_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_xwin_bwd(ctypes.byref(geom), int(shifted), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                              _ptr(dout), scale, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
+                              _stream(stream)))
 
 
 def vattn_pool_kv(geom: Geom, k, v, kp, vp, stream=None) -> None:

@@ -62,12 +62,12 @@ __device__ __forceinline__ RowStream flat_stream(int n) {
 __device__ __forceinline__ RowStream window_stream(const DevGeom& g, int q) {
   const int at = q / (g.Nh * g.Nw), ah = (q / g.Nw) % g.Nh, aw = q % g.Nw;
   RowStream s;
-  s.t0 = win_start(at, g.wt, g.Nt);
-  s.h0 = win_start(ah, g.wh, g.Nh);
-  s.w0 = win_start(aw, g.ww, g.Nw);
-  s.eh = win_extent(g.wh, g.Nh);
-  s.runs = win_extent(g.wt, g.Nt) * s.eh;
-  s.run_len = win_extent(g.ww, g.Nw) * g.s;
+  int et, ew;
+  tile_range(at, g.wt, g.Nt, g.wmode, &s.t0, &et);
+  tile_range(ah, g.wh, g.Nh, g.wmode, &s.h0, &s.eh);
+  tile_range(aw, g.ww, g.Nw, g.wmode, &s.w0, &ew);
+  s.runs = et * s.eh;
+  s.run_len = ew * g.s;
   s.tiled = true;
   return s;
 }
@@ -77,9 +77,9 @@ __device__ __forceinline__ RowStream window_stream(const DevGeom& g, int q) {
 __device__ __forceinline__ RowStream inverse_stream(const DevGeom& g, int k) {
   const int kt = k / (g.Nh * g.Nw), kh = (k / g.Nw) % g.Nh, kw = k % g.Nw;
   int lt, ht, lh, hh, lw, hw;
-  inverse_range(kt, g.wt, g.Nt, &lt, &ht);
-  inverse_range(kh, g.wh, g.Nh, &lh, &hh);
-  inverse_range(kw, g.ww, g.Nw, &lw, &hw);
+  tile_inverse(kt, g.wt, g.Nt, g.wmode, &lt, &ht);
+  tile_inverse(kh, g.wh, g.Nh, g.wmode, &lh, &hh);
+  tile_inverse(kw, g.ww, g.Nw, g.wmode, &lw, &hw);
   RowStream s;
   s.t0 = lt;
   s.h0 = lh;

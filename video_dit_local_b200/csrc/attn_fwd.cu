@@ -82,13 +82,12 @@ __device__ __forceinline__ Stream make_stream(const Params& p, int q_tile) {
   if (p.mode == FWD_STA) {
     const DevGeom& g = p.g;
     const int at = q_tile / (g.Nh * g.Nw), ah = (q_tile / g.Nw) % g.Nh, aw = q_tile % g.Nw;
-    s.t0 = win_start(at, g.wt, g.Nt);
-    s.h0 = win_start(ah, g.wh, g.Nh);
-    s.w0 = win_start(aw, g.ww, g.Nw);
-    const int et = win_extent(g.wt, g.Nt);
-    s.eh = win_extent(g.wh, g.Nh);
+    int et, ew;
+    tile_range(at, g.wt, g.Nt, g.wmode, &s.t0, &et);
+    tile_range(ah, g.wh, g.Nh, g.wmode, &s.h0, &s.eh);
+    tile_range(aw, g.ww, g.Nw, g.wmode, &s.w0, &ew);
     s.runs = et * s.eh;
-    s.run_len = win_extent(g.ww, g.Nw) * g.s;
+    s.run_len = ew * g.s;
   } else {
     s.runs = 1;
     s.run_len = p.Nk;

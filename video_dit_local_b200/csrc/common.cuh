@@ -317,6 +317,37 @@ __host__ __device__ __forceinline__ void inverse_range(int k, int w, int n, int*
   *hi = h;
 }
 
+// Window of tile a along one dim for any window mode (see WIN_* in
+// vattn_internal.h); ext may vary from tile to tile for the partition modes.
+__host__ __device__ __forceinline__ void tile_range(int a, int w, int n, int mode, int* start, int* ext) {
+  if (mode == WIN_SLIDING) {
+    *start = win_start(a, w, n);
+    *ext = win_extent(w, n);
+    return;
+  }
+  const int size = mode == WIN_SHIFTED ? w + 1 : w;
+  const int off = mode == WIN_SHIFTED ? (w + 1) / 2 : 0;
+  const int b = (a + off) / size;
+  int lo = b * size - off, hi = (b + 1) * size - off;
+  lo = lo < 0 ? 0 : lo;
+  hi = hi > n ? n : hi;
+  *start = lo;
+  *ext = hi - lo;
+}
+
+// Query tiles whose window holds key tile k along one dim, for any mode: the
+// partition modes are symmetric (the block itself).
+__host__ __device__ __forceinline__ void tile_inverse(int k, int w, int n, int mode, int* lo, int* hi) {
+  if (mode == WIN_SLIDING) {
+    inverse_range(k, w, n, lo, hi);
+    return;
+  }
+  int s, e;
+  tile_range(k, w, n, mode, &s, &e);
+  *lo = s;
+  *hi = s + e - 1;
+}
+
 // A box of tiles streamed as runs: for every (t, h) tile row of the box, the
 // w-range of tiles is contiguous in tile-major memory.
 struct TileBox {

@@ -151,6 +151,7 @@ static int build_geom(const vattn_geom* in, int need, DevGeom* g) {
   g->s = g->tt * g->th * g->tw;
   g->n_tiles = g->Nt * g->Nh * g->Nw;
   g->kept = win_extent(g->wt, g->Nt) * win_extent(g->wh, g->Nh) * win_extent(g->ww, g->Nw);
+  g->wmode = WIN_SLIDING;
   g->PT = g->T / g->pt;
   g->PH = g->H / g->ph;
   g->PW = g->W / g->pw;
@@ -328,6 +329,30 @@ int vattn_sta_fwd(const vattn_geom* geom, const void* q, const void* k, const vo
   return ok();
 }
 
+int vattn_xwin_fwd(const vattn_geom* geom, int shifted, const void* q, const void* k, const void* v, float scale,
+                   void* o, float* lse, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (shifted != 0 && shifted != 1) return fail(VATTN_ERR_INVALID_ARG, "shifted must be 0 or 1");
+  g.wmode = shifted ? WIN_SHIFTED : WIN_PARTITION;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  if (lse && !aligned16(lse)) return fail(VATTN_ERR_ALIGN, "lse is not 16-byte aligned");
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, (cudaStream_t)stream), "xwin_fwd launch");
+  return ok();
+}
+
 int vattn_pool_kv(const vattn_geom* geom, const void* k, const void* v, void* kp, void* vp, void* stream) {
   DevGeom g;
   int r = build_geom(geom, NEED_TILE | NEED_POOL, &g);
@@ -458,6 +483,48 @@ int vattn_sta_bwd(const vattn_geom* geom, const void* q, const void* k, const vo
   CHECK_LAUNCH(launch_bwd_preprocess(g, a, false, st), "sta_bwd preprocess launch");
   CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, false, st), "sta_bwd dk/dv launch");
   CHECK_LAUNCH(launch_bwd_dq(g, a, false, st), "sta_bwd dq launch");
+  return ok();
+}
+
+int vattn_xwin_bwd(const vattn_geom* geom, int shifted, const void* q, const void* k, const void* v, const void* o,
+                   const float* lse, const void* dout, float scale, void* dq, void* dk, void* dv, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (shifted != 0 && shifted != 1) return fail(VATTN_ERR_INVALID_ARG, "shifted must be 0 or 1");
+  g.wmode = shifted ? WIN_SHIFTED : WIN_PARTITION;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(lse);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  const BwdWs w = bwd_ws(g, false);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.o_l = o;
+  a.lse_l = lse;
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ndelta_l = (float*)((uint8_t*)workspace + w.ndelta_l);
+  a.nlse2_l = (float*)((uint8_t*)workspace + w.nlse2_l);
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_bwd_preprocess(g, a, false, st), "xwin_bwd preprocess launch");
+  CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, false, st), "xwin_bwd dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dq(g, a, false, st), "xwin_bwd dq launch");
   return ok();
 }
 

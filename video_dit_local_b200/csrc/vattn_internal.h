@@ -22,7 +22,15 @@ struct DevGeom {
   int s;                    // tile volume
   int n_tiles, kept;        // tiles, kept tiles per query tile
   int PT, PH, PW;           // pooled grid
+  int wmode;                // key-tile window: WIN_SLIDING, WIN_PARTITION, WIN_SHIFTED
 };
+
+// Key-tile window of a query tile along one dim:
+//   WIN_SLIDING   the sliding tile window (clamped into the grid);
+//   WIN_PARTITION the block of `window` consecutive tiles holding the tile;
+//   WIN_SHIFTED   the block of `window + 1` tiles with cuts moved by
+//                 floor((window + 1) / 2) (cross-window attention).
+enum { WIN_SLIDING = 0, WIN_PARTITION = 1, WIN_SHIFTED = 2 };
 
 // Runtime knobs shared by the attention kernels.
 struct DevCtl {
