@@ -3,6 +3,7 @@
 // allocated here.
 #include <atomic>
 #include <cstdarg>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -20,8 +21,10 @@ static std::atomic<long long> s_timeout_ns{2000000000ll};
 // Address of this device's status word (cached per device).
 static int* error_word_ptr() {
   static int* cache[64] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
   if (!cache[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) cache[dev] = (int*)p;
@@ -72,14 +75,14 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 static EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
-  static std::atomic<bool> tried{false};
-  if (!fn && !tried.exchange(true)) {
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  });
   return fn;
 }
 
