@@ -540,3 +540,84 @@ def xwin_backward(q, k, v, do, g: Geom, scale: float, shifted: bool):
                 dk[b, h, kj] += bk
                 dv[b, h, kj] += c
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# symmetric compressed global branch ("UltraGen ..." §4.2: latents are
+# downsampled before global attention and restored afterwards by upsampling).
+# Reading taken: queries, keys and values are all average-pooled; the pooled
+# queries attend to all pooled keys; the result is brought back to the full
+# grid by separable linear interpolation along t, y and x with half-pixel
+# centres (source coordinate (i + 1/2) / p - 1/2, clamped to the pooled grid at
+# the edges).  The learned convolutions of the pages need trained weights and
+# are not part of this definition.
+# ---------------------------------------------------------------------------
+
+def _interp_weights(n_out: int, n_in: int, p: int) -> np.ndarray:
+    """[n_out, n_in] linear interpolation matrix along one dim."""
+    m = np.zeros((n_out, n_in))
+    for i in range(n_out):
+        src = (i + 0.5) / p - 0.5
+        src = min(max(src, 0.0), n_in - 1.0)
+        i0 = int(math.floor(src))
+        i1 = min(i0 + 1, n_in - 1)
+        f = src - i0
+        m[i, i0] += 1.0 - f
+        m[i, i1] += f
+    return m
+
+
+def upsample(x_pooled: np.ndarray, g: Geom) -> np.ndarray:
+    """Pooled-raster [..., N_p, d] -> raster [..., N, d] by the separable
+    interpolation above."""
+    PT, PH, PW = g.pooled_dims
+    lead = x_pooled.shape[:-2]
+    d = x_pooled.shape[-1]
+    x = x_pooled.reshape(lead + (PT, PH, PW, d))
+    mt = _interp_weights(g.T, PT, g.pool[0])
+    mh = _interp_weights(g.H, PH, g.pool[1])
+    mw = _interp_weights(g.W, PW, g.pool[2])
+    y = np.einsum("tT,...THWd->...tHWd", mt, x)
+    y = np.einsum("hH,...tHWd->...thWd", mh, y)
+    y = np.einsum("wW,...thWd->...thwd", mw, y)
+    return y.reshape(lead + (g.n, d))
+
+
+def upsample_transpose(y: np.ndarray, g: Geom) -> np.ndarray:
+    """Adjoint of upsample: raster [..., N, d] -> pooled-raster [..., N_p, d]."""
+    PT, PH, PW = g.pooled_dims
+    lead = y.shape[:-2]
+    d = y.shape[-1]
+    z = y.reshape(lead + (g.T, g.H, g.W, d))
+    mt = _interp_weights(g.T, PT, g.pool[0])
+    mh = _interp_weights(g.H, PH, g.pool[1])
+    mw = _interp_weights(g.W, PW, g.pool[2])
+    z = np.einsum("tT,...thwd->...Thwd", mt, z)
+    z = np.einsum("hH,...Thwd->...THwd", mh, z)
+    z = np.einsum("wW,...THwd->...THWd", mw, z)
+    return z.reshape(lead + (g.n_pooled, d))
+
+
+def global_sym_forward(q, k, v, g: Geom, scale: float):
+    """Symmetric global branch: (O_g [raster, full grid], O_p, LSE_p [pooled])."""
+    qp, kp, vp = pool(q, g), pool(k, g), pool(v, g)
+    o_p, lse_p = full_attention(qp, kp, vp, scale)
+    return upsample(o_p, g), o_p, lse_p
+
+
+def dual_sym_forward(q, k, v, gvec, g: Geom, scale: float):
+    o_l, lse_l = sta_attention(q, k, v, g, scale)
+    o_g, o_p, lse_p = global_sym_forward(q, k, v, g, scale)
+    gb = np.asarray(gvec, dtype=np.float64)[None, :, None, None]
+    return dict(O=gb * o_l + (1.0 - gb) * o_g, O_l=o_l, LSE_l=lse_l, O_p=o_p, LSE_p=lse_p)
+
+
+def dual_sym_backward(q, k, v, gvec, do, g: Geom, scale: float):
+    """Gradients of g*O_l + (1-g)*upsample(attn(pool q, pool k, pool v))."""
+    gb = np.asarray(gvec, dtype=np.float64)[None, :, None, None]
+    dq_l, dk_l, dv_l = sta_backward(q, k, v, gb * do, g, scale)
+    qp, kp, vp = pool(q, g), pool(k, g), pool(v, g)
+    do_p = upsample_transpose((1.0 - gb) * do, g)
+    dqp, dkp, dvp = global_backward(qp, kp, vp, do_p, scale)
+    return dict(dQ=dq_l + pool_transpose(dqp, g), dK=dk_l + pool_transpose(dkp, g),
+                dV=dv_l + pool_transpose(dvp, g), dQ_p=dqp, dK_p=dkp, dV_p=dvp)

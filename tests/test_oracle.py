@@ -448,3 +448,59 @@ def test_xwin_backward_finite_differences(shifted):
             lm = loss()
             arr[idx] = old
             assert abs((lp - lm) / (2 * eps) - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx]))
+
+
+# ---------------------------------------------------------------- symmetric global branch
+
+@pytest.mark.parametrize("g", [O.Geom(4, 8, 12, (2, 4, 4), (1, 1, 1), (2, 4, 4)),
+                               O.Geom(3, 16, 8, (1, 8, 8), (1, 1, 1), (1, 2, 4))],
+                         ids=["pool244", "pool124"])
+def test_upsample_matches_torch_trilinear(g):
+    x = _rand((2, g.n_pooled, 3), 50)
+    PT, PH, PW = g.pooled_dims
+    t = torch.from_numpy(x).reshape(2, PT, PH, PW, 3).permute(0, 4, 1, 2, 3)
+    ref = torch.nn.functional.interpolate(t, size=(g.T, g.H, g.W), mode="trilinear", align_corners=False)
+    ref = ref.permute(0, 2, 3, 4, 1).reshape(2, g.n, 3).numpy()
+    assert np.abs(O.upsample(x, g) - ref).max() < 1e-12
+
+
+def test_upsample_adjoint_and_constants():
+    g = O.Geom(4, 8, 12, (2, 4, 4), (1, 1, 1), (2, 4, 4))
+    x = _rand((2, g.n_pooled, 3), 51)
+    y = _rand((2, g.n, 3), 52)
+    assert abs((O.upsample(x, g) * y).sum() - (x * O.upsample_transpose(y, g)).sum()) < 1e-10
+    c = np.full((g.n_pooled, 2), -0.75)
+    assert np.abs(O.upsample(c, g) + 0.75).max() < 1e-15        # partition of unity
+    g1 = O.Geom(4, 8, 12, (2, 4, 4), (1, 1, 1), (1, 1, 1))   # pool 1: upsampling is the identity
+    assert np.array_equal(O.upsample(y, g1), y)
+
+
+def test_symmetric_global_pool_one_is_full_attention():
+    g = O.Geom(4, 8, 8, (2, 4, 4), (1, 2, 2), (1, 1, 1))
+    q, k, v = (_rand((1, 2, g.n, 8), s) for s in (53, 54, 55))
+    o_g, _, _ = O.global_sym_forward(q, k, v, g, 0.3)
+    assert np.abs(o_g - _sdpa(q, k, v, 0.3)).max() < 1e-12
+
+
+def test_dual_sym_backward_finite_differences():
+    g = O.Geom(4, 8, 8, (2, 4, 4), (1, 2, 2), (2, 2, 4))
+    rng = np.random.default_rng(56)
+    q, k, v = (rng.standard_normal((1, 2, g.n, 4)) for _ in range(3))
+    do = 0.1 * rng.standard_normal((1, 2, g.n, 4))
+    gvec = np.array([0.35, 0.8])
+    r = O.dual_sym_backward(q, k, v, gvec, do, g, 0.4)
+
+    def loss():
+        return float((O.dual_sym_forward(q, k, v, gvec, g, 0.4)["O"] * do).sum())
+    eps = 1e-5
+    for arr, key in ((q, "dQ"), (k, "dK"), (v, "dV")):
+        for _ in range(8):
+            idx = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            old = arr[idx]
+            arr[idx] = old + eps
+            lp = loss()
+            arr[idx] = old - eps
+            lm = loss()
+            arr[idx] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - r[key][idx]) <= 1e-6 * max(1.0, abs(fd)), (key, fd, r[key][idx])
