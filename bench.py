@@ -374,7 +374,42 @@ def run_extras(V, dev):
         torch.cuda.empty_cache()
     out["train_fwd_bwd"] = _bench_train(V, dev, peaks)
     out.update(_bench_xwin(V, dev, peaks))
+    out["1080p_dual_sym_fwd"] = _bench_sym(V, dev, peaks)
     return out
+
+
+def _bench_sym(V, dev, peaks):
+    """Dual forward with the symmetric (query-pooled) global branch at the
+    1080p workload; effective FLOPs: local pairs + pooled N_p x N_p pairs."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["1080p"]
+    geom = _geom(V, w)
+    T, H, W = w.grid
+    npool = (T // w.pool[0]) * (H // w.pool[1]) * (W // w.pool[2])
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 600 + i) for i in range(3))
+    gvec = torch.rand(w.heads, device=dev)
+    o = torch.empty_like(q)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_DUAL_SYM_FWD, geom), dtype=torch.uint8, device=dev)
+    fl, _ = _flops_fwd(w)
+    fl += 4 * w.head_dim * w.batch * w.heads * npool * npool
+    scale = 1 / math.sqrt(w.head_dim)
+    for _ in range(2):
+        V.vattn_dual_sym_fwd(geom, q, k, v, gvec, scale, o, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(4):
+        V.vattn_dual_sym_fwd(geom, q, k, v, gvec, scale, o, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 4
+    res = {"ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
+           "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status()}
+    del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def _xwin_pairs(w, shifted: bool) -> int:

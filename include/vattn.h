@@ -74,7 +74,13 @@ typedef enum {
 } vattn_status;
 
 /* Operation ids for vattn_workspace_size. */
-enum { VATTN_OP_DUAL_FWD = 1, VATTN_OP_STA_BWD = 2, VATTN_OP_DUAL_BWD = 3 };
+enum {
+  VATTN_OP_DUAL_FWD = 1,
+  VATTN_OP_STA_BWD = 2,
+  VATTN_OP_DUAL_BWD = 3,
+  VATTN_OP_DUAL_SYM_FWD = 4,
+  VATTN_OP_DUAL_SYM_BWD = 5
+};
 
 /* Raster -> tile-major row gather.  Tile-major position of raster token
  * (t, y, x) is tile_id*s + local_id with
@@ -170,6 +176,30 @@ int vattn_dual_fwd(const vattn_geom* geom, const void* q, const void* k, const v
  * Arguments, layouts and errors are otherwise those of vattn_dual_fwd. */
 int vattn_dual_fwd_noalloc(const vattn_geom* geom, const void* q, const void* k, const void* v,
                            const float* g, float scale, void* o, void* stream);
+
+/* Dual-branch forward with the symmetric compressed global branch
+ * ("UltraGen ..." §4.2: the latent is downsampled before global attention
+ * and brought back to full resolution afterwards).  Q, K and V are all
+ * average-pooled; the pooled queries attend to all pooled keys; the pooled
+ * result O_p is upsampled to the full grid by separable linear interpolation
+ * along t, y and x with half-pixel centres (source coordinate (i + 1/2)/p -
+ * 1/2, clamped at the edges); O = g*O_l + (1-g)*upsample(O_p).
+ * Saved outputs for the backward (all seven NULL for inference, then the
+ * intermediates live in `workspace` of vattn_workspace_size
+ * (VATTN_OP_DUAL_SYM_FWD)): o_l [B,h,N,d] bf16, lse_l [B,h,N] fp32 (both
+ * tile-major), qp, kp, vp, o_p [B,h,N_p,d] bf16 and lse_p [B,h,N_p] fp32 (all
+ * pooled-raster). */
+int vattn_dual_sym_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                       const float* g, float scale, void* o, void* o_l, float* lse_l, void* qp, void* kp,
+                       void* vp, void* o_p, float* lse_p, void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of vattn_dual_sym_fwd from its saved outputs: dq, dk, dv (bf16,
+ * tile-major) through the pooling of all three inputs and the upsampling.
+ * workspace >= vattn_workspace_size(VATTN_OP_DUAL_SYM_BWD). */
+int vattn_dual_sym_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                       const float* g, const void* o_l, const float* lse_l, const void* qp, const void* kp,
+                       const void* vp, const void* o_p, const float* lse_p, const void* dout, float scale,
+                       void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, void* stream);
 
 /* Sliding-tile attention backward.  Given q, k, v, the forward's o and lse
  * and the upstream gradient dout (all tile-major), writes dq, dk, dv (bf16,

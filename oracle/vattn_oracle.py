@@ -407,10 +407,12 @@ def global_attention_rows(q, kp, vp, scale: float, rows):
     return o, lse
 
 
-def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_tiles, k_tiles, chunk: int = 8192):
-    """dual_backward for one head ([N, d] raster inputs) restricted to the
-    tokens of `q_tiles` (dQ) and of `k_tiles` (dK, dV).  Every softmax row it
-    uses is the full row of the definition; only the outputs are restricted.
+def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_tiles, k_tiles, chunk: int = 8192,
+                          symmetric: bool = False):
+    """dual_backward (or, with symmetric=True, dual_sym_backward) for one head
+    ([N, d] raster inputs) restricted to the tokens of `q_tiles` (dQ) and of
+    `k_tiles` (dK, dV).  Every softmax row it uses is the full row of the
+    definition; only the outputs are restricted.
 
     Returns dict(q_ids, dQ, k_ids, dK, dV) with rows in the order of the ids.
     """
@@ -427,12 +429,22 @@ def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_til
         return qi, kj
 
     kp, vp = pool(k, g), pool(v, g)
+    u_all = pooled_index(g)
+    cnt = g.pool[0] * g.pool[1] * g.pool[2]
+    if symmetric:
+        # the pooled branch is small: its gradients are computed in full
+        qp = pool(q, g)
+        do_p = upsample_transpose(gg * do, g)
+        dqp, dkp_s, dvp_s = _softmax_attend_bwd(qp, kp, vp, do_p, scale)
     # dQ rows: local branch of the query tile, global branch of the same rows
     q_ids, dq_rows = [], []
     for tid in q_tiles:
         qi, kj = window_ids(tid)
         dq_l, _, _ = _softmax_attend_bwd(q[qi], k[kj], v[kj], gl * do[qi], scale)
-        dq_g, _, _ = _softmax_attend_bwd(q[qi], kp, vp, gg * do[qi], scale)
+        if symmetric:
+            dq_g = dqp[u_all[qi]] / cnt
+        else:
+            dq_g, _, _ = _softmax_attend_bwd(q[qi], kp, vp, gg * do[qi], scale)
         q_ids.append(qi)
         dq_rows.append(dq_l + dq_g)
     # dK/dV rows, local branch: every query tile whose window holds the key tile
@@ -454,9 +466,12 @@ def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_til
             if r is not None:
                 dk[r] += dk_a[col]
                 dv[r] += dv_a[col]
+    if symmetric:
+        dk += dkp_s[u_all[want]] / cnt
+        dv += dvp_s[u_all[want]] / cnt
+        return dict(q_ids=np.concatenate(q_ids), dQ=np.concatenate(dq_rows), k_ids=want, dK=dk, dV=dv)
     # pooled branch: dK_p, dV_p at the pool blocks of the wanted tokens, summed
     # over every query (row chunks of the full softmax)
-    u_all = pooled_index(g)
     cols = np.unique(u_all[want])
     dkp = np.zeros((len(cols), q.shape[1]))
     dvp = np.zeros_like(dkp)
@@ -473,7 +488,6 @@ def dual_backward_sampled(q, k, v, gval: float, do, g: Geom, scale: float, q_til
         dvp += pc.T @ doc
         dkp += scale * (ds.T @ qc)
     cidx = {int(c): i for i, c in enumerate(cols)}
-    cnt = g.pool[0] * g.pool[1] * g.pool[2]
     for r, tok in enumerate(want):
         c = cidx[int(u_all[tok])]
         dk[r] += dkp[c] / cnt

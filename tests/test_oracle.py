@@ -504,3 +504,15 @@ def test_dual_sym_backward_finite_differences():
             arr[idx] = old
             fd = (lp - lm) / (2 * eps)
             assert abs(fd - r[key][idx]) <= 1e-6 * max(1.0, abs(fd)), (key, fd, r[key][idx])
+
+
+def test_sampled_symmetric_backward_equals_full():
+    g = ODD
+    rng = np.random.default_rng(57)
+    q, k, v = (rng.standard_normal((1, 1, g.n, 8)) for _ in range(3))
+    do = rng.standard_normal((1, 1, g.n, 8))
+    full = O.dual_sym_backward(q, k, v, [0.4], do, g, 0.4)
+    s = O.dual_backward_sampled(q[0, 0], k[0, 0], v[0, 0], 0.4, do[0, 0], g, 0.4, [0, 7, 44], [0, 13, 44],
+                                symmetric=True)
+    for key, ids in (("dQ", "q_ids"), ("dK", "k_ids"), ("dV", "k_ids")):
+        assert np.abs(s[key] - full[key][0, 0][s[ids]]).max() < 1e-12

@@ -11,6 +11,8 @@ from .binding import (  # noqa: F401
     vattn_dual_bwd,
     vattn_dual_fwd,
     vattn_dual_fwd_noalloc,
+    vattn_dual_sym_bwd,
+    vattn_dual_sym_fwd,
     vattn_get_status,
     vattn_global_fwd,
     vattn_kept_tiles,
@@ -27,4 +29,6 @@ from .binding import (  # noqa: F401
     VATTN_OP_DUAL_FWD,
     VATTN_OP_STA_BWD,
     VATTN_OP_DUAL_BWD,
+    VATTN_OP_DUAL_SYM_BWD,
+    VATTN_OP_DUAL_SYM_FWD,
 )

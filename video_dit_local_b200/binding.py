@@ -27,6 +27,8 @@ VATTN_ERR_WORKSPACE = -7
 VATTN_OP_DUAL_FWD = 1
 VATTN_OP_STA_BWD = 2
 VATTN_OP_DUAL_BWD = 3
+VATTN_OP_DUAL_SYM_FWD = 4
+VATTN_OP_DUAL_SYM_BWD = 5
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -80,6 +82,8 @@ _SIGS = {
     "vattn_dual_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_fwd_noalloc": [_GP, _P, _P, _P, _P, _F, _P, _P],
     "vattn_xwin_fwd": [_GP, _INT, _P, _P, _P, _F, _P, _P, _P],
+    "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "vattn_dual_sym_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_xwin_bwd": [_GP, _INT, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_workspace_size": [_INT, _GP, ctypes.POINTER(_SZ)],
     "vattn_get_status": [_P],
@@ -161,6 +165,24 @@ def vattn_xwin_bwd(geom: Geom, shifted: int, q, k, v, o, lse, dout, scale: float
     _check(lib.vattn_xwin_bwd(ctypes.byref(geom), int(shifted), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
                               _ptr(dout), scale, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
                               _stream(stream)))
+
+
+def vattn_dual_sym_fwd(geom: Geom, q, k, v, g, scale: float, o, o_l=None, lse_l=None, qp=None, kp=None, vp=None,
+                       o_p=None, lse_p=None, workspace=None, ws_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_dual_sym_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), scale, _ptr(o), _ptr(o_l),
+                                  _ptr(lse_l), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(o_p), _ptr(lse_p), _ptr(workspace),
+                                  ws_bytes, _stream(stream)))
+
+
+def vattn_dual_sym_bwd(geom: Geom, q, k, v, g, o_l, lse_l, qp, kp, vp, o_p, lse_p, dout, scale: float, dq, dk, dv,
+                       workspace, ws_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_dual_sym_bwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o_l), _ptr(lse_l),
+                                  _ptr(qp), _ptr(kp), _ptr(vp), _ptr(o_p), _ptr(lse_p), _ptr(dout), scale, _ptr(dq),
+                                  _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def vattn_pool_kv(geom: Geom, k, v, kp, vp, stream=None) -> None:

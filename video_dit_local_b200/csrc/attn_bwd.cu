@@ -327,19 +327,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int i = 0; i < nblk; ++i) {
         const int s = i % NQ, r = i / NQ;
         if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
-        // LSE / D rows: whole 16-byte groups by bulk copy, a ragged tail of
-        // fewer than 4 rows (only at the end of a flat query stream) by plain
-        // loads, written before the arrival that publishes the stage
+        // LSE / D rows: whole 16-byte groups by bulk copy when the source is
+        // 16-byte aligned; a ragged tail (end of a flat query stream) or an
+        // unaligned source (a pooled grid used as the token sequence, N_p not
+        // a multiple of 4) by plain loads, written before the arrival that
+        // publishes the stage.
         uint32_t tx = L::QB_BYTES;
+        int nbulk[4] = {0, 0, 0, 0};  // subs <= 4 (Gq >= 16)
         for (int u = 0; u < subs; ++u) {
           const int v = i * 64 + u * p.Gq;
           if (v >= Lq) break;
-          const int n = min(p.Gq, Lq - v), nb = n & ~3;
+          const int n = min(p.Gq, Lq - v);
+          const size_t gi = (size_t)bh * g.N + qs.row(g, v);
+          const int nb = (gi % 4 == 0) ? (n & ~3) : 0;
+          nbulk[u] = nb;
           tx += nb * 4;
-          if (nb < n) {
-            const int row = qs.row(g, v);
-            for (int t = nb; t < n; ++t) vec_s[s * 64 + u * p.Gq + t] = vec[(size_t)bh * g.N + row + t];
-          }
+          for (int t = nb; t < n; ++t) vec_s[s * 64 + u * p.Gq + t] = vec[gi + t];
         }
         mbar_arrive_expect_tx(&full[s], tx);
         for (int u = 0; u < subs; ++u) {
@@ -348,10 +351,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int row = ok ? qs.row(g, v) : g.N;
           for (int c = 0; c < L::CHUNKS; ++c)
             tma_load_3d(smem + off_x + s * L::QB_BYTES + c * QBOX + u * p.Gq * 128, tm, &full[s], c * 64, row, bh);
-          if (ok) {
-            const int nb = min(p.Gq, Lq - v) & ~3;
-            if (nb > 0) bulk_load(vec_s + s * 64 + u * p.Gq, vec + (size_t)bh * g.N + row, nb * 4, &full[s]);
-          }
+          if (ok && nbulk[u] > 0)
+            bulk_load(vec_s + s * 64 + u * p.Gq, vec + (size_t)bh * g.N + row, nbulk[u] * 4, &full[s]);
         }
         ++issued;
       }
@@ -573,6 +574,7 @@ struct DqParams {
   const float* nlse2;    // log2(gamma) - LSE*log2(e) of this branch
   const float* ndelta;   // -rowsum(dO*O)
   const float* acc_in;   // LOCAL: fp32 global-branch dQ to add (NULL = none)
+  int acc_pooled;        // acc_in holds pooled rows: add acc_in[pool(tok)] / block size
   float* acc_out;        // GLOBAL: fp32 output
   __nv_bfloat16* dq;     // LOCAL: bf16 output
   DevCtl ctl;
@@ -794,14 +796,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(f[4 * v4], f[4 * v4 + 1], f[4 * v4 + 2], f[4 * v4 + 3]);
           } else {
             if (p.acc_in) {
-              const float4* src = reinterpret_cast<const float4*>(p.acc_in + grow * D + c0);
+              const size_t arow =
+                  p.acc_pooled ? (size_t)bh * g.Np + pooled_of_tiled(g, q_row0 + row) : grow;
+              const float w = p.acc_pooled ? 1.f / (float)(g.pt * g.ph * g.pw) : 1.f;
+              const float4* src = reinterpret_cast<const float4*>(p.acc_in + arow * D + c0);
 #pragma unroll
               for (int v4 = 0; v4 < 8; ++v4) {
                 const float4 a4 = __ldg(src + v4);
-                f[4 * v4] += a4.x;
-                f[4 * v4 + 1] += a4.y;
-                f[4 * v4 + 2] += a4.z;
-                f[4 * v4 + 3] += a4.w;
+                f[4 * v4] += a4.x * w;
+                f[4 * v4 + 1] += a4.y * w;
+                f[4 * v4 + 2] += a4.z * w;
+                f[4 * v4 + 3] += a4.w * w;
               }
             }
             uint4* dst = reinterpret_cast<uint4*>(p.dq + grow * D + c0);
@@ -883,6 +888,7 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   p.nlse2 = global ? a.nlse2_g : a.nlse2_l;
   p.ndelta = global ? a.ndelta_g : a.ndelta_l;
   p.acc_in = (!global && add_acc) ? a.dq_acc : nullptr;
+  p.acc_pooled = a.dq_acc_pooled ? 1 : 0;
   p.acc_out = global ? a.dq_acc : nullptr;
   p.dq = (__nv_bfloat16*)a.dq;
   p.ctl = current_ctl();
@@ -925,6 +931,32 @@ cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual,
   pa.nlse2_g = dual ? a.nlse2_g : nullptr;
   pa.dg = dual ? a.dg : nullptr;
   pa.gvec = dual ? a.g : nullptr;
+  pa.vpr = g.d / 8;
+  pa.N = g.N;
+  pa.heads = g.heads;
+  const int rows_per_block = 256 / pa.vpr;
+  int blocks = (g.N + rows_per_block - 1) / rows_per_block;
+  if (blocks > 64) blocks = 64;
+  bwd::bwd_preprocess_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>(pa);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_preprocess_branch(const DevGeom& g, const void* dout, const void* o, const float* lse,
+                                     const float* gvec, float* ndelta, float* nlse2, cudaStream_t st) {
+  const long long bh = (long long)g.B * g.heads;
+  if (bh == 0 || g.N == 0) return cudaSuccess;
+  bwd::PreArgs pa;
+  pa.dout = (const uint4*)dout;
+  pa.o_l = (const uint4*)o;
+  pa.o_g = nullptr;
+  pa.lse_l = lse;
+  pa.lse_g = nullptr;
+  pa.ndelta_l = ndelta;
+  pa.ndelta_g = nullptr;
+  pa.nlse2_l = nlse2;
+  pa.nlse2_g = nullptr;
+  pa.dg = nullptr;
+  pa.gvec = gvec;
   pa.vpr = g.d / 8;
   pa.N = g.N;
   pa.heads = g.heads;

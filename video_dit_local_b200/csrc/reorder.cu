@@ -174,28 +174,33 @@ struct PoolParams {
   float inv_cnt;
 };
 
+// Up to three tensors pooled in one launch (K and V; or Q, K and V).
+struct PoolTensors {
+  const uint4* src[3];
+  uint4* dst[3];
+  int count;
+};
+
 // One thread produces one 16-byte vector (8 bf16) of one pooled row: the fp32
-// sum of the block's tokens in (t, y, x) order, times 1/count (exact: count is
-// a product of the pool sizes; a power of two at every shipped geometry),
-// one round-to-nearest-even to bf16.
+// sum of the block's tokens in (t, y, x) order, divided by the block size
+// (one correctly rounded fp32 division), one round-to-nearest-even to bf16.
 __global__ void __launch_bounds__(256) pool_kv_kernel(PoolParams p, FastDiv per_row, FastDiv n_prow,
-                                                       const uint4* __restrict__ k, const uint4* __restrict__ v,
-                                                       uint4* __restrict__ kp, uint4* __restrict__ vp,
-                                                       uint32_t rows_per_tensor) {
-  const uint32_t total = 2 * rows_per_tensor * p.vpr;
+                                                       FastDiv rows_per_tensor, PoolTensors ts) {
+  const uint32_t total = (uint32_t)ts.count * rows_per_tensor.d * p.vpr;
   const uint32_t stride = gridDim.x * blockDim.x;
+  const float cnt = (float)(p.pt * p.ph * p.pw);
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
     const uint32_t row2 = per_row.div(i);
     const uint32_t c = i - row2 * p.vpr;
-    const bool is_v = row2 >= rows_per_tensor;
-    const uint32_t row = is_v ? row2 - rows_per_tensor : row2;
+    const uint32_t which = rows_per_tensor.div(row2);
+    const uint32_t row = row2 - which * rows_per_tensor.d;
     const uint32_t bh = n_prow.div(row);
     const uint32_t u = row - bh * p.Np;
     const uint32_t r = p.PW.div(u);
     const uint32_t ux = u - r * p.PWv;
     const uint32_t ut = p.PH.div(r);
     const uint32_t uy = r - ut * p.PHv;
-    const uint4* src = (is_v ? v : k) + (size_t)bh * p.N * p.vpr + c;
+    const uint4* src = ts.src[which] + (size_t)bh * p.N * p.vpr + c;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -212,15 +217,15 @@ __global__ void __launch_bounds__(256) pool_kv_kernel(PoolParams p, FastDiv per_
           }
         }
     uint4 o;
-    o.x = pack_bf16(acc[0] * p.inv_cnt, acc[1] * p.inv_cnt);
-    o.y = pack_bf16(acc[2] * p.inv_cnt, acc[3] * p.inv_cnt);
-    o.z = pack_bf16(acc[4] * p.inv_cnt, acc[5] * p.inv_cnt);
-    o.w = pack_bf16(acc[6] * p.inv_cnt, acc[7] * p.inv_cnt);
-    (is_v ? vp : kp)[(size_t)row * p.vpr + c] = o;
+    o.x = pack_bf16(acc[0] / cnt, acc[1] / cnt);
+    o.y = pack_bf16(acc[2] / cnt, acc[3] / cnt);
+    o.z = pack_bf16(acc[4] / cnt, acc[5] / cnt);
+    o.w = pack_bf16(acc[6] / cnt, acc[7] / cnt);
+    ts.dst[which][(size_t)row * p.vpr + c] = o;
   }
 }
 
-cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void* kp, void* vp, cudaStream_t st) {
+static PoolParams make_pool_params(const DevGeom& g) {
   PoolParams p;
   p.rp = make_params(g);
   p.PW = FastDiv(g.PW);
@@ -234,19 +239,222 @@ cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void*
   p.Np = g.Np;
   p.vpr = g.d / 8;
   p.inv_cnt = 1.0f / (float)(g.pt * g.ph * g.pw);
+  return p;
+}
+
+static cudaError_t pool_tensors(const DevGeom& g, int count, const void* const* src, void* const* dst,
+                                cudaStream_t st) {
+  const PoolParams p = make_pool_params(g);
   const long long per_bh = (long long)g.Np * p.vpr;
   const long long bh_total = (long long)g.B * g.heads;
   if (per_bh * bh_total == 0) return cudaSuccess;
-  const long long chunk = ((1ll << 30) - 1) / per_bh;  // 2 tensors per launch: stay below 2^31 vectors
+  const long long chunk = ((1ll << 31) - 1) / (per_bh * count);  // every launch below 2^31 vectors
   if (chunk < 1) return cudaErrorInvalidValue;
   for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
     const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
     const uint32_t rows = (uint32_t)(nb * g.Np);
     const size_t in_off = (size_t)b0 * g.N * p.vpr, out_off = (size_t)b0 * g.Np * p.vpr;
-    pool_kv_kernel<<<grid_for(2ll * rows * p.vpr, 256), 256, 0, st>>>(
-        p, FastDiv(p.vpr), FastDiv(g.Np), (const uint4*)k + in_off, (const uint4*)v + in_off,
-        (uint4*)kp + out_off, (uint4*)vp + out_off, rows);
+    PoolTensors ts;
+    ts.count = count;
+    for (int i = 0; i < 3; ++i) {
+      const int j = i < count ? i : 0;
+      ts.src[i] = (const uint4*)src[j] + in_off;
+      ts.dst[i] = (uint4*)dst[j] + out_off;
+    }
+    pool_kv_kernel<<<grid_for((long long)count * rows * p.vpr, 256), 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np),
+                                                                                 FastDiv(rows), ts);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void* kp, void* vp, cudaStream_t st) {
+  const void* src[2] = {k, v};
+  void* dst[2] = {kp, vp};
+  return pool_tensors(g, 2, src, dst, st);
+}
+
+cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, const void* v, void* qp, void* kp,
+                            void* vp, cudaStream_t st) {
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qp, kp, vp};
+  return pool_tensors(g, 3, src, dst, st);
+}
+
+// ---------------------------------------------------------------------------
+// Upsampling of the symmetric global branch ("UltraGen ..." §4.2: the
+// compressed latent is brought back to the full grid): separable linear
+// interpolation along t, y, x with half-pixel centres, source coordinate
+// (i + 1/2)/p - 1/2 clamped to the pooled grid.
+// ---------------------------------------------------------------------------
+struct Interp {
+  int i0, i1;
+  float f;  // weight of i1; i0 gets 1 - f
+};
+
+__device__ __forceinline__ Interp interp_of(int i, int p, int n_in) {
+  float src = ((float)i + 0.5f) / (float)p - 0.5f;
+  src = fminf(fmaxf(src, 0.f), (float)(n_in - 1));
+  Interp r;
+  r.i0 = (int)floorf(src);
+  r.i1 = min(r.i0 + 1, n_in - 1);
+  r.f = src - (float)r.i0;
+  return r;
+}
+
+struct UpParams {
+  ReorderParams rp;
+  int N, Np, PT, PH, PW, pt, ph, pw, vpr, heads;
+  int bh_offset;  // batch*head index of the launch's first slice (for g)
+};
+
+// O[tok] = g*O_l[tok] + (1 - g)*upsample(O_p)[tok], tile-major out; one thread
+// per 16-byte vector of an output row.
+__global__ void __launch_bounds__(256) upsample_blend_kernel(UpParams p, FastDiv per_row, FastDiv n_rows,
+                                                              const uint4* __restrict__ op, const uint4* __restrict__ ol,
+                                                              const float* __restrict__ gvec, uint4* __restrict__ out,
+                                                              uint32_t total) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t row = per_row.div(i);
+    const uint32_t c = i - row * p.vpr;
+    const uint32_t bh = n_rows.div(row);
+    const uint32_t m = row - bh * p.N;
+    const uint32_t n = tiled_to_raster(p.rp, m);
+    const uint32_t ty = p.rp.W.div(n);
+    const uint32_t x = n - ty * p.rp.Ww;
+    const uint32_t t = p.rp.H.div(ty);
+    const uint32_t y = ty - t * p.rp.Hh;
+    const Interp it = interp_of(t, p.pt, p.PT), iy = interp_of(y, p.ph, p.PH), ix = interp_of(x, p.pw, p.PW);
+    const uint4* base = op + (size_t)bh * p.Np * p.vpr + c;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const float w = (a ? it.f : 1.f - it.f) * (b ? iy.f : 1.f - iy.f) * (cc ? ix.f : 1.f - ix.f);
+          if (w == 0.f) continue;
+          const int u = ((a ? it.i1 : it.i0) * p.PH + (b ? iy.i1 : iy.i0)) * p.PW + (cc ? ix.i1 : ix.i0);
+          const uint4 v = __ldg(base + (size_t)u * p.vpr);
+          const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += w * bf16lo(vv[e]);
+            acc[2 * e + 1] += w * bf16hi(vv[e]);
+          }
+        }
+    const float gh = gvec[(bh + p.bh_offset) % p.heads];
+    const uint4 l = __ldg(ol + (size_t)row * p.vpr + c);
+    const uint32_t lv[4] = {l.x, l.y, l.z, l.w};
+    uint32_t r[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      r[e] = pack_bf16(gh * bf16lo(lv[e]) + (1.f - gh) * acc[2 * e], gh * bf16hi(lv[e]) + (1.f - gh) * acc[2 * e + 1]);
+    out[(size_t)row * p.vpr + c] = make_uint4(r[0], r[1], r[2], r[3]);
+  }
+}
+
+// dO_p[u] = (1 - g) * sum over full-grid tokens of w(token, u) * dO[token]:
+// the adjoint of the upsampling, gathered per pooled row (bf16 out, fp32 sums).
+// Along a dim the tokens whose stencil reaches pooled index j lie in
+// [j*p - p, j*p + 2p) (clamped); their weights are recomputed here.
+__global__ void __launch_bounds__(256) upsample_transpose_kernel(UpParams p, FastDiv per_row, FastDiv n_rows,
+                                                                  const uint4* __restrict__ dout,
+                                                                  const float* __restrict__ gvec,
+                                                                  uint4* __restrict__ dop, uint32_t total) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t row = per_row.div(i);
+    const uint32_t c = i - row * p.vpr;
+    const uint32_t bh = n_rows.div(row);
+    const int u = (int)(row - bh * p.Np);
+    const int ux = u % p.PW, uy = (u / p.PW) % p.PH, ut = u / (p.PW * p.PH);
+    const uint4* base = dout + (size_t)bh * p.N * p.vpr + c;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const int t0 = max(ut * p.pt - p.pt, 0), t1 = min(ut * p.pt + 2 * p.pt, p.rp.T);
+    const int y0 = max(uy * p.ph - p.ph, 0), y1 = min(uy * p.ph + 2 * p.ph, p.rp.Hh);
+    const int x0 = max(ux * p.pw - p.pw, 0), x1 = min(ux * p.pw + 2 * p.pw, p.rp.Ww);
+    for (int t = t0; t < t1; ++t) {
+      const Interp it = interp_of(t, p.pt, p.PT);
+      const float wt = (it.i0 == ut ? 1.f - it.f : 0.f) + (it.i1 == ut ? it.f : 0.f);
+      if (wt == 0.f) continue;
+      for (int y = y0; y < y1; ++y) {
+        const Interp iy = interp_of(y, p.ph, p.PH);
+        const float wy = (iy.i0 == uy ? 1.f - iy.f : 0.f) + (iy.i1 == uy ? iy.f : 0.f);
+        if (wy == 0.f) continue;
+        for (int x = x0; x < x1; ++x) {
+          const Interp ix = interp_of(x, p.pw, p.PW);
+          const float wx = (ix.i0 == ux ? 1.f - ix.f : 0.f) + (ix.i1 == ux ? ix.f : 0.f);
+          if (wx == 0.f) continue;
+          const float w = wt * wy * wx;
+          const uint32_t m = coords_to_tiled(p.rp, t, y, x);
+          const uint4 v = __ldg(base + (size_t)m * p.vpr);
+          const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += w * bf16lo(vv[e]);
+            acc[2 * e + 1] += w * bf16hi(vv[e]);
+          }
+        }
+      }
+    }
+    const float gg = 1.f - gvec[(bh + p.bh_offset) % p.heads];
+    dop[(size_t)row * p.vpr + c] = make_uint4(pack_bf16(gg * acc[0], gg * acc[1]), pack_bf16(gg * acc[2], gg * acc[3]),
+                                              pack_bf16(gg * acc[4], gg * acc[5]), pack_bf16(gg * acc[6], gg * acc[7]));
+  }
+}
+
+static UpParams make_up_params(const DevGeom& g) {
+  UpParams p;
+  p.rp = make_params(g);
+  p.N = g.N;
+  p.Np = g.Np;
+  p.PT = g.PT;
+  p.PH = g.PH;
+  p.PW = g.PW;
+  p.pt = g.pt;
+  p.ph = g.ph;
+  p.pw = g.pw;
+  p.vpr = g.d / 8;
+  p.heads = g.heads;
+  p.bh_offset = 0;
+  return p;
+}
+
+cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void* o_l, const float* gvec, void* out,
+                                  cudaStream_t st) {
+  const UpParams p = make_up_params(g);
+  const long long per_bh = (long long)g.N * p.vpr, bh_total = (long long)g.B * g.heads;
+  if (per_bh * bh_total == 0) return cudaSuccess;
+  const long long chunk = ((1ll << 31) - 1) / per_bh;
+  if (chunk < 1) return cudaErrorInvalidValue;
+  for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
+    const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
+    const uint32_t total = (uint32_t)(nb * per_bh);
+    const size_t full = (size_t)b0 * g.N * p.vpr, pooled = (size_t)b0 * g.Np * p.vpr;
+    UpParams q = p;
+    q.bh_offset = (int)b0;
+    upsample_blend_kernel<<<grid_for(total, 256), 256, 0, st>>>(q, FastDiv(p.vpr), FastDiv(g.N),
+                                                              (const uint4*)o_p + pooled, (const uint4*)o_l + full,
+                                                              gvec, (uint4*)out + full, total);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_upsample_transpose(const DevGeom& g, const void* dout, const float* gvec, void* dop,
+                                      cudaStream_t st) {
+  const UpParams p = make_up_params(g);
+  const long long per_bh = (long long)g.Np * p.vpr, bh_total = (long long)g.B * g.heads;
+  if (per_bh * bh_total == 0) return cudaSuccess;
+  if (per_bh * bh_total >= (1ll << 31)) return cudaErrorInvalidValue;
+  const uint32_t total = (uint32_t)(per_bh * bh_total);
+  upsample_transpose_kernel<<<grid_for(total, 256), 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np),
+                                                                 (const uint4*)dout, gvec, (uint4*)dop, total);
   return cudaGetLastError();
 }
 

@@ -218,6 +218,47 @@ static BwdWs bwd_ws(const DevGeom& g, bool dual) {
   return w;
 }
 
+struct SymFwdWs {
+  size_t o_l, qp, kp, vp, o_p, total;
+};
+static SymFwdWs sym_fwd_ws(const DevGeom& g) {
+  SymFwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t pooled = align256(bh * g.Np * g.d * 2);
+  w.o_l = 0;
+  w.qp = align256(bh * g.N * g.d * 2);
+  w.kp = w.qp + pooled;
+  w.vp = w.kp + pooled;
+  w.o_p = w.vp + pooled;
+  w.total = w.o_p + pooled;
+  return w;
+}
+struct SymBwdWs {
+  size_t dop, ndelta_l, nlse2_l, ndelta_p, nlse2_p, dkp, dvp, dqp, total;
+};
+static SymBwdWs sym_bwd_ws(const DevGeom& g) {
+  SymBwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t row = align256(bh * g.N * 4), prow = align256(bh * g.Np * 4), pf = align256(bh * g.Np * g.d * 4);
+  w.dop = 0;
+  w.ndelta_l = align256(bh * g.Np * g.d * 2);
+  w.nlse2_l = w.ndelta_l + row;
+  w.ndelta_p = w.nlse2_l + row;
+  w.nlse2_p = w.ndelta_p + prow;
+  w.dkp = w.nlse2_p + prow;
+  w.dvp = w.dkp + pf;
+  w.dqp = w.dvp + pf;
+  w.total = w.dqp + pf;
+  return w;
+}
+
+// The pooled grid seen as a token sequence of its own (queries = pooled rows).
+static DevGeom pooled_as_tokens(const DevGeom& g) {
+  DevGeom p = g;
+  p.N = g.Np;
+  return p;
+}
+
 }  // namespace vattn
 
 using namespace vattn;
@@ -270,6 +311,8 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_DUAL_FWD: *bytes = dual_fwd_ws(g).total; break;
     case VATTN_OP_STA_BWD: *bytes = bwd_ws(g, false).total; break;
     case VATTN_OP_DUAL_BWD: *bytes = bwd_ws(g, true).total; break;
+    case VATTN_OP_DUAL_SYM_FWD: *bytes = sym_fwd_ws(g).total; break;
+    case VATTN_OP_DUAL_SYM_BWD: *bytes = sym_bwd_ws(g).total; break;
     default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
   return ok();
@@ -446,6 +489,137 @@ int vattn_dual_fwd(const vattn_geom* geom, const void* q, const void* k, const v
   b.g = gvec;
   b.blend_out = o;
   CHECK_LAUNCH(launch_attn_fwd(g, FWD_GLOBAL, b, st), "dual_fwd global launch");
+  return ok();
+}
+
+int vattn_dual_sym_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* gvec,
+                       float scale, void* o, void* o_l, float* lse_l, void* qp, void* kp, void* vp, void* o_p,
+                       float* lse_p, void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(gvec);
+  REQUIRE_PTR(o);
+  const int n_saved = (o_l != nullptr) + (lse_l != nullptr) + (qp != nullptr) + (kp != nullptr) + (vp != nullptr) +
+                      (o_p != nullptr) + (lse_p != nullptr);
+  if (n_saved != 0 && n_saved != 7)
+    return fail(VATTN_ERR_INVALID_ARG, "o_l, lse_l, qp, kp, vp, o_p, lse_p must be all NULL or all non-NULL");
+  if (n_saved == 0) {
+    const SymFwdWs w = sym_fwd_ws(g);
+    if (!workspace || ws_bytes < w.total)
+      return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+    if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+    uint8_t* ws = (uint8_t*)workspace;
+    o_l = ws + w.o_l;
+    qp = ws + w.qp;
+    kp = ws + w.kp;
+    vp = ws + w.vp;
+    o_p = ws + w.o_p;
+  } else {
+    REQUIRE_PTR(o_l);
+    REQUIRE_PTR(lse_l);
+    REQUIRE_PTR(qp);
+    REQUIRE_PTR(kp);
+    REQUIRE_PTR(vp);
+    REQUIRE_PTR(o_p);
+    REQUIRE_PTR(lse_p);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_pool_qkv(g, q, k, v, qp, kp, vp, st), "dual_sym_fwd pool launch");
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o_l;
+  a.lse = lse_l;
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "dual_sym_fwd local launch");
+  FwdArgs b{};
+  b.q = qp;
+  b.k = kp;
+  b.v = vp;
+  b.o = o_p;
+  b.lse = lse_p;
+  b.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(pooled_as_tokens(g), FWD_GLOBAL, b, st), "dual_sym_fwd pooled attention launch");
+  CHECK_LAUNCH(launch_upsample_blend(g, o_p, o_l, gvec, o, st), "dual_sym_fwd upsample launch");
+  return ok();
+}
+
+int vattn_dual_sym_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* gvec,
+                       const void* o_l, const float* lse_l, const void* qp, const void* kp, const void* vp,
+                       const void* o_p, const float* lse_p, const void* dout, float scale, void* dq, void* dk,
+                       void* dv, void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(gvec);
+  REQUIRE_PTR(o_l);
+  REQUIRE_PTR(lse_l);
+  REQUIRE_PTR(qp);
+  REQUIRE_PTR(kp);
+  REQUIRE_PTR(vp);
+  REQUIRE_PTR(o_p);
+  REQUIRE_PTR(lse_p);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  const SymBwdWs w = sym_bwd_ws(g);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  uint8_t* ws = (uint8_t*)workspace;
+  void* dop = ws + w.dop;
+  cudaStream_t st = (cudaStream_t)stream;
+  const DevGeom gp = pooled_as_tokens(g);
+  // pooled branch: dO_p = (1-g) * upsample^T(dO), then the pooled attention backward
+  CHECK_LAUNCH(launch_upsample_transpose(g, dout, gvec, dop, st), "dual_sym_bwd upsample^T launch");
+  CHECK_LAUNCH(launch_preprocess_branch(gp, dop, o_p, lse_p, nullptr, (float*)(ws + w.ndelta_p),
+                                        (float*)(ws + w.nlse2_p), st),
+               "dual_sym_bwd pooled preprocess launch");
+  BwdArgs b{};
+  b.q = qp;
+  b.kp = kp;
+  b.vp = vp;
+  b.dout = dop;
+  b.scale = scale;
+  b.ndelta_g = (float*)(ws + w.ndelta_p);
+  b.nlse2_g = (float*)(ws + w.nlse2_p);
+  b.dkp = (float*)(ws + w.dkp);
+  b.dvp = (float*)(ws + w.dvp);
+  b.dq_acc = (float*)(ws + w.dqp);
+  CHECK_LAUNCH(launch_bwd_dkdv_global(gp, b, st), "dual_sym_bwd pooled dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dq_global(gp, b, st), "dual_sym_bwd pooled dq launch");
+  // local branch (gamma = g), with the pooled gradients added through pool^T
+  CHECK_LAUNCH(launch_preprocess_branch(g, dout, o_l, lse_l, gvec, (float*)(ws + w.ndelta_l),
+                                        (float*)(ws + w.nlse2_l), st),
+               "dual_sym_bwd local preprocess launch");
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.dout = dout;
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ndelta_l = (float*)(ws + w.ndelta_l);
+  a.nlse2_l = (float*)(ws + w.nlse2_l);
+  a.dkp = (float*)(ws + w.dkp);
+  a.dvp = (float*)(ws + w.dvp);
+  a.dq_acc = (float*)(ws + w.dqp);
+  a.dq_acc_pooled = true;
+  CHECK_LAUNCH(launch_bwd_dkdv_local(g, a, true, st), "dual_sym_bwd local dk/dv launch");
+  CHECK_LAUNCH(launch_bwd_dq(g, a, true, st), "dual_sym_bwd local dq launch");
   return ok();
 }
 

@@ -49,6 +49,12 @@ cudaError_t launch_permute(const DevGeom& g, const void* src, void* dst, int64_t
                            cudaStream_t st);
 cudaError_t launch_kept_tiles(const DevGeom& g, int32_t* out, cudaStream_t st);
 cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void* kp, void* vp, cudaStream_t st);
+cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, const void* v, void* qp, void* kp,
+                            void* vp, cudaStream_t st);
+cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void* o_l, const float* gvec, void* out,
+                                  cudaStream_t st);
+cudaError_t launch_upsample_transpose(const DevGeom& g, const void* dout, const float* gvec, void* dop,
+                                      cudaStream_t st);
 
 // -- attention forward (attn_fwd.cu) --
 enum FwdMode { FWD_STA = 0, FWD_GLOBAL = 1 };
@@ -93,8 +99,13 @@ struct BwdArgs {
   float* dkp;             // [B,h,Np,d] fp32
   float* dvp;
   float* dq_acc;          // [B,h,N,d] fp32 global-branch part of dQ (dual only)
+  bool dq_acc_pooled;     // dq_acc holds pooled rows [B,h,Np,d]: add dq_acc[pool(tok)] / block size
 };
 cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
+// One branch: -D = -rowsum(dout*o), -L = log2(gamma) - lse*log2(e) with gamma = gvec[h]
+// (gvec NULL: gamma = 1).
+cudaError_t launch_preprocess_branch(const DevGeom& g, const void* dout, const void* o, const float* lse,
+                                     const float* gvec, float* ndelta, float* nlse2, cudaStream_t st);
 cudaError_t launch_bwd_dq(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
 cudaError_t launch_bwd_dq_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
