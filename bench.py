@@ -39,8 +39,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic per launch of the sliding-tile forward kernel at the 720p
 # workload (read+write bytes), and the hash of the kernel source it was taken
 # from.  When the source changes the figure is stale and reported as null.
-STA_FWD_TRAFFIC = 2692600000  # bytes per launch, from profiles/sta_fwd_720p.md (2-head capture x 12)
-STA_FWD_TRAFFIC_SRC_SHA = "c50b52bee3199efa"
+STA_FWD_TRAFFIC = 2689440768  # bytes per launch, from profiles/sta_fwd_720p.md (2-head capture x 12)
+STA_FWD_TRAFFIC_SRC_SHA = "8011bf150a2117ef"
 
 
 def reduce_max(values, world: int, device=None):
@@ -276,25 +276,40 @@ def run_ours(args, rank, world, local_rank):
     o_host = torch.empty(shape, dtype=torch.bfloat16, pin_memory=True)
     lse_host = torch.empty(shape[:3], dtype=torch.float32, pin_memory=True)
 
-    def e2e_step():
+    def serial_step():   # copies, then the device step, then copies, on one stream
         for p, dst in zip(pinned, (qr, kr, vr)):
             dst.view(torch.int16).copy_(p, non_blocking=True)
         step()
         o_host.copy_(o_r, non_blocking=True)
         lse_host.copy_(lse_r, non_blocking=True)
 
+    # the library's pipelined host-buffer entry point: chunks of batch*head
+    # slices, copies in both directions overlapping the compute
+    chunk = min(args.e2e_chunk, w.batch * w.heads)
+    one = V.make_geom(1, chunk, w.head_dim, w.grid, w.tile, w.window, w.pool)
+    host_ws = torch.empty(2 * V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, one), dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        V.vattn_sta_fwd_host(geom, pinned[0], pinned[1], pinned[2], scale, o_host, lse_host, chunk, host_ws)
+
+    def time_steps(fn, n):
+        fn()
+        torch.cuda.synchronize()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n):
+            fn()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        return reduce_max([a0.elapsed_time(a1) / n], world, dev)[0]
+
     e2e_steps = max(3, min(args.steps, 10))
-    e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    a1.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = a0.elapsed_time(a1) / e2e_steps
-    ms_e2e = reduce_max([ms_e2e], world, dev)[0]
+    ms_e2e = time_steps(e2e_step, e2e_steps)
+    if V.vattn_get_status() != 0:
+        raise RuntimeError("device status after the host-buffer steps: " + V.vattn_last_error())
+    ms_serial = time_steps(serial_step, e2e_steps)
+    del host_ws
     h2d = sum(p.numel() * p.element_size() for p in pinned)
     d2h = o_host.numel() * 2 + lse_host.numel() * 4
 
@@ -326,7 +341,9 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "attn_fwd_kernel<128> (sliding tile)", "kernel_ms": round(ms_kernel, 4),
                      "algorithmic_flop_per_launch": flops_local},
         "e2e": {"value": round(whole_job_tflops(flops_local, ms_e2e, world), 2), "unit": "TFLOP/s",
-                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "call": f"vattn_sta_fwd_host, pinned host buffers, chunks of {chunk} slices",
+                "serial_ms_per_step": round(ms_serial, 3)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
@@ -599,6 +616,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--e2e-chunk", type=int, default=3, help="batch*head slices per host-copy chunk (e2e)")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: fewer heads than the workload")
     ap.add_argument("--workload", choices=["720p", "train"], default="720p",
                     help="720p: the benchmark line; train: profiling of the training step alone")

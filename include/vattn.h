@@ -79,7 +79,8 @@ enum {
   VATTN_OP_STA_BWD = 2,
   VATTN_OP_DUAL_BWD = 3,
   VATTN_OP_DUAL_SYM_FWD = 4,
-  VATTN_OP_DUAL_SYM_BWD = 5
+  VATTN_OP_DUAL_SYM_BWD = 5,
+  VATTN_OP_STA_FWD_HOST = 6  /* per chunk of batch*head slices: pass heads = the chunk size in geom */
 };
 
 /* Raster -> tile-major row gather.  Tile-major position of raster token
@@ -128,6 +129,23 @@ int vattn_xwin_fwd(const vattn_geom* geom, int shifted, const void* q, const voi
 int vattn_xwin_bwd(const vattn_geom* geom, int shifted, const void* q, const void* k, const void* v,
                    const void* o, const float* lse, const void* dout, float scale, void* dq, void* dk,
                    void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Sliding-tile forward on HOST buffers in raster order, pipelined.  The
+ * batch*head range is cut into chunks of `chunk_slices` slices; for every
+ * chunk the host->device copy of Q, K, V, the permute + vattn_sta_fwd +
+ * unpermute, and the device->host copy of O (and LSE) run on three library
+ * streams, so that copies in both directions overlap the compute of the
+ * neighbouring chunks (two staging slots, reused in turn).
+ *  q, k, v : host bf16 [B,h,N,d] raster; o: host bf16 raster; lse: host fp32
+ *            [B,h,N] raster or NULL.  Pinned host memory gives full overlap.
+ *  workspace: device memory, >= 2 * vattn_workspace_size(VATTN_OP_STA_FWD_HOST)
+ *            computed on a geometry whose heads = chunk_slices and batch = 1.
+ *  The work is ordered after earlier work on `stream`, and `stream` is made
+ *  to wait for all of it: synchronise `stream` before reading o / lse.
+ *  Calls from several host threads on one device are serialised. */
+int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale,
+                       void* o, float* lse, int64_t chunk_slices, void* workspace, size_t ws_bytes,
+                       void* stream);
 
 /* Average pooling of K and V over p_t x p_h x p_w token blocks ("UltraGen ..."
  * §4.2: latents downsampled before global attention).  Inputs tile-major

@@ -78,6 +78,15 @@ def test_argument_errors(V):
         V.vattn_dual_fwd(g, 16, 16, 16, 16, 0.1, 16, workspace=32, ws_bytes=8)
     assert e.value.code == B.VATTN_ERR_WORKSPACE
     with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd_host(g, 16, 16, 16, 0.1, 16, 0, 0, 32, 1 << 30)    # chunk of zero slices
+    assert e.value.code == B.VATTN_ERR_INVALID_ARG
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd_host(g, 16, 16, 16, 0.1, 16, 0, 3, 32, 1 << 30)    # more slices than batch*heads
+    assert e.value.code == B.VATTN_ERR_INVALID_ARG
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd_host(g, 16, 16, 16, 0.1, 16, 0, 1, 32, 64)         # two slots needed
+    assert e.value.code == B.VATTN_ERR_WORKSPACE
+    with pytest.raises(V.VattnError) as e:
         V.vattn_workspace_size(99, g)
     assert e.value.code == B.VATTN_ERR_INVALID_ARG
 
@@ -96,6 +105,8 @@ def test_workspace_sizes(V):
         return (x + 255) // 256 * 256
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, g) == a(bh * n * d * 2) + 2 * a(bh * npool * d * 2)
     assert V.vattn_workspace_size(V.VATTN_OP_STA_BWD, g) == 2 * a(bh * n * 4)
+    # host-buffer forward, per slot: 8 bf16 token tensors and 2 fp32 rows
+    assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, g) == 8 * a(bh * n * d * 2) + 2 * a(bh * n * 4)
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == (4 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)
                                                               + a(bh * n * d * 4))
 

@@ -252,6 +252,57 @@ static SymBwdWs sym_bwd_ws(const DevGeom& g) {
   return w;
 }
 
+// Device staging of one chunk of the host-buffer forward: raster Q, K, V,
+// tile-major Q, K, V, O, LSE, and raster O, LSE.
+struct HostChunkWs {
+  size_t qr, kr, vr, qt, kt, vt, ot, lt, orr, lr, total;
+};
+static HostChunkWs host_chunk_ws(const DevGeom& g) {
+  HostChunkWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t t = align256(bh * g.N * g.d * 2), l = align256(bh * g.N * 4);
+  w.qr = 0;
+  w.kr = t;
+  w.vr = 2 * t;
+  w.qt = 3 * t;
+  w.kt = 4 * t;
+  w.vt = 5 * t;
+  w.ot = 6 * t;
+  w.orr = 7 * t;
+  w.lt = 8 * t;
+  w.lr = 8 * t + l;
+  w.total = 8 * t + 2 * l;
+  return w;
+}
+
+// Library streams and events of the host-buffer pipeline, one set per device.
+struct HostPipe {
+  cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+  std::mutex mu;
+  bool ready = false;
+};
+static HostPipe* host_pipe(int dev) {
+  static HostPipe pipes[64];
+  if (dev < 0 || dev >= 64) return nullptr;
+  return &pipes[dev];
+}
+static cudaError_t host_pipe_init(HostPipe& p) {
+  if (p.ready) return cudaSuccess;
+  cudaError_t e;
+  if ((e = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+  if ((e = cudaStreamCreateWithFlags(&p.comp, cudaStreamNonBlocking)) != cudaSuccess) return e;
+  if ((e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+  if ((e = cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming)) != cudaSuccess) return e;
+  for (int i = 0; i < 2; ++i) {
+    if ((e = cudaEventCreateWithFlags(&p.in_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&p.comp_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&p.out_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  p.ready = true;
+  return cudaSuccess;
+}
+
 // The pooled grid seen as a token sequence of its own (queries = pooled rows).
 static DevGeom pooled_as_tokens(const DevGeom& g) {
   DevGeom p = g;
@@ -313,6 +364,7 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_DUAL_BWD: *bytes = bwd_ws(g, true).total; break;
     case VATTN_OP_DUAL_SYM_FWD: *bytes = sym_fwd_ws(g).total; break;
     case VATTN_OP_DUAL_SYM_BWD: *bytes = sym_bwd_ws(g).total; break;
+    case VATTN_OP_STA_FWD_HOST: *bytes = host_chunk_ws(g).total; break;
     default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
   return ok();
@@ -396,6 +448,82 @@ int vattn_xwin_fwd(const vattn_geom* geom, int shifted, const void* q, const voi
   a.lse = lse;
   a.scale = scale;
   CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, (cudaStream_t)stream), "xwin_fwd launch");
+  return ok();
+}
+
+int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                       float* lse, int64_t chunk_slices, void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  if (!q || !k || !v || !o) return fail(VATTN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL host pointers");
+  const long long total = (long long)g.B * g.heads;
+  if (chunk_slices <= 0 || chunk_slices > total) return fail(VATTN_ERR_INVALID_ARG, "chunk_slices out of range");
+  DevGeom gc = g;  // one chunk: batch 1, heads = chunk_slices (the attention path has no per-head state here)
+  gc.B = 1;
+  gc.heads = (int)chunk_slices;
+  const HostChunkWs w = host_chunk_ws(gc);
+  if (!workspace || ws_bytes < 2 * w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", 2 * w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  int dev = 0;
+  CHECK_LAUNCH(cudaGetDevice(&dev), "cudaGetDevice");
+  HostPipe* pp = host_pipe(dev);
+  if (!pp) return fail(VATTN_ERR_UNSUPPORTED, "device index out of range");
+  std::lock_guard<std::mutex> lk(pp->mu);
+  CHECK_LAUNCH(host_pipe_init(*pp), "pipeline stream/event creation");
+  HostPipe& p = *pp;
+  cudaStream_t caller = (cudaStream_t)stream;
+  CHECK_LAUNCH(cudaEventRecord(p.start, caller), "event record");
+  CHECK_LAUNCH(cudaStreamWaitEvent(p.in, p.start, 0), "stream wait");
+  CHECK_LAUNCH(cudaStreamWaitEvent(p.comp, p.start, 0), "stream wait");
+  CHECK_LAUNCH(cudaStreamWaitEvent(p.out, p.start, 0), "stream wait");
+  const size_t row = (size_t)g.N * g.d * 2, lrow = (size_t)g.N * 4;
+  const int nchunks = (int)((total + chunk_slices - 1) / chunk_slices);
+  for (int c = 0; c < nchunks; ++c) {
+    const int slot = c & 1;
+    const long long s0 = (long long)c * chunk_slices;
+    const long long ns = total - s0 < chunk_slices ? total - s0 : chunk_slices;
+    DevGeom gk = gc;
+    gk.heads = (int)ns;
+    uint8_t* ws = (uint8_t*)workspace + slot * w.total;
+    // the slot's inputs are free once the compute two chunks back is done; its
+    // outputs once that chunk's copy-out is done
+    if (c >= 2) {
+      CHECK_LAUNCH(cudaStreamWaitEvent(p.in, p.comp_done[slot], 0), "stream wait");
+      CHECK_LAUNCH(cudaStreamWaitEvent(p.comp, p.out_done[slot], 0), "stream wait");
+    }
+    const size_t bytes = (size_t)ns * row;
+    CHECK_LAUNCH(cudaMemcpyAsync(ws + w.qr, (const uint8_t*)q + s0 * row, bytes, cudaMemcpyHostToDevice, p.in), "H2D q");
+    CHECK_LAUNCH(cudaMemcpyAsync(ws + w.kr, (const uint8_t*)k + s0 * row, bytes, cudaMemcpyHostToDevice, p.in), "H2D k");
+    CHECK_LAUNCH(cudaMemcpyAsync(ws + w.vr, (const uint8_t*)v + s0 * row, bytes, cudaMemcpyHostToDevice, p.in), "H2D v");
+    CHECK_LAUNCH(cudaEventRecord(p.in_done[slot], p.in), "event record");
+    CHECK_LAUNCH(cudaStreamWaitEvent(p.comp, p.in_done[slot], 0), "stream wait");
+    CHECK_LAUNCH(launch_permute(gk, ws + w.qr, ws + w.qt, g.d * 2, true, p.comp), "permute q");
+    CHECK_LAUNCH(launch_permute(gk, ws + w.kr, ws + w.kt, g.d * 2, true, p.comp), "permute k");
+    CHECK_LAUNCH(launch_permute(gk, ws + w.vr, ws + w.vt, g.d * 2, true, p.comp), "permute v");
+    FwdArgs a{};
+    a.q = ws + w.qt;
+    a.k = ws + w.kt;
+    a.v = ws + w.vt;
+    a.o = ws + w.ot;
+    a.lse = lse ? (float*)(ws + w.lt) : nullptr;
+    a.scale = scale;
+    CHECK_LAUNCH(launch_attn_fwd(gk, FWD_STA, a, p.comp), "sta_fwd");
+    CHECK_LAUNCH(launch_permute(gk, ws + w.ot, ws + w.orr, g.d * 2, false, p.comp), "unpermute o");
+    if (lse) CHECK_LAUNCH(launch_permute(gk, ws + w.lt, ws + w.lr, 4, false, p.comp), "unpermute lse");
+    CHECK_LAUNCH(cudaEventRecord(p.comp_done[slot], p.comp), "event record");
+    CHECK_LAUNCH(cudaStreamWaitEvent(p.out, p.comp_done[slot], 0), "stream wait");
+    CHECK_LAUNCH(cudaMemcpyAsync((uint8_t*)o + s0 * row, ws + w.orr, bytes, cudaMemcpyDeviceToHost, p.out), "D2H o");
+    if (lse)
+      CHECK_LAUNCH(cudaMemcpyAsync((uint8_t*)lse + s0 * lrow, ws + w.lr, (size_t)ns * lrow, cudaMemcpyDeviceToHost, p.out),
+                   "D2H lse");
+    CHECK_LAUNCH(cudaEventRecord(p.out_done[slot], p.out), "event record");
+  }
+  // the caller's stream waits for every copy-out (and therefore for everything)
+  for (int slot = 0; slot < 2 && slot < nchunks; ++slot)
+    CHECK_LAUNCH(cudaStreamWaitEvent(caller, p.out_done[slot], 0), "stream wait");
   return ok();
 }
 
