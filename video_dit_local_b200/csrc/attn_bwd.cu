@@ -206,7 +206,7 @@ struct DkdvSmem {
   static constexpr int OFF_LSE = OFF_DO + NQ * QB_BYTES;
   static constexpr int OFF_DEL = OFF_LSE + NQ * 256;
   static constexpr int OFF_BAR = OFF_DEL + NQ * 256;
-  static constexpr int NBAR = 1 + 4 * NQ + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 2 * NQ + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int TOTAL = OFF_MISC + 16;
   static constexpr int ALLOC = TOTAL + 1024;
@@ -242,11 +242,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = q_full + NQ;
-  uint64_t* do_full = q_empty + NQ;
-  uint64_t* do_empty = do_full + NQ;
-  uint64_t* sdp_full = do_empty + NQ;
+  // One full / empty pair per query stage for Q, dO and the L / D rows: the two
+  // loader warps each arrive (with their byte counts) on the same full
+  // barrier, and one commit releases the whole stage.  Every barrier wait or
+  // commit costs the MMA thread about as long as an MMA, and the tensor pipe
+  // holds little more than one MMA in flight, so fewer of them per block keep
+  // the pipe busier.
+  uint64_t* qd_full = bars + 1;
+  uint64_t* qd_empty = qd_full + NQ;
+  uint64_t* sdp_full = qd_empty + NQ;
   uint64_t* p_full = sdp_full + 2;
   uint64_t* acc_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -281,10 +285,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int i = 0; i < NQ; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
-      mbar_init(&do_full[i], 1);
-      mbar_init(&do_empty[i], 1);
+      mbar_init(&qd_full[i], 2);  // one arrival per loader warp
+      mbar_init(&qd_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sdp_full[i], 1);
@@ -317,8 +319,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_3d(smem + L::OFF_V + c * KBOX, &tm_v, kv_full, c * 64, key_row0, bh);
         }
       }
-      uint64_t* full = is_a ? q_full : do_full;
-      uint64_t* empty = is_a ? q_empty : do_empty;
+      uint64_t* full = qd_full;
+      uint64_t* empty = qd_empty;
       const CUtensorMap* tm = is_a ? &tm_q : &tm_do;
       const float* vec = is_a ? p.nlse2 : p.ndelta;
       float* vec_s = is_a ? lse_s : del_s;
@@ -368,8 +370,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool ok = mbar_wait(kv_full, 0, wc);
       auto issue_sdp = [&](int i) -> bool {
         const int s = i % NQ, w = i & 1;
-        if (!mbar_wait(&q_full[s], (i / NQ) & 1, wc)) return false;
-        if (!mbar_wait(&do_full[s], (i / NQ) & 1, wc)) return false;
+        if (!mbar_wait(&qd_full[s], (i / NQ) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t qb = q_base + s * L::QB_BYTES, db = do_base + s * L::QB_BYTES;
 #pragma unroll
@@ -398,8 +399,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_ts(tmem + 384, tmem + 128 + w * 64 + kk * 8, smem_desc_sw128(qb + kk * 2048, QBOX, 1024), IDESC_ACC,
                  (i > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&q_empty[s]);
-        tc_commit(&do_empty[s]);
+        tc_commit(&qd_empty[s]);
         if (i + 2 < nblk) ok = issue_sdp(i + 2);
       }
       tc_commit(acc_done);
@@ -415,8 +415,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = w; i < nblk; i += 2) {
       const int it = i >> 1, s = i % NQ;
       ok = mbar_wait(&sdp_full[w], it & 1, wc);
-      ok = ok && mbar_wait(&q_full[s], (i / NQ) & 1, wc);    // L rows in shared memory
-      ok = ok && mbar_wait(&do_full[s], (i / NQ) & 1, wc);   // D rows in shared memory
+      ok = ok && mbar_wait(&qd_full[s], (i / NQ) & 1, wc);   // L and D rows in shared memory
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -553,7 +552,8 @@ struct DqSmem {
   static constexpr int OFF_K = 2 * QB_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KB_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * KB_BYTES;
-  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 1;
+  static_assert(NK == NV, "K and V stages share their barriers");
+  static constexpr int NBAR = 1 + 2 * NK + 2 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int TOTAL = OFF_MISC + 16;
   static constexpr int ALLOC = TOTAL + 1024;
@@ -591,11 +591,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* qdo_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + NK;
-  uint64_t* v_full = k_empty + NK;
-  uint64_t* v_empty = v_full + NV;
-  uint64_t* sdp_full = v_empty + NV;
+  // K and V of key block j share stage j % NK: one full barrier that both
+  // loader warps arrive on, and one empty barrier committed after the dQ
+  // product (the last reader of K) -- one wait and one commit per block
+  // fewer for the MMA thread.
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + NK;
+  uint64_t* sdp_full = kv_empty + NK;
   uint64_t* p_full = sdp_full + 2;
   uint64_t* acc_done = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -627,12 +629,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(qdo_full, 1);
     for (int i = 0; i < NK; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-    }
-    for (int i = 0; i < NV; ++i) {
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
+      mbar_init(&kv_full[i], 2);  // one arrival per loader warp
+      mbar_init(&kv_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sdp_full[i], 1);
@@ -665,8 +663,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       const int NS = is_k ? NK : NV;
-      uint64_t* full = is_k ? k_full : v_full;
-      uint64_t* empty = is_k ? k_empty : v_empty;
+      uint64_t* full = kv_full;
+      uint64_t* empty = kv_empty;
       const uint32_t off = is_k ? L::OFF_K : L::OFF_V;
       int issued = 0;
       for (int j = 0; j < nblk; ++j) {
@@ -695,9 +693,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t k_base = smem_u32(smem + L::OFF_K), v_base = smem_u32(smem + L::OFF_V);
       bool ok = mbar_wait(qdo_full, 0, wc);
       auto issue_sdp = [&](int j) -> bool {
-        const int w = j & 1, sk = j % NK, sv = j % NV;
-        if (!mbar_wait(&k_full[sk], (j / NK) & 1, wc)) return false;
-        if (!mbar_wait(&v_full[sv], (j / NV) & 1, wc)) return false;
+        const int w = j & 1, sk = j % NK, sv = sk;
+        if (!mbar_wait(&kv_full[sk], (j / NK) & 1, wc)) return false;
         tc_fence_after();
         const uint32_t kb = k_base + sk * L::KB_BYTES, vb = v_base + sv * L::KB_BYTES;
 #pragma unroll
@@ -708,7 +705,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_ss(tmem + (w ? DQ_P1 : DQ_P0), smem_desc_sw128(do_base + qo, 16, 1024),
                  smem_desc_sw128(vb + ko, 16, 1024), IDESC_S, kk > 0);
         }
-        tc_commit(&v_empty[sv]);
         tc_commit(&sdp_full[w]);
         return true;
       };
@@ -723,7 +719,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int kk = 0; kk < DQ_BN / 16; ++kk)
           mma_ts(tmem + DQ_ACC, tmem + (w ? DQ_P1 : DQ_P0) + kk * 8, smem_desc_sw128(kb + kk * 2048, KBOX, 1024),
                  IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&k_empty[sk]);
+        tc_commit(&kv_empty[sk]);
         if (j + 2 < nblk) ok = issue_sdp(j + 2);
       }
       tc_commit(acc_done);
