@@ -49,7 +49,7 @@ struct Smem {
   static constexpr int OFF_K = OFF_Q + BLOCK_BYTES;
   static constexpr int OFF_V = OFF_K + NK * BLOCK_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * BLOCK_BYTES;
-  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_XCH = OFF_MISC + 16;
   static constexpr int TOTAL = OFF_XCH + 2 * 128 * 2 * 4;
@@ -116,11 +116,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + NK;
-  uint64_t* v_full = k_empty + NK;
+  // qk_done[j % NK] completes when Q*K_j^T is done: it tells softmax group
+  // j & 1 that S_j is in TMEM and the K loader that stage j % NK is free.  Both
+  // wait for a phase before the barrier can complete the next one (block j+3
+  // needs K_{j+3}, loaded after the loader's wait, and its Q*K^T is issued
+  // after P_j, produced after the group's wait), so one commit serves both.
+  uint64_t* qk_done = k_full + NK;
+  uint64_t* v_full = qk_done + NK;
   uint64_t* v_empty = v_full + NV;
-  uint64_t* s_full = v_empty + NV;
-  uint64_t* p_full = s_full + 2;
+  uint64_t* p_full = v_empty + NV;
   uint64_t* o_final = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
@@ -155,14 +159,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(q_full, 1);
     for (int i = 0; i < NK; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
+      mbar_init(&qk_done[i], 1);
     }
     for (int i = 0; i < NV; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);  // one arrival per softmax warp
     }
     mbar_init(o_final, 1);
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NK, r = j / NK;
-        if (!mbar_wait(&k_empty[s], (r & 1) ^ 1, wc)) break;
+        if (!mbar_wait(&qk_done[s], (r & 1) ^ 1, wc)) break;
         mbar_arrive_expect_tx(&k_full[s], L::BLOCK_BYTES);
         uint8_t* dst = smem + L::OFF_K + s * L::BLOCK_BYTES;
         for (int u = 0; u < subs; ++u) {
@@ -254,8 +257,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
                  kk > 0);
         }
-        tc_commit(&k_empty[s]);
-        tc_commit(&s_full[j & 1]);
+        tc_commit(&qk_done[s]);
         return true;
       };
       if (ok) ok = issue_qk(0);
@@ -292,11 +294,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tO = tmem + lane_addr + 256u + (uint32_t)(w * 128);
     const float c2 = p.scale_log2;
     float m_ref = -INFINITY, l_sum = 0.f;
+    int qs = w;          // qk_done stage of this group's next block (j % NK) ...
+    uint32_t qph = 0;    // ... and its phase parity ((j / NK) & 1)
     bool ok = true;
     for (int i = 0;; ++i) {
       const int j = 2 * i + w;
       if (j >= nblk) break;
-      ok = mbar_wait(&s_full[w], i & 1, wc);
+      ok = mbar_wait(&qk_done[qs], qph, wc);
+      qs += 2;  // next block of this group: j + 2
+      if (qs >= NK) {
+        qs -= NK;
+        qph ^= 1u;
+      }
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
