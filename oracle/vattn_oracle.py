@@ -635,3 +635,103 @@ def dual_sym_backward(q, k, v, gvec, do, g: Geom, scale: float):
     dqp, dkp, dvp = global_backward(qp, kp, vp, do_p, scale)
     return dict(dQ=dq_l + pool_transpose(dqp, g), dK=dk_l + pool_transpose(dkp, g),
                 dV=dv_l + pool_transpose(dvp, g), dQ_p=dqp, dK_p=dkp, dV_p=dvp)
+
+
+# ---------------------------------------------------------------------------
+# NEXT-2: hierarchical local attention ("UltraGen ..." §4.3, hierarchical local
+# attention: intermediate-scale attention over coarse windows).  Reading: the
+# local branch also sees K and V average-pooled by a medium factor h_pool,
+# through a window of coarse tiles -- the pooled grid cut into tiles of the
+# same shape, one coarse tile covering h_pool fine tiles per dim -- around the
+# coarse tile that holds the query tile; fine and coarse keys share one
+# softmax.
+# ---------------------------------------------------------------------------
+
+def hier_geom(g: Geom, hpool: tuple) -> Geom:
+    """The medium-pooled grid with the fine tile shape and window (its tiles
+    are the coarse tiles)."""
+    pt, ph, pw = hpool
+    return Geom(g.T // pt, g.H // ph, g.W // pw, g.tile, g.window)
+
+
+def coarse_tile_of(a: tuple, hpool: tuple) -> tuple:
+    """Coarse tile holding fine tile a: a coarse tile spans h_pool fine tiles
+    per dim (the same tile shape over a grid pooled by h_pool)."""
+    return tuple(x // p for x, p in zip(a, hpool))
+
+
+def _hier_query_tiles(g: Geom, hpool: tuple):
+    """Yield (query ids, fine key ids, coarse key ids) per query tile: raster
+    ids in the fine grid, and in the medium-pooled grid for the coarse keys."""
+    gc = hier_geom(g, hpool)
+    ncd = gc.tiles_per_dim
+    nt, nh, nw = g.tiles_per_dim
+    fine = _query_tiles(g)
+    for at in range(nt):
+        for ah in range(nh):
+            for aw in range(nw):
+                qi, kj = next(fine)
+                c = coarse_tile_of((at, ah, aw), hpool)
+                r = [window_range(c[ax], g.window[ax], ncd[ax]) for ax in range(3)]
+                kc = _tile_token_box(gc, (r[0].start, r[1].start, r[2].start), (r[0].stop, r[1].stop, r[2].stop))
+                yield qi, kj, kc
+
+
+def hier_attention(q, k, v, g: Geom, hpool: tuple, scale: float):
+    """Joint softmax over each query tile's fine sliding-tile keys and its
+    coarse-window medium-pooled keys.  Raster in and out: (O, LSE)."""
+    gh = g._replace(pool=tuple(hpool))
+    kh, vh = pool(k, gh), pool(v, gh)
+    B, nh, n, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, nh, n))
+    for b in range(B):
+        for h in range(nh):
+            for qi, kj, kc in _hier_query_tiles(g, hpool):
+                keys = np.concatenate([k[b, h, kj], kh[b, h, kc]])
+                vals = np.concatenate([v[b, h, kj], vh[b, h, kc]])
+                o[b, h, qi], lse[b, h, qi], _ = _softmax_attend(q[b, h, qi], keys, vals, scale)
+    return o, lse
+
+
+def hier_backward(q, k, v, do, g: Geom, hpool: tuple, scale: float):
+    """Gradients of hier_attention w.r.t. q, k, v (the coarse keys' gradients
+    flow back through the medium pooling)."""
+    gh = g._replace(pool=tuple(hpool))
+    kh, vh = pool(k, gh), pool(v, gh)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dkh = np.zeros_like(kh)
+    dvh = np.zeros_like(vh)
+    B, nh = q.shape[:2]
+    for b in range(B):
+        for h in range(nh):
+            for qi, kj, kc in _hier_query_tiles(g, hpool):
+                keys = np.concatenate([k[b, h, kj], kh[b, h, kc]])
+                vals = np.concatenate([v[b, h, kj], vh[b, h, kc]])
+                a, dkeys, dvals = _softmax_attend_bwd(q[b, h, qi], keys, vals, do[b, h, qi], scale)
+                nf = len(kj)
+                dq[b, h, qi] += a
+                dk[b, h, kj] += dkeys[:nf]
+                dv[b, h, kj] += dvals[:nf]
+                dkh[b, h, kc] += dkeys[nf:]
+                dvh[b, h, kc] += dvals[nf:]
+    return dq, dk + pool_transpose(dkh, gh), dv + pool_transpose(dvh, gh)
+
+
+def hier_attention_tiles(q, k, v, g: Geom, hpool: tuple, scale: float, tile_ids):
+    """hier_attention for the listed query tiles of one head (2-D q, k, v):
+    returns (raster query ids, O rows, LSE rows)."""
+    gh = g._replace(pool=tuple(hpool))
+    kh, vh = pool(k, gh), pool(v, gh)
+    want = set(int(t) for t in tile_ids)
+    ids, os_, ls_ = [], [], []
+    for t, (qi, kj, kc) in enumerate(_hier_query_tiles(g, hpool)):
+        if t not in want:
+            continue
+        o, l, _ = _softmax_attend(q[qi], np.concatenate([k[kj], kh[kc]]), np.concatenate([v[kj], vh[kc]]), scale)
+        ids.append(qi)
+        os_.append(o)
+        ls_.append(l)
+    return np.concatenate(ids), np.concatenate(os_), np.concatenate(ls_)

@@ -516,3 +516,119 @@ def test_sampled_symmetric_backward_equals_full():
                                 symmetric=True)
     for key, ids in (("dQ", "q_ids"), ("dK", "k_ids"), ("dV", "k_ids")):
         assert np.abs(s[key] - full[key][0, 0][s[ids]]).max() < 1e-12
+
+
+# ---------------------------------------------------------------- hierarchical local attention (NEXT-2)
+
+def _pool_reshape(x, g, hp):
+    """Independent block mean by reshape: [..., N, d] raster -> [..., N_h, d]."""
+    lead, d = x.shape[:-2], x.shape[-1]
+    y = x.reshape(lead + (g.T // hp[0], hp[0], g.H // hp[1], hp[1], g.W // hp[2], hp[2], d))
+    return y.mean(axis=(-6, -4, -2)).reshape(lead + (-1, d))
+
+
+def _hier_brute_mask(g, hp):
+    """[N, N + N_h] visibility built token by token from coordinates: the fine
+    part is the sliding-tile mask; pooled key j is visible to query i iff j's
+    coarse tile (its pooled coordinates // tile) lies in the clamped window of
+    the coarse tile holding i's fine tile (fine tile coordinates // h_pool)."""
+    fine = _brute_mask(g)
+    dims_p = (g.T // hp[0], g.H // hp[1], g.W // hp[2])
+    nc = tuple(dp // t for dp, t in zip(dims_p, g.tile))
+    cq = []
+    for n in range(g.n):
+        t, rem = divmod(n, g.H * g.W)
+        y, x = divmod(rem, g.W)
+        cq.append((t // g.tile[0] // hp[0], y // g.tile[1] // hp[1], x // g.tile[2] // hp[2]))
+    ck = []
+    for j in range(math.prod(dims_p)):
+        t, rem = divmod(j, dims_p[1] * dims_p[2])
+        y, x = divmod(rem, dims_p[2])
+        ck.append((t // g.tile[0], y // g.tile[1], x // g.tile[2]))
+    wins = [[_brute_window(a, g.window[ax], nc[ax]) for a in range(nc[ax])] for ax in range(3)]
+    coarse = np.zeros((g.n, len(ck)), dtype=bool)
+    for i, c in enumerate(cq):
+        for j, e in enumerate(ck):
+            coarse[i, j] = all(e[ax] in wins[ax][c[ax]] for ax in range(3))
+    return np.concatenate([fine, coarse], axis=1)
+
+
+HIER_CASES = [
+    (O.Geom(4, 16, 32, (2, 4, 4), (1, 3, 3)), (1, 2, 2)),   # coarse window clamps along W only
+    (O.Geom(4, 16, 16, (1, 4, 4), (3, 1, 1)), (2, 2, 2)),   # pooled in time as well
+]
+
+
+@pytest.mark.parametrize("g,hp", HIER_CASES)
+def test_hier_equals_independent_masked_softmax(g, hp):
+    q, k, v = (_rand((1, 2, g.n, 16), s) for s in (41, 42, 43))
+    o, lse = O.hier_attention(q, k, v, g, hp, 0.3)
+    keys = np.concatenate([k, _pool_reshape(k, g, hp)], axis=2)
+    vals = np.concatenate([v, _pool_reshape(v, g, hp)], axis=2)
+    mask = _hier_brute_mask(g, hp)
+    np.testing.assert_allclose(o, _sdpa(q, keys, vals, 0.3, mask), rtol=0, atol=1e-12)
+    s = np.einsum("bhnd,bhmd->bhnm", q, keys) * 0.3
+    ref_lse = np.log(np.where(mask, np.exp(s), 0.0).sum(-1))
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_hier_pool_one_duplicates_every_local_key():
+    """With h_pool = 1 the coarse keys are the fine keys again: each key counts
+    twice, so O is the sliding-tile O and the LSE grows by exactly ln 2."""
+    g = O.Geom(4, 8, 16, (2, 4, 4), (1, 1, 3))
+    q, k, v = (_rand((2, 1, g.n, 8), s) for s in (44, 45, 46))
+    o, lse = O.hier_attention(q, k, v, g, (1, 1, 1), 0.5)
+    o_l, lse_l = O.sta_attention(q, k, v, g, 0.5)
+    np.testing.assert_allclose(o, o_l, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_l + math.log(2.0), rtol=0, atol=1e-13)
+
+
+def test_hier_windows_covering_everything_is_full_attention_over_both_sets():
+    g = O.Geom(2, 8, 16, (1, 4, 4), (5, 5, 5))
+    hp = (1, 2, 2)
+    q, k, v = (_rand((1, 1, g.n, 8), s) for s in (47, 48, 49))
+    o, lse = O.hier_attention(q, k, v, g, hp, 0.4)
+    keys = np.concatenate([k, _pool_reshape(k, g, hp)], axis=2)
+    vals = np.concatenate([v, _pool_reshape(v, g, hp)], axis=2)
+    np.testing.assert_allclose(o, _sdpa(q, keys, vals, 0.4), rtol=0, atol=1e-12)
+
+
+def test_hier_backward_finite_differences():
+    g = O.Geom(2, 8, 16, (1, 4, 4), (1, 1, 3))
+    hp = (1, 2, 2)
+    q, k, v, do = (_rand((1, 1, g.n, 4), s) for s in (50, 51, 52, 53))
+    dq, dk, dv = O.hier_backward(q, k, v, do, g, hp, 0.7)
+
+    def loss(q_, k_, v_):
+        return float((O.hier_attention(q_, k_, v_, g, hp, 0.7)[0] * do).sum())
+
+    rng = np.random.default_rng(54)
+    eps = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(6):
+            idx = (0, 0, int(rng.integers(g.n)), int(rng.integers(4)))
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grad[idx]) < 1e-7, (name, idx, fd, grad[idx])
+
+
+def test_hier_sampled_evaluator_equals_full_definition():
+    g, hp = HIER_CASES[0]
+    q, k, v = (_rand((1, 1, g.n, 8), s) for s in (55, 56, 57))
+    o, lse = O.hier_attention(q, k, v, g, hp, 0.3)
+    tiles = [0, 5, 17, 63]
+    ids, o_s, l_s = O.hier_attention_tiles(q[0, 0], k[0, 0], v[0, 0], g, hp, 0.3, tiles)
+    np.testing.assert_allclose(o_s, o[0, 0][ids], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l_s, lse[0, 0][ids], rtol=0, atol=1e-13)
+
+
+def test_pins_catch_coarse_tile_without_division(monkeypatch):
+    """Planted mistake: the coarse window centred on the fine tile index."""
+    monkeypatch.setattr(O, "coarse_tile_of", lambda a, hp: tuple(a))
+    g, hp = HIER_CASES[0]
+    with pytest.raises(AssertionError):
+        test_hier_equals_independent_masked_softmax(g, hp)
