@@ -392,7 +392,46 @@ def run_extras(V, dev):
     out["train_fwd_bwd"] = _bench_train(V, dev, peaks)
     out.update(_bench_xwin(V, dev, peaks))
     out["1080p_dual_sym_fwd"] = _bench_sym(V, dev, peaks)
+    out["720p_hier_fwd"] = _bench_hier(V, dev, peaks)
     return out
+
+
+def _bench_hier(V, dev, peaks):
+    """Hierarchical local attention at the 720p workload with h_pool 1x2x2
+    (coarse tiles 5x3x5): effective FLOPs count the fine and the coarse pairs
+    (27 kept tiles of 384 tokens each, per query)."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["720p"]
+    hp = (1, 2, 2)
+    geom = V.make_geom(w.batch, w.heads, w.head_dim, w.grid, w.tile, w.window, hp)
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 700 + i) for i in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_HIER_FWD, geom), dtype=torch.uint8, device=dev)
+    nc = [g // t // p for g, t, p in zip(w.grid, w.tile, hp)]
+    s = math.prod(w.tile)
+    coarse_keys = math.prod(min(win, n) for win, n in zip(w.window, nc)) * s
+    fl, _ = _flops_fwd(w)
+    fl += 4 * w.head_dim * w.batch * w.heads * w.n_tokens * coarse_keys
+    scale = 1 / math.sqrt(w.head_dim)
+    for _ in range(2):
+        V.vattn_hier_fwd(geom, q, k, v, scale, o, lse, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(4):
+        V.vattn_hier_fwd(geom, q, k, v, scale, o, lse, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 4
+    res = {"ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
+           "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status(),
+           "h_pool": list(hp)}
+    del q, k, v, o, lse, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def _bench_sym(V, dev, peaks):

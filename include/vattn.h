@@ -80,7 +80,9 @@ enum {
   VATTN_OP_DUAL_BWD = 3,
   VATTN_OP_DUAL_SYM_FWD = 4,
   VATTN_OP_DUAL_SYM_BWD = 5,
-  VATTN_OP_STA_FWD_HOST = 6  /* per chunk of batch*head slices: pass heads = the chunk size in geom */
+  VATTN_OP_STA_FWD_HOST = 6, /* per chunk of batch*head slices: pass heads = the chunk size in geom */
+  VATTN_OP_HIER_FWD = 7,     /* geom->pool = the medium pool factor h_pool */
+  VATTN_OP_HIER_BWD = 8
 };
 
 /* Raster -> tile-major row gather.  Tile-major position of raster token
@@ -129,6 +131,24 @@ int vattn_xwin_fwd(const vattn_geom* geom, int shifted, const void* q, const voi
 int vattn_xwin_bwd(const vattn_geom* geom, int shifted, const void* q, const void* k, const void* v,
                    const void* o, const float* lse, const void* dout, float scale, void* dq, void* dk,
                    void* dv, void* workspace, size_t ws_bytes, void* stream);
+
+/* Hierarchical local attention ("UltraGen: High-Resolution Video Generation
+ * with Hierarchical Attention" §4.3, hierarchical local attention: an
+ * intermediate-scale attention over coarse windows).  Each query attends, in
+ * ONE softmax, to
+ *   - its sliding-tile keys (as vattn_sta_fwd), and
+ *   - the keys and values average-pooled by h_pool = geom->pool, restricted to
+ *     a window of geom->window coarse tiles: the pooled grid is cut into tiles
+ *     of the same shape, a coarse tile spans h_pool fine tiles per dim, and
+ *     the window (clamped as the sliding tile's) is centred on the coarse tile
+ *     holding the query tile.
+ * Needs tiles-per-dim divisible by h_pool.  Tile-major q, k, v [B,h,N,d] bf16;
+ * o tile-major; lse [B,h,N] fp32 tile-major (the joint softmax's natural-log
+ * denominator) or NULL.  workspace >= vattn_workspace_size(VATTN_OP_HIER_FWD):
+ * medium-pooled K/V in coarse tile-major order, then O and LSE of the fine
+ * keys alone.  Errors are returned before any launch. */
+int vattn_hier_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                   float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /* Sliding-tile forward on HOST buffers in raster order, pipelined.  The
  * batch*head range is cut into chunks of `chunk_slices` slices; for every

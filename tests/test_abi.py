@@ -86,6 +86,13 @@ def test_argument_errors(V):
     with pytest.raises(V.VattnError) as e:
         V.vattn_sta_fwd_host(g, 16, 16, 16, 0.1, 16, 0, 1, 32, 64)         # two slots needed
     assert e.value.code == B.VATTN_ERR_WORKSPACE
+    with pytest.raises(V.VattnError) as e:   # tiles per dim (1, 3, 5) not divisible by h_pool (1, 2, 2)
+        V.vattn_hier_fwd(V.make_geom(1, 1, 128, (3, 24, 40), (3, 8, 8), (1, 3, 3), (1, 2, 2)), 16, 16, 16, 0.1, 16,
+                         None, 32, 1 << 30)
+    assert e.value.code == B.VATTN_ERR_SHAPE and "hierarchical pool" in str(e.value)
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_hier_fwd(g, 16, 16, 16, 0.1, 16, None, 32, 64)
+    assert e.value.code == B.VATTN_ERR_WORKSPACE
     with pytest.raises(V.VattnError) as e:
         V.vattn_workspace_size(99, g)
     assert e.value.code == B.VATTN_ERR_INVALID_ARG
@@ -105,6 +112,9 @@ def test_workspace_sizes(V):
         return (x + 255) // 256 * 256
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, g) == a(bh * n * d * 2) + 2 * a(bh * npool * d * 2)
     assert V.vattn_workspace_size(V.VATTN_OP_STA_BWD, g) == 2 * a(bh * n * 4)
+    # hierarchical forward (pool = h_pool): pooled K, V, then fine O and LSE
+    assert V.vattn_workspace_size(V.VATTN_OP_HIER_FWD, g) == (2 * a(bh * npool * d * 2) + a(bh * n * d * 2)
+                                                              + a(bh * n * 4))
     # host-buffer forward, per slot: 8 bf16 token tensors and 2 fp32 rows
     assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, g) == 8 * a(bh * n * d * 2) + 2 * a(bh * n * 4)
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == (4 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)

@@ -30,6 +30,8 @@ VATTN_OP_DUAL_BWD = 3
 VATTN_OP_DUAL_SYM_FWD = 4
 VATTN_OP_DUAL_SYM_BWD = 5
 VATTN_OP_STA_FWD_HOST = 6
+VATTN_OP_HIER_FWD = 7
+VATTN_OP_HIER_BWD = 8
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -83,6 +85,7 @@ _SIGS = {
     "vattn_dual_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_fwd_noalloc": [_GP, _P, _P, _P, _P, _F, _P, _P],
     "vattn_xwin_fwd": [_GP, _INT, _P, _P, _P, _F, _P, _P, _P],
+    "vattn_hier_fwd": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_host": [_GP, _P, _P, _P, _F, _P, _P, _I64, _P, _SZ, _P],
     "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_sym_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
@@ -185,6 +188,15 @@ def vattn_dual_sym_bwd(geom: Geom, q, k, v, g, o_l, lse_l, qp, kp, vp, o_p, lse_
     _check(lib.vattn_dual_sym_bwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o_l), _ptr(lse_l),
                                   _ptr(qp), _ptr(kp), _ptr(vp), _ptr(o_p), _ptr(lse_p), _ptr(dout), scale, _ptr(dq),
                                   _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def vattn_hier_fwd(geom: Geom, q, k, v, scale: float, o, lse=None, workspace=None, ws_bytes: int = 0,
+                   stream=None) -> None:
+    """Hierarchical local attention (geom.pool = the medium pool factor)."""
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_hier_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
+                              _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def vattn_sta_fwd_host(geom: Geom, q, k, v, scale: float, o, lse, chunk_slices: int, workspace,

@@ -68,6 +68,11 @@ struct Params {
   const __nv_bfloat16* o_local;
   const float* gvec;
   __nv_bfloat16* blend_out;
+  // key-side tile grid and coarse factor (STA): the sliding tile has the query
+  // grid and factor 1; the hierarchical branch the coarse grid and h_pool
+  int kNt, kNh, kNw, cft, cfh, cfw;
+  const __nv_bfloat16* merge_o;  // hierarchical: fine-key O and LSE to merge with (NULL = none)
+  const float* merge_lse;
   DevCtl ctl;
 };
 
@@ -83,9 +88,9 @@ __device__ __forceinline__ Stream make_stream(const Params& p, int q_tile) {
     const DevGeom& g = p.g;
     const int at = q_tile / (g.Nh * g.Nw), ah = (q_tile / g.Nw) % g.Nh, aw = q_tile % g.Nw;
     int et, ew;
-    tile_range(at, g.wt, g.Nt, g.wmode, &s.t0, &et);
-    tile_range(ah, g.wh, g.Nh, g.wmode, &s.h0, &s.eh);
-    tile_range(aw, g.ww, g.Nw, g.wmode, &s.w0, &ew);
+    tile_range(at / p.cft, g.wt, p.kNt, g.wmode, &s.t0, &et);
+    tile_range(ah / p.cfh, g.wh, p.kNh, g.wmode, &s.h0, &s.eh);
+    tile_range(aw / p.cfw, g.ww, p.kNw, g.wmode, &s.w0, &ew);
     s.runs = et * s.eh;
     s.run_len = ew * g.s;
   } else {
@@ -102,7 +107,7 @@ __device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int 
   if (p.mode != FWD_STA) return v;
   const int r = v / s.run_len, o = v - r * s.run_len;
   const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
-  return ((kt * p.g.Nh + kh) * p.g.Nw + s.w0) * p.g.s + o;
+  return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + o;
 }
 
 template <int D>
@@ -401,6 +406,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool have1 = nblk >= 2;
       const bool row_ok = row < q_valid;
       const size_t grow = (size_t)bh * p.g.N + (size_t)(q_row0 + row);
+      // hierarchical merge: one softmax over the fine keys (O_f, LSE_f given)
+      // and this kernel's coarse keys, in log2 units
+      float wf = 0.f, wc = 1.f, lse2_out = m + __log2f(l);
+      if (p.merge_o && row_ok) {
+        const float lf2 = p.merge_lse[grow] * 1.4426950408889634f;
+        const float mm = fmaxf(lf2, lse2_out);
+        wf = ex2(lf2 - mm);
+        wc = ex2(lse2_out - mm);
+        const float inv = 1.f / (wf + wc);
+        lse2_out = mm + __log2f(wf + wc);
+        wf *= inv;
+        wc *= inv;
+      }
       const uint32_t tO0 = tmem + lane_addr + 256u, tO1 = tmem + lane_addr + 384u;
       float gh = 0.f;
       if (p.blend_out) gh = p.gvec[bh % p.g.heads];
@@ -414,6 +432,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           o[c] = __uint_as_float(x0[c]) * a0 + (have1 ? __uint_as_float(x1[c]) * a1 : 0.f);
+        if (row_ok && p.merge_o) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.merge_o + grow * D + c0);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const uint4 of = src[v4];
+            const uint32_t w4[4] = {of.x, of.y, of.z, of.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o[8 * v4 + 2 * e] = wf * bf16lo(w4[e]) + wc * o[8 * v4 + 2 * e];
+              o[8 * v4 + 2 * e + 1] = wf * bf16hi(w4[e]) + wc * o[8 * v4 + 2 * e + 1];
+            }
+          }
+        }
         if (row_ok) {
           if (p.o) {
             uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + c0);
@@ -439,7 +470,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
       }
-      if (w == 0 && row_ok && p.lse) p.lse[grow] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (w == 0 && row_ok && p.lse) p.lse[grow] = lse2_out * 0.69314718055994531f;
     }
   }
 
@@ -469,6 +500,12 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   p.gvec = a.g;
   p.blend_out = a.o_local ? (__nv_bfloat16*)a.blend_out : nullptr;
   p.ctl = current_ctl();
+  p.kNt = g.Nt;
+  p.kNh = g.Nh;
+  p.kNw = g.Nw;
+  p.cft = p.cfh = p.cfw = 1;
+  p.merge_o = nullptr;
+  p.merge_lse = nullptr;
   int qblocks;
   if (mode == FWD_STA) {
     int G = 1;
@@ -476,6 +513,17 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
     p.G = G;
     p.q_blocks_per_tile = (g.s + BM - 1) / BM;
     p.Nk = g.N;
+    if (a.kgeom) {  // hierarchical: coarse tiles of the medium-pooled grid (same tile volume)
+      p.kNt = a.kgeom->Nt;
+      p.kNh = a.kgeom->Nh;
+      p.kNw = a.kgeom->Nw;
+      p.cft = a.cf[0];
+      p.cfh = a.cf[1];
+      p.cfw = a.cf[2];
+      p.Nk = a.kgeom->N;
+      p.merge_o = (const __nv_bfloat16*)a.merge_o;
+      p.merge_lse = a.merge_lse;
+    }
     qblocks = g.n_tiles * p.q_blocks_per_tile;
   } else {
     p.G = BN;

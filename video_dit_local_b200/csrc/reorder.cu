@@ -169,9 +169,11 @@ cudaError_t launch_kept_tiles(const DevGeom& g, int32_t* out, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 struct PoolParams {
   ReorderParams rp;
+  ReorderParams rpo;   // output order when out_tiled: tile-major over the pooled grid
   FastDiv PW, PH;      // pooled grid divisions
   uint32_t pt, ph, pw, PWv, PHv, N, Np, vpr;
   float inv_cnt;
+  int out_tiled;
 };
 
 // Up to three tensors pooled in one launch (K and V; or Q, K and V).
@@ -221,7 +223,8 @@ __global__ void __launch_bounds__(256) pool_kv_kernel(PoolParams p, FastDiv per_
     o.y = pack_bf16(acc[2] / cnt, acc[3] / cnt);
     o.z = pack_bf16(acc[4] / cnt, acc[5] / cnt);
     o.w = pack_bf16(acc[6] / cnt, acc[7] / cnt);
-    ts.dst[which][(size_t)row * p.vpr + c] = o;
+    const uint32_t uo = p.out_tiled ? coords_to_tiled(p.rpo, ut, uy, ux) : u;
+    ts.dst[which][((size_t)bh * p.Np + uo) * p.vpr + c] = o;
   }
 }
 
@@ -239,12 +242,18 @@ static PoolParams make_pool_params(const DevGeom& g) {
   p.Np = g.Np;
   p.vpr = g.d / 8;
   p.inv_cnt = 1.0f / (float)(g.pt * g.ph * g.pw);
+  p.rpo = p.rp;
+  p.out_tiled = 0;
   return p;
 }
 
 static cudaError_t pool_tensors(const DevGeom& g, int count, const void* const* src, void* const* dst,
-                                cudaStream_t st) {
-  const PoolParams p = make_pool_params(g);
+                                cudaStream_t st, const DevGeom* gout = nullptr) {
+  PoolParams p = make_pool_params(g);
+  if (gout) {
+    p.rpo = make_params(*gout);
+    p.out_tiled = 1;
+  }
   const long long per_bh = (long long)g.Np * p.vpr;
   const long long bh_total = (long long)g.B * g.heads;
   if (per_bh * bh_total == 0) return cudaSuccess;
@@ -271,6 +280,13 @@ cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void*
   const void* src[2] = {k, v};
   void* dst[2] = {kp, vp};
   return pool_tensors(g, 2, src, dst, st);
+}
+
+cudaError_t launch_pool_kv_tiled(const DevGeom& g, const DevGeom& gc, const void* k, const void* v, void* kp,
+                                 void* vp, cudaStream_t st) {
+  const void* src[2] = {k, v};
+  void* dst[2] = {kp, vp};
+  return pool_tensors(g, 2, src, dst, st, &gc);
 }
 
 cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, const void* v, void* qp, void* kp,

@@ -252,6 +252,23 @@ static SymBwdWs sym_bwd_ws(const DevGeom& g) {
   return w;
 }
 
+// Hierarchical forward: medium-pooled K, V (coarse tile-major), then the
+// fine-key O and LSE that the coarse pass merges with.
+struct HierFwdWs {
+  size_t kh, vh, o_f, lse_f, total;
+};
+static HierFwdWs hier_fwd_ws(const DevGeom& g) {
+  HierFwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t kv = align256(bh * g.Np * g.d * 2);
+  w.kh = 0;
+  w.vh = kv;
+  w.o_f = 2 * kv;
+  w.lse_f = w.o_f + align256(bh * g.N * g.d * 2);
+  w.total = w.lse_f + align256(bh * g.N * 4);
+  return w;
+}
+
 // Device staging of one chunk of the host-buffer forward: raster Q, K, V,
 // tile-major Q, K, V, O, LSE, and raster O, LSE.
 struct HostChunkWs {
@@ -365,6 +382,7 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_DUAL_SYM_FWD: *bytes = sym_fwd_ws(g).total; break;
     case VATTN_OP_DUAL_SYM_BWD: *bytes = sym_bwd_ws(g).total; break;
     case VATTN_OP_STA_FWD_HOST: *bytes = host_chunk_ws(g).total; break;
+    case VATTN_OP_HIER_FWD: *bytes = hier_fwd_ws(g).total; break;
     default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
   return ok();
@@ -524,6 +542,64 @@ int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, con
   // the caller's stream waits for every copy-out (and therefore for everything)
   for (int slot = 0; slot < 2 && slot < nchunks; ++slot)
     CHECK_LAUNCH(cudaStreamWaitEvent(caller, p.out_done[slot], 0), "stream wait");
+  return ok();
+}
+
+// Fine geometry (pool = h_pool) and the coarse grid: the medium-pooled grid
+// cut into tiles of the same shape.
+static int build_hier(const vattn_geom* geom, DevGeom* g, DevGeom* gc) {
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, g);
+  if (r) return r;
+  if (g->Nt % g->pt || g->Nh % g->ph || g->Nw % g->pw)
+    return fail(VATTN_ERR_SHAPE, "tiles per dim %dx%dx%d not divisible by the hierarchical pool %dx%dx%d", g->Nt, g->Nh,
+                g->Nw, g->pt, g->ph, g->pw);
+  vattn_geom c = *geom;
+  c.T = geom->T / geom->pool[0];
+  c.H = geom->H / geom->pool[1];
+  c.W = geom->W / geom->pool[2];
+  c.pool[0] = c.pool[1] = c.pool[2] = 1;
+  return build_geom(&c, NEED_TILE | NEED_ATTN, gc);
+}
+
+int vattn_hier_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                   float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g, gc;
+  int r = build_hier(geom, &g, &gc);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  const HierFwdWs w = hier_fwd_ws(g);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  uint8_t* ws = (uint8_t*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_pool_kv_tiled(g, gc, k, v, ws + w.kh, ws + w.vh, st), "hier_fwd pool launch");
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = ws + w.o_f;
+  a.lse = (float*)(ws + w.lse_f);
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "hier_fwd fine launch");
+  FwdArgs b{};
+  b.q = q;
+  b.k = ws + w.kh;
+  b.v = ws + w.vh;
+  b.o = o;
+  b.lse = lse;
+  b.scale = scale;
+  b.kgeom = &gc;
+  b.cf[0] = g.pt;
+  b.cf[1] = g.ph;
+  b.cf[2] = g.pw;
+  b.merge_o = ws + w.o_f;
+  b.merge_lse = (const float*)(ws + w.lse_f);
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, b, st), "hier_fwd coarse launch");
   return ok();
 }
 

@@ -49,6 +49,10 @@ cudaError_t launch_permute(const DevGeom& g, const void* src, void* dst, int64_t
                            cudaStream_t st);
 cudaError_t launch_kept_tiles(const DevGeom& g, int32_t* out, cudaStream_t st);
 cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void* kp, void* vp, cudaStream_t st);
+// Pooling with the pooled rows written in the tile-major order of `gc`, the
+// pooled grid cut into tiles (the coarse tiles of the hierarchical branch).
+cudaError_t launch_pool_kv_tiled(const DevGeom& g, const DevGeom& gc, const void* k, const void* v, void* kp,
+                                 void* vp, cudaStream_t st);
 cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, const void* v, void* qp, void* kp,
                             void* vp, cudaStream_t st);
 cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void* o_l, const float* gvec, void* out,
@@ -69,6 +73,14 @@ struct FwdArgs {
   const void* o_local;  // NULL = no blend
   const float* g;
   void* blend_out;
+  // STA only, hierarchical branch: keys are the tiles of `kgeom` (the coarse
+  // grid) and a query tile's window is centred on its tile index divided by
+  // cf; the result is merged with (merge_o, merge_lse) as one softmax over
+  // both key sets.  kgeom NULL = plain sliding tile.
+  const DevGeom* kgeom;
+  int cf[3];
+  const void* merge_o;
+  const float* merge_lse;
 };
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st);
