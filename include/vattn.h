@@ -150,6 +150,16 @@ int vattn_xwin_bwd(const vattn_geom* geom, int shifted, const void* q, const voi
 int vattn_hier_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
                    float* lse, void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward of vattn_hier_fwd: dq, dk, dv (bf16, tile-major) from q, k, v, the
+ * forward's o and lse (required) and dout.  The medium-pooled keys' gradients
+ * flow back to every token of their pool block divided by its size.
+ * workspace >= vattn_workspace_size(VATTN_OP_HIER_BWD): pooled K/V, the row
+ * terms D and L, fp32 dK/dV of the pooled keys and the fp32 coarse part of dQ.
+ * Deterministic (no atomics). */
+int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const void* o,
+                   const float* lse, const void* dout, float scale, void* dq, void* dk, void* dv, void* workspace,
+                   size_t ws_bytes, void* stream);
+
 /* Sliding-tile forward on HOST buffers in raster order, pipelined.  The
  * batch*head range is cut into chunks of `chunk_slices` slices; for every
  * chunk the host->device copy of Q, K, V, the permute + vattn_sta_fwd +

@@ -92,3 +92,54 @@ def test_hier_fwd_rejects_tiles_not_divisible_by_pool(V):
     with pytest.raises(V.VattnError) as e:
         V.vattn_hier_fwd(geom, t, t, t, 0.1, t, None, t, 1 << 30)
     assert e.value.code == V.binding.VATTN_ERR_SHAPE
+
+
+# ---------------------------------------------------------------- backward
+
+def _hier_fwd_bwd(V, w, check):
+    """GPU forward (o, lse saved) then backward; returns raster dQ, dK, dV."""
+    import torch
+    geom = geom_for(V, w)
+    tiled = []
+    for tid in (S.Q_ID, S.K_ID, S.V_ID, S.DO_ID):
+        x = gpu_tensor(w, tid, check)
+        t = torch.empty_like(x)
+        V.vattn_tile_permute(geom, x, t)
+        tiled.append(t)
+    q, k, v, do = tiled
+    scale = 1 / math.sqrt(w.head_dim)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_HIER_FWD, geom), dtype=torch.uint8, device="cuda")
+    V.vattn_hier_fwd(geom, q, k, v, scale, o, lse, ws)
+    dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
+    wsb = torch.empty(V.vattn_workspace_size(V.VATTN_OP_HIER_BWD, geom), dtype=torch.uint8, device="cuda")
+    V.vattn_hier_bwd(geom, q, k, v, o, lse, do, scale, dq, dk, dv, wsb)
+    torch.cuda.synchronize()
+    assert V.vattn_get_status() == 0, V.vattn_last_error()
+    out = []
+    for t in (dq, dk, dv):
+        r = torch.empty_like(t)
+        V.vattn_tile_unpermute(geom, t, r)
+        out.append(r)
+    return out
+
+
+@pytest.mark.parametrize("grid,tile,window,hpool,d,batch,heads", [
+    ((6, 16, 32), (3, 8, 8), (1, 3, 3), (1, 2, 2), 128, 1, 2),
+    ((4, 16, 16), (1, 4, 4), (3, 1, 1), (2, 2, 2), 64, 2, 1),
+    ((2, 16, 48), (2, 8, 8), (1, 1, 1), (1, 2, 3), 128, 1, 1),
+    ((6, 32, 48), (3, 8, 8), (1, 3, 3), (1, 2, 3), 128, 1, 1),   # fine windows clamp in H and W
+])
+def test_hier_bwd_small_full(V, grid, tile, window, hpool, d, batch, heads):
+    w = S.small_workload("hier_bwd", 63, batch, heads, d, grid, tile, window, hpool)
+    check = [(b, h) for b in range(batch) for h in range(heads)]
+    dq, dk, dv = _hier_fwd_bwd(V, w, check)
+    g = O.geom_of(w)._replace(pool=(1, 1, 1))
+    scale = 1 / math.sqrt(d)
+    q, k, v, do = (np.stack([np.stack([host_f64(w, i, b, h) for h in range(heads)]) for b in range(batch)])
+                   for i in (S.Q_ID, S.K_ID, S.V_ID, S.DO_ID))
+    rq, rk, rv = O.hier_backward(q, k, v, do, g, tuple(hpool), scale)
+    for name, got, ref in (("dQ", dq, rq), ("dK", dk, rk), ("dV", dv, rv)):
+        for b, h in check:
+            assert_close(to_f64(got[b, h]), ref[b, h], O_MAX_ABS, O_MEAN_ABS, f"{name} b{b} h{h}")

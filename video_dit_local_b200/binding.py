@@ -86,6 +86,7 @@ _SIGS = {
     "vattn_dual_fwd_noalloc": [_GP, _P, _P, _P, _P, _F, _P, _P],
     "vattn_xwin_fwd": [_GP, _INT, _P, _P, _P, _F, _P, _P, _P],
     "vattn_hier_fwd": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
+    "vattn_hier_bwd": [_GP, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_host": [_GP, _P, _P, _P, _F, _P, _P, _I64, _P, _SZ, _P],
     "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_sym_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
@@ -197,6 +198,15 @@ def vattn_hier_fwd(geom: Geom, q, k, v, scale: float, o, lse=None, workspace=Non
         ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.vattn_hier_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
                               _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def vattn_hier_bwd(geom: Geom, q, k, v, o, lse, dout, scale: float, dq, dk, dv, workspace, ws_bytes: int = 0,
+                   stream=None) -> None:
+    """Backward of vattn_hier_fwd (geom.pool = the medium pool factor)."""
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_hier_bwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), scale,
+                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def vattn_sta_fwd_host(geom: Geom, q, k, v, scale: float, o, lse, chunk_slices: int, workspace,

@@ -58,35 +58,41 @@ __device__ __forceinline__ RowStream flat_stream(int n) {
   return s;
 }
 
-// key tiles kept by query tile q (its window)
-__device__ __forceinline__ RowStream window_stream(const DevGeom& g, int q) {
+// Key tiles kept by query tile q (its window).  The keys are the tiles of gk:
+// the query grid itself for the sliding tile (cf = 1); the coarse grid of the
+// hierarchical branch, whose window is centred on q's tile index / cf.  Rows
+// of the stream are rows of gk (RowStream::row(gk, v)).
+__device__ __forceinline__ RowStream window_stream(const DevGeom& g, const DevGeom& gk, int cft, int cfh, int cfw,
+                                                   int q) {
   const int at = q / (g.Nh * g.Nw), ah = (q / g.Nw) % g.Nh, aw = q % g.Nw;
   RowStream s;
   int et, ew;
-  tile_range(at, g.wt, g.Nt, g.wmode, &s.t0, &et);
-  tile_range(ah, g.wh, g.Nh, g.wmode, &s.h0, &s.eh);
-  tile_range(aw, g.ww, g.Nw, g.wmode, &s.w0, &ew);
+  tile_range(at / cft, g.wt, gk.Nt, g.wmode, &s.t0, &et);
+  tile_range(ah / cfh, g.wh, gk.Nh, g.wmode, &s.h0, &s.eh);
+  tile_range(aw / cfw, g.ww, gk.Nw, g.wmode, &s.w0, &ew);
   s.runs = et * s.eh;
   s.run_len = ew * g.s;
   s.tiled = true;
   return s;
 }
 
-// query tiles whose window holds key tile k (the inverse window): per dim a
-// contiguous range, so again a box of tiles
-__device__ __forceinline__ RowStream inverse_stream(const DevGeom& g, int k) {
-  const int kt = k / (g.Nh * g.Nw), kh = (k / g.Nw) % g.Nh, kw = k % g.Nw;
+// Query tiles whose window holds key tile k of gk (the inverse window): per
+// dim a contiguous range of gk tiles, i.e. of query tiles [lo*cf, (hi+1)*cf),
+// so again a box of tiles; rows are rows of the query grid g.
+__device__ __forceinline__ RowStream inverse_stream(const DevGeom& g, const DevGeom& gk, int cft, int cfh, int cfw,
+                                                    int k) {
+  const int kt = k / (gk.Nh * gk.Nw), kh = (k / gk.Nw) % gk.Nh, kw = k % gk.Nw;
   int lt, ht, lh, hh, lw, hw;
-  tile_inverse(kt, g.wt, g.Nt, g.wmode, &lt, &ht);
-  tile_inverse(kh, g.wh, g.Nh, g.wmode, &lh, &hh);
-  tile_inverse(kw, g.ww, g.Nw, g.wmode, &lw, &hw);
+  tile_inverse(kt, g.wt, gk.Nt, g.wmode, &lt, &ht);
+  tile_inverse(kh, g.wh, gk.Nh, g.wmode, &lh, &hh);
+  tile_inverse(kw, g.ww, gk.Nw, g.wmode, &lw, &hw);
   RowStream s;
-  s.t0 = lt;
-  s.h0 = lh;
-  s.w0 = lw;
-  s.eh = hh - lh + 1;
-  s.runs = (ht - lt + 1) * s.eh;
-  s.run_len = (hw - lw + 1) * g.s;
+  s.t0 = lt * cft;
+  s.h0 = lh * cfh;
+  s.w0 = lw * cfw;
+  s.eh = (hh - lh + 1) * cfh;
+  s.runs = (ht - lt + 1) * cft * s.eh;
+  s.run_len = (hw - lw + 1) * cfw * g.s;
   s.tiled = true;
   return s;
 }
@@ -97,6 +103,18 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
           smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Index, in gk's tile-major order, of the pool block holding tile-major token
+// `tok` of g (the medium-pooled grid cut into tiles: hierarchical branch).
+__device__ __forceinline__ int coarse_of_tiled(const DevGeom& g, const DevGeom& gk, int tok) {
+  const int tile = tok / g.s, l = tok - tile * g.s;
+  const int at = tile / (g.Nh * g.Nw), ah = (tile / g.Nw) % g.Nh, aw = tile % g.Nw;
+  const int lt = l / (g.th * g.tw), lh = (l / g.tw) % g.th, lw = l % g.tw;
+  const int t = (at * g.tt + lt) / g.pt, y = (ah * g.th + lh) / g.ph, x = (aw * g.tw + lw) / g.pw;
+  const int ct = t / gk.tt, ch = y / gk.th, cw = x / gk.tw;
+  return ((ct * gk.Nh + ch) * gk.Nw + cw) * gk.s + ((t - ct * gk.tt) * gk.th + (y - ch * gk.th)) * gk.tw +
+         (x - cw * gk.tw);
 }
 
 // pooled-raster index of the pool block holding tile-major token `tok`
@@ -191,7 +209,9 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const PreArgs a) {
 // ---------------------------------------------------------------------------
 // dK / dV
 // ---------------------------------------------------------------------------
-enum { DKDV_LOCAL = 0, DKDV_GLOBAL = 1 };
+// HIER: keys are the coarse tiles of the medium-pooled grid (hierarchical
+// branch): the inverse coarse window of fine query tiles, fp32 dK_h / dV_h out.
+enum { DKDV_LOCAL = 0, DKDV_GLOBAL = 1, DKDV_HIER = 2 };
 
 template <int D>
 struct DkdvSmem {
@@ -214,7 +234,11 @@ struct DkdvSmem {
 
 struct DkdvParams {
   DevGeom g;
-  int mode;          // DKDV_LOCAL / DKDV_GLOBAL
+  DevGeom gk;        // key tile grid (= g but for DKDV_HIER: the coarse grid)
+  int cft, cfh, cfw; // coarse factor (1 but for DKDV_HIER)
+  int hier_add;      // LOCAL: dkp_in / dvp_in are rows of gadd in tile-major order
+  DevGeom gadd;      // the coarse grid of those rows (hier_add only)
+  int mode;          // DKDV_LOCAL / DKDV_GLOBAL / DKDV_HIER
   int Gq;            // query sub-box rows (divides the tile volume, <= 64)
   int kv_blocks_per_tile;
   int Nk;            // key rows per batch*head (N or Np)
@@ -268,12 +292,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   int key_row0, key_valid;
   RowStream qs;
-  if (p.mode == DKDV_LOCAL) {
+  if (p.mode != DKDV_GLOBAL) {
     const int kt = blockIdx.x / p.kv_blocks_per_tile;
     const int sb = blockIdx.x - kt * p.kv_blocks_per_tile;
     key_row0 = kt * g.s + sb * 128;
     key_valid = min(128, g.s - sb * 128);
-    qs = inverse_stream(g, kt);
+    qs = inverse_stream(g, p.gk, p.cft, p.cfh, p.cfw, kt);
   } else {
     key_row0 = blockIdx.x * 128;
     key_valid = min(128, p.Nk - key_row0);
@@ -469,7 +493,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t tAcc = tmem + lane_addr + (w == 0 ? 256u : 384u);
       const float mul = (w == 0) ? 1.f : p.scale;
       const size_t tok = (size_t)key_row0 + row;
-      if (p.mode == DKDV_GLOBAL) {
+      if (p.mode != DKDV_LOCAL) {
         float* dst = (w == 0 ? p.dvp_out : p.dkp_out) + ((size_t)bh * p.Nk + tok) * D;
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -489,7 +513,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float* add_row = nullptr;
         float inv_cnt = 0.f;
         if (add && row_ok) {
-          add_row = add + ((size_t)bh * g.Np + pooled_of_tiled(g, (int)tok)) * D;
+          const int prow = p.hier_add ? coarse_of_tiled(g, p.gadd, (int)tok) : pooled_of_tiled(g, (int)tok);
+          add_row = add + ((size_t)bh * g.Np + prow) * D;
           inv_cnt = 1.f / (float)(g.pt * g.ph * g.pw);
         }
         __nv_bfloat16* dst = (w == 0 ? p.dv : p.dk) + ((size_t)bh * g.N + tok) * D;
@@ -562,11 +587,15 @@ struct DqSmem {
 // Two launches make dQ: GLOBAL (dense 128-row query blocks against all pooled
 // keys, fp32 result to a workspace) and LOCAL (query blocks inside one query
 // tile against its kept window; adds the GLOBAL part and writes bf16 dQ).
-enum { DQ_LOCAL = 0, DQ_GLOBAL = 1 };
+// HIER: the coarse window of medium-pooled keys (hierarchical branch), fp32
+// partial dQ out (acc_out) for the fine pass to add.
+enum { DQ_LOCAL = 0, DQ_GLOBAL = 1, DQ_HIER = 2 };
 
 struct DqParams {
   DevGeom g;
-  int mode;          // DQ_LOCAL / DQ_GLOBAL
+  DevGeom gk;        // key tile grid (= g but for DQ_HIER: the coarse grid)
+  int cft, cfh, cfw; // coarse factor (1 but for DQ_HIER)
+  int mode;          // DQ_LOCAL / DQ_GLOBAL / DQ_HIER
   int G0;            // key sub-box rows of the local stream
   int q_blocks_per_tile;
   float c2;
@@ -622,7 +651,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     q_row0 = q_tile * g.s + sub * 128;
     q_valid = min(128, g.s - sub * 128);
   }
-  const RowStream ks = glob ? flat_stream(g.Np) : window_stream(g, q_tile);
+  const RowStream ks = glob ? flat_stream(g.Np) : window_stream(g, p.gk, p.cft, p.cfh, p.cfw, q_tile);
   const int Lk = ks.length();
   const int nblk = (Lk + DQ_BN - 1) / DQ_BN;
 
@@ -673,10 +702,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(&full[s], L::KB_BYTES);
         const int G = glob ? DQ_BN : p.G0;
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
-        const int oob = glob ? g.Np : g.N;
+        const int oob = glob ? g.Np : p.gk.N;
         for (int u = 0; u < DQ_BN / G; ++u) {
           const int v = j * DQ_BN + u * G;
-          const int row = v < Lk ? ks.row(g, v) : oob;
+          const int row = v < Lk ? ks.row(p.gk, v) : oob;
           for (int c = 0; c < L::CHUNKS; ++c)
             tma_load_3d(smem + off + s * L::KB_BYTES + c * KBOX + u * G * 128, tm, &full[s], c * 64, row, bh);
         }
@@ -786,7 +815,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           float f[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) f[c] = __uint_as_float(x[c]) * p.scale;
-          if (glob) {
+          if (p.acc_out) {
             float4* dst = reinterpret_cast<float4*>(p.acc_out + grow * D + c0);
 #pragma unroll
             for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(f[4 * v4], f[4 * v4 + 1], f[4 * v4 + 2], f[4 * v4 + 3]);
@@ -835,14 +864,34 @@ static cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// hk != NULL: hierarchical (coarse grid hk, factor = g's pool).  With global,
+// the coarse-key pass (DKDV_HIER); without, the fine pass adding the coarse
+// keys' fp32 gradients a.dkp / a.dvp through the medium pooling.
 template <int D>
-static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global, bool dual, cudaStream_t st) {
+static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global, bool dual, cudaStream_t st,
+                                 const DevGeom* hk = nullptr) {
   DkdvParams p;
   p.g = g;
+  p.gk = g;
+  p.gadd = g;
+  p.cft = p.cfh = p.cfw = 1;
+  p.hier_add = 0;
   p.mode = global ? DKDV_GLOBAL : DKDV_LOCAL;
   p.Gq = global ? 64 : pow2_rows(g.s, 64);
   p.kv_blocks_per_tile = (g.s + 127) / 128;
   p.Nk = global ? g.Np : g.N;
+  if (hk && global) {
+    p.gk = *hk;
+    p.cft = g.pt;
+    p.cfh = g.ph;
+    p.cfw = g.pw;
+    p.mode = DKDV_HIER;
+    p.Gq = pow2_rows(g.s, 64);
+    p.Nk = hk->N;
+  } else if (hk) {  // fine keys: the streams stay on g, only the addend rows are coarse
+    p.gadd = *hk;
+    p.hier_add = 1;
+  }
   p.scale = a.scale;
   p.c2 = a.scale * LOG2E;
   p.nlse2 = global ? a.nlse2_g : a.nlse2_l;
@@ -855,7 +904,9 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   p.dvp_in = (!global && dual) ? a.dvp : nullptr;
   p.ctl = current_ctl();
   const long long bh = (long long)g.B * g.heads;
-  const int blocks = global ? (g.Np + 127) / 128 : g.n_tiles * p.kv_blocks_per_tile;
+  const int blocks = p.mode == DKDV_GLOBAL ? (g.Np + 127) / 128
+                     : p.mode == DKDV_HIER ? hk->n_tiles * p.kv_blocks_per_tile
+                                           : g.n_tiles * p.kv_blocks_per_tile;
   if (bh == 0 || blocks == 0) return cudaSuccess;
   CUtensorMap tk, tv, tq, tdo;
   const char* err = nullptr;
@@ -870,11 +921,18 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   return cudaGetLastError();
 }
 
+// hk != NULL: the coarse-key pass of the hierarchical branch (DQ_HIER) into
+// the fp32 a.dq_acc; keys a.kp / a.vp in hk's tile-major order.
 template <int D>
-static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, bool add_acc, cudaStream_t st) {
+static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, bool add_acc, cudaStream_t st,
+                               const DevGeom* hk = nullptr) {
   DqParams p;
   p.g = g;
-  p.mode = global ? DQ_GLOBAL : DQ_LOCAL;
+  p.gk = hk ? *hk : g;
+  p.cft = hk ? g.pt : 1;
+  p.cfh = hk ? g.ph : 1;
+  p.cfw = hk ? g.pw : 1;
+  p.mode = global ? DQ_GLOBAL : hk ? DQ_HIER : DQ_LOCAL;
   int G0 = DQ_BN;  // largest multiple of 8 dividing both the key block and the tile volume
   while (G0 > 8 && (DQ_BN % G0 != 0 || g.s % G0 != 0)) G0 -= 8;
   p.G0 = G0;
@@ -883,9 +941,9 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   p.c2 = a.scale * LOG2E;
   p.nlse2 = global ? a.nlse2_g : a.nlse2_l;
   p.ndelta = global ? a.ndelta_g : a.ndelta_l;
-  p.acc_in = (!global && add_acc) ? a.dq_acc : nullptr;
+  p.acc_in = (!global && !hk && add_acc) ? a.dq_acc : nullptr;
   p.acc_pooled = a.dq_acc_pooled ? 1 : 0;
-  p.acc_out = global ? a.dq_acc : nullptr;
+  p.acc_out = (global || hk) ? a.dq_acc : nullptr;
   p.dq = (__nv_bfloat16*)a.dq;
   p.ctl = current_ctl();
   const long long bh = (long long)g.B * g.heads;
@@ -893,9 +951,9 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   if (bh == 0 || blocks == 0) return cudaSuccess;
   CUtensorMap tq, tdo, tk, tv;
   const char* err = nullptr;
-  const void* kk = global ? a.kp : a.k;
-  const void* vv = global ? a.vp : a.v;
-  const long long nk = global ? g.Np : g.N;
+  const void* kk = (global || hk) ? a.kp : a.k;
+  const void* vv = (global || hk) ? a.vp : a.v;
+  const long long nk = global ? g.Np : hk ? hk->N : g.N;
   const int G = global ? DQ_BN : p.G0;
   if (!make_tmap_rows(&tq, a.q, D, g.N, bh, 128, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, 128, &err) ||
       !make_tmap_rows(&tk, kk, D, nk, bh, G, &err) || !make_tmap_rows(&tv, vv, D, nk, bh, G, &err))
@@ -978,6 +1036,19 @@ cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual,
 cudaError_t launch_bwd_dq_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st) {
   if (g.d == 128) return bwd::launch_dq_d<128>(g, a, true, false, st);
   if (g.d == 64) return bwd::launch_dq_d<64>(g, a, true, false, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_dkdv_hier(const DevGeom& g, const DevGeom& gc, const BwdArgs& a, bool coarse_keys,
+                                 cudaStream_t st) {
+  if (g.d == 128) return bwd::launch_dkdv_d<128>(g, a, coarse_keys, !coarse_keys, st, &gc);
+  if (g.d == 64) return bwd::launch_dkdv_d<64>(g, a, coarse_keys, !coarse_keys, st, &gc);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_dq_hier(const DevGeom& g, const DevGeom& gc, const BwdArgs& a, cudaStream_t st) {
+  if (g.d == 128) return bwd::launch_dq_d<128>(g, a, false, false, st, &gc);
+  if (g.d == 64) return bwd::launch_dq_d<64>(g, a, false, false, st, &gc);
   return cudaErrorInvalidValue;
 }
 

@@ -269,6 +269,26 @@ static HierFwdWs hier_fwd_ws(const DevGeom& g) {
   return w;
 }
 
+// Hierarchical backward: pooled K, V (bf16, coarse tile-major), -D and -L
+// rows, fp32 dK/dV of the pooled keys, fp32 coarse part of dQ.
+struct HierBwdWs {
+  size_t kh, vh, ndelta, nlse2, dkh, dvh, dq_acc, total;
+};
+static HierBwdWs hier_bwd_ws(const DevGeom& g) {
+  HierBwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t kv = align256(bh * g.Np * g.d * 2), row = align256(bh * g.N * 4), kvf = align256(bh * g.Np * g.d * 4);
+  w.kh = 0;
+  w.vh = kv;
+  w.ndelta = 2 * kv;
+  w.nlse2 = w.ndelta + row;
+  w.dkh = w.nlse2 + row;
+  w.dvh = w.dkh + kvf;
+  w.dq_acc = w.dvh + kvf;
+  w.total = w.dq_acc + align256(bh * g.N * g.d * 4);
+  return w;
+}
+
 // Device staging of one chunk of the host-buffer forward: raster Q, K, V,
 // tile-major Q, K, V, O, LSE, and raster O, LSE.
 struct HostChunkWs {
@@ -383,6 +403,7 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_DUAL_SYM_BWD: *bytes = sym_bwd_ws(g).total; break;
     case VATTN_OP_STA_FWD_HOST: *bytes = host_chunk_ws(g).total; break;
     case VATTN_OP_HIER_FWD: *bytes = hier_fwd_ws(g).total; break;
+    case VATTN_OP_HIER_BWD: *bytes = hier_bwd_ws(g).total; break;
     default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
   return ok();
@@ -600,6 +621,56 @@ int vattn_hier_fwd(const vattn_geom* geom, const void* q, const void* k, const v
   b.merge_o = ws + w.o_f;
   b.merge_lse = (const float*)(ws + w.lse_f);
   CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, b, st), "hier_fwd coarse launch");
+  return ok();
+}
+
+int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const void* o,
+                   const float* lse, const void* dout, float scale, void* dq, void* dk, void* dv, void* workspace,
+                   size_t ws_bytes, void* stream) {
+  DevGeom g, gc;
+  int r = build_hier(geom, &g, &gc);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(lse);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(dq);
+  REQUIRE_PTR(dk);
+  REQUIRE_PTR(dv);
+  const HierBwdWs w = hier_bwd_ws(g);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  uint8_t* ws = (uint8_t*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_pool_kv_tiled(g, gc, k, v, ws + w.kh, ws + w.vh, st), "hier_bwd pool launch");
+  float* ndelta = (float*)(ws + w.ndelta);
+  float* nlse2 = (float*)(ws + w.nlse2);
+  CHECK_LAUNCH(launch_preprocess_branch(g, dout, o, lse, nullptr, ndelta, nlse2, st), "hier_bwd preprocess launch");
+  BwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.kp = ws + w.kh;
+  a.vp = ws + w.vh;
+  a.dout = dout;
+  a.scale = scale;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.ndelta_l = a.ndelta_g = ndelta;  // one softmax over both key sets
+  a.nlse2_l = a.nlse2_g = nlse2;
+  a.dkp = (float*)(ws + w.dkh);
+  a.dvp = (float*)(ws + w.dvh);
+  a.dq_acc = (float*)(ws + w.dq_acc);
+  a.dq_acc_pooled = false;
+  CHECK_LAUNCH(launch_bwd_dkdv_hier(g, gc, a, true, st), "hier_bwd coarse dK/dV launch");
+  CHECK_LAUNCH(launch_bwd_dkdv_hier(g, gc, a, false, st), "hier_bwd fine dK/dV launch");
+  CHECK_LAUNCH(launch_bwd_dq_hier(g, gc, a, st), "hier_bwd coarse dQ launch");
+  CHECK_LAUNCH(launch_bwd_dq(g, a, true, st), "hier_bwd fine dQ launch");
   return ok();
 }
 

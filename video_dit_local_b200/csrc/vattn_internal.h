@@ -122,6 +122,14 @@ cudaError_t launch_bwd_dq(const DevGeom& g, const BwdArgs& a, bool dual, cudaStr
 cudaError_t launch_bwd_dq_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_local(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st);
 cudaError_t launch_bwd_dkdv_global(const DevGeom& g, const BwdArgs& a, cudaStream_t st);
+// Hierarchical branch (g.pool = h_pool, gc = the coarse grid).  coarse_keys:
+// dK/dV of the medium-pooled keys a.kp / a.vp into fp32 a.dkp / a.dvp; else the
+// fine keys' dK/dV (bf16 a.dk / a.dv) plus a.dkp / a.dvp through the pooling.
+// Both use the joint softmax's a.nlse2_l / a.ndelta_l.
+cudaError_t launch_bwd_dkdv_hier(const DevGeom& g, const DevGeom& gc, const BwdArgs& a, bool coarse_keys,
+                                 cudaStream_t st);
+// dQ of the coarse keys into fp32 a.dq_acc (launch_bwd_dq(dual = true) adds it).
+cudaError_t launch_bwd_dq_hier(const DevGeom& g, const DevGeom& gc, const BwdArgs& a, cudaStream_t st);
 
 // TMA descriptor for a [rows_per_bh x bh] stack of rows of `d` bf16 elements,
 // box = 64 elements x box_rows rows x 1, 128-byte swizzle.  Returns false and
