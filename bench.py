@@ -392,7 +392,7 @@ def run_extras(V, dev):
     out["train_fwd_bwd"] = _bench_train(V, dev, peaks)
     out.update(_bench_xwin(V, dev, peaks))
     out["1080p_dual_sym_fwd"] = _bench_sym(V, dev, peaks)
-    out["720p_hier_fwd"] = _bench_hier(V, dev, peaks)
+    out["720p_hier_fwd_bwd"] = _bench_hier(V, dev, peaks)
     return out
 
 
@@ -426,10 +426,26 @@ def _bench_hier(V, dev, peaks):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / 4
-    res = {"ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
-           "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status(),
+    # backward: 10*d effective FLOPs per pair (the forward counts 4*d)
+    do = _device_randn(shape, 703)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    wsb = torch.empty(V.vattn_workspace_size(V.VATTN_OP_HIER_BWD, geom), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        V.vattn_hier_bwd(geom, q, k, v, o, lse, do, scale, dq, dk, dv, wsb)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(3):
+        V.vattn_hier_bwd(geom, q, k, v, o, lse, do, scale, dq, dk, dv, wsb)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_b = e0.elapsed_time(e1) / 3
+    fl_b = fl * 10 // 4
+    res = {"fwd_ms": round(ms, 3), "fwd_eff_tflops": round(fl / ms / 1e9, 1),
+           "fwd_frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4),
+           "bwd_ms": round(ms_b, 3), "bwd_eff_tflops": round(fl_b / ms_b / 1e9, 1),
+           "bwd_frac": round(fl_b / ms_b / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status(),
            "h_pool": list(hp)}
-    del q, k, v, o, lse, ws
+    del q, k, v, o, lse, ws, do, dq, dk, dv, wsb
     torch.cuda.empty_cache()
     return res
 
