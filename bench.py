@@ -671,7 +671,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--e2e-chunk", type=int, default=3, help="batch*head slices per host-copy chunk (e2e)")
+    ap.add_argument("--e2e-chunk", type=int, default=1, help="batch*head slices per host-copy chunk (e2e)")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: fewer heads than the workload")
     ap.add_argument("--workload", choices=["720p", "train"], default="720p",
                     help="720p: the benchmark line; train: profiling of the training step alone")
