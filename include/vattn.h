@@ -82,7 +82,8 @@ enum {
   VATTN_OP_DUAL_SYM_BWD = 5,
   VATTN_OP_STA_FWD_HOST = 6, /* per chunk of batch*head slices: pass heads = the chunk size in geom */
   VATTN_OP_HIER_FWD = 7,     /* geom->pool = the medium pool factor h_pool */
-  VATTN_OP_HIER_BWD = 8
+  VATTN_OP_HIER_BWD = 8,
+  VATTN_OP_STA_FWD_FP8 = 9
 };
 
 /* Raster -> tile-major row gather.  Tile-major position of raster token
@@ -159,6 +160,19 @@ int vattn_hier_fwd(const vattn_geom* geom, const void* q, const void* k, const v
 int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const void* v, const void* o,
                    const float* lse, const void* dout, float scale, void* dq, void* dk, void* dv, void* workspace,
                    size_t ws_bytes, void* stream);
+
+/* Sliding-tile forward with Q*K^T in FP8 (e4m3) on the f8f6f4 tensor path,
+ * P*V in bf16: an inference variant in the spirit of the 8-bit attention the
+ * pages cite ("SageAttention"), which the pages do not define further.
+ * Q and K are quantised per batch*head: scale s = absmax / 448 (the largest
+ * finite e4m3), byte = round-to-nearest-even e4m3 of x * (448 / absmax) with
+ * saturation; S = bytes(Q) bytes(K)^T * s_Q * s_K * scale in fp32.  Same
+ * arguments and layouts as vattn_sta_fwd; d = 128 only.
+ * workspace >= vattn_workspace_size(VATTN_OP_STA_FWD_FP8): e4m3 Q [B,h,N,d]
+ * bytes at offset 0, e4m3 K at offset align256(B*h*N*d), then the absmax
+ * bits as int32 [B*h][2] (Q, K); they hold this call's values afterwards. */
+int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                      float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /* Sliding-tile forward on HOST buffers in raster order, pipelined.  The
  * batch*head range is cut into chunks of `chunk_slices` slices; for every

@@ -93,6 +93,12 @@ def test_argument_errors(V):
     with pytest.raises(V.VattnError) as e:
         V.vattn_hier_fwd(g, 16, 16, 16, 0.1, 16, None, 32, 64)
     assert e.value.code == B.VATTN_ERR_WORKSPACE
+    with pytest.raises(V.VattnError) as e:   # the FP8 forward is d = 128 only
+        V.vattn_sta_fwd_fp8(_geom(V, head_dim=64), 16, 16, 16, 0.1, 16, None, 32, 1 << 30)
+    assert e.value.code == B.VATTN_ERR_UNSUPPORTED
+    with pytest.raises(V.VattnError) as e:
+        V.vattn_sta_fwd_fp8(_geom(V, head_dim=128), 16, 16, 16, 0.1, 16, None, 32, 64)
+    assert e.value.code == B.VATTN_ERR_WORKSPACE
     with pytest.raises(V.VattnError) as e:
         V.vattn_workspace_size(99, g)
     assert e.value.code == B.VATTN_ERR_INVALID_ARG
@@ -115,6 +121,8 @@ def test_workspace_sizes(V):
     # hierarchical forward (pool = h_pool): pooled K, V, then fine O and LSE
     assert V.vattn_workspace_size(V.VATTN_OP_HIER_FWD, g) == (2 * a(bh * npool * d * 2) + a(bh * n * d * 2)
                                                               + a(bh * n * 4))
+    # FP8 forward: e4m3 Q and K bytes, then two absmax words per batch*head
+    assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_FP8, g) == 2 * a(bh * n * d) + a(bh * 8)
     # host-buffer forward, per slot: 8 bf16 token tensors and 2 fp32 rows
     assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, g) == 8 * a(bh * n * d * 2) + 2 * a(bh * n * 4)
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == (4 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)

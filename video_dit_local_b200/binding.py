@@ -32,6 +32,7 @@ VATTN_OP_DUAL_SYM_BWD = 5
 VATTN_OP_STA_FWD_HOST = 6
 VATTN_OP_HIER_FWD = 7
 VATTN_OP_HIER_BWD = 8
+VATTN_OP_STA_FWD_FP8 = 9
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -87,6 +88,7 @@ _SIGS = {
     "vattn_xwin_fwd": [_GP, _INT, _P, _P, _P, _F, _P, _P, _P],
     "vattn_hier_fwd": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_hier_bwd": [_GP, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
+    "vattn_sta_fwd_fp8": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_host": [_GP, _P, _P, _P, _F, _P, _P, _I64, _P, _SZ, _P],
     "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "vattn_dual_sym_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
@@ -207,6 +209,15 @@ def vattn_hier_bwd(geom: Geom, q, k, v, o, lse, dout, scale: float, dq, dk, dv, 
         ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.vattn_hier_bwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), scale,
                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def vattn_sta_fwd_fp8(geom: Geom, q, k, v, scale: float, o, lse=None, workspace=None, ws_bytes: int = 0,
+                      stream=None) -> None:
+    """Sliding-tile forward with e4m3 Q*K^T (per-head absmax scales), bf16 P*V."""
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_sta_fwd_fp8(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
+                                 _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def vattn_sta_fwd_host(geom: Geom, q, k, v, scale: float, o, lse, chunk_slices: int, workspace,

@@ -41,13 +41,17 @@ constexpr float RESCALE_LOG2_THRESHOLD = 8.0f;
 #endif
 constexpr int POLY_CHUNK = VATTN_POLY_CHUNK;
 
-template <int D>
+// F8: Q and K are e4m3 bytes (one 128-byte box per row at d = 128), V bf16.
+template <int D, bool F8 = false>
 struct Smem {
   static constexpr int CHUNKS = D / 64;                 // 64-column (128-byte) swizzle boxes
   static constexpr int BLOCK_BYTES = CHUNKS * 128 * 128; // 128 rows x D bf16
+  static constexpr int QK_CHUNKS = F8 ? D / 128 : CHUNKS;   // 128-byte boxes per Q / K row
+  static constexpr int QK_ELEMS = F8 ? 128 : 64;            // elements per box row
+  static constexpr int QK_BYTES = QK_CHUNKS * 128 * 128;    // 128 rows of Q or K
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + BLOCK_BYTES;
-  static constexpr int OFF_V = OFF_K + NK * BLOCK_BYTES;
+  static constexpr int OFF_K = OFF_Q + QK_BYTES;
+  static constexpr int OFF_V = OFF_K + NK * QK_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * BLOCK_BYTES;
   static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -73,8 +77,23 @@ struct Params {
   int kNt, kNh, kNw, cft, cfh, cfw;
   const __nv_bfloat16* merge_o;  // hierarchical: fine-key O and LSE to merge with (NULL = none)
   const float* merge_lse;
+  const int* qk_amax;            // e4m3 Q*K^T: absmax bits of Q and K per batch*head
   DevCtl ctl;
 };
+
+// D[tmem] (+)= A[smem] * B[smem], e4m3 x e4m3 -> f32, K = 32 per instruction
+__device__ __forceinline__ void mma_ss_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Instruction descriptor, kind::f8f6f4: A, B e4m3 (format 0), K-major; D f32.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 
 // Key stream of one CTA: `runs` runs of `run_len` contiguous rows.
 struct Stream {
@@ -110,11 +129,11 @@ __device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int 
   return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + o;
 }
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  using L = Smem<D>;
+  using L = Smem<D, F8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -199,20 +218,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       int issued_k = 0;
       if (!(p.ctl.debug_flags & 1)) {
-        mbar_arrive_expect_tx(q_full, L::BLOCK_BYTES);
-        for (int c = 0; c < L::CHUNKS; ++c)
-          tma_load_3d(smem + L::OFF_Q + c * BOX_BYTES, &tm_q, q_full, c * 64, q_row0, bh);
+        mbar_arrive_expect_tx(q_full, L::QK_BYTES);
+        for (int c = 0; c < L::QK_CHUNKS; ++c)
+          tma_load_3d(smem + L::OFF_Q + c * BOX_BYTES, &tm_q, q_full, c * L::QK_ELEMS, q_row0, bh);
       }
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NK, r = j / NK;
         if (!mbar_wait(&qk_done[s], (r & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&k_full[s], L::BLOCK_BYTES);
-        uint8_t* dst = smem + L::OFF_K + s * L::BLOCK_BYTES;
+        mbar_arrive_expect_tx(&k_full[s], L::QK_BYTES);
+        uint8_t* dst = smem + L::OFF_K + s * L::QK_BYTES;
         for (int u = 0; u < subs; ++u) {
           const int v = j * BN + u * p.G;
           const int row = v < L_total ? stream_row(p, st, v) : p.Nk;  // past the end: zero fill
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * 64, row, bh);
+          for (int c = 0; c < L::QK_CHUNKS; ++c)
+            tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * L::QK_ELEMS, row, bh);
         }
         ++issued_k;
       }
@@ -254,13 +273,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = j % NK;
         if (!mbar_wait(&k_full[s], (j / NK) & 1, wc)) return false;
         tc_fence_after();
-        const uint32_t kb = k_base + s * L::BLOCK_BYTES;
+        const uint32_t kb = k_base + s * L::QK_BYTES;
         const uint32_t d_tmem = tmem + (uint32_t)((j & 1) * 128);
+        // four 32-byte K-steps per 128-byte box: 16 bf16 or 32 e4m3 elements each
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < L::QK_CHUNKS * 4; ++kk) {
           const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
-                 kk > 0);
+          if constexpr (F8)
+            mma_ss_e4m3(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                        idesc_e4m3_f32(BM, BN), kk > 0);
+          else
+            mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), IDESC_QK,
+                   kk > 0);
         }
         tc_commit(&qk_done[s]);
         return true;
@@ -297,7 +321,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 128);
     const uint32_t tO = tmem + lane_addr + 256u + (uint32_t)(w * 128);
-    const float c2 = p.scale_log2;
+    float c2 = p.scale_log2;
+    if constexpr (F8) {  // S = bytes(Q) bytes(K)^T * (absmax_Q / 448) * (absmax_K / 448)
+      const float aq = __int_as_float(p.qk_amax[2 * bh]), ak = __int_as_float(p.qk_amax[2 * bh + 1]);
+      c2 *= (aq > 0.f ? aq / 448.f : 1.f) * (ak > 0.f ? ak / 448.f : 1.f);
+    }
     float m_ref = -INFINITY, l_sum = 0.f;
     int qs = w;          // qk_done stage of this group's next block (j % NK) ...
     uint32_t qph = 0;    // ... and its phase parity ((j / NK) & 1)
@@ -487,7 +515,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                     const char** err);
 
-template <int D>
+template <int D, bool F8 = false>
 static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
   using namespace fwd;
   Params p;
@@ -506,6 +534,7 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   p.cft = p.cfh = p.cfw = 1;
   p.merge_o = nullptr;
   p.merge_lse = nullptr;
+  p.qk_amax = a.qk_amax;
   int qblocks;
   if (mode == FWD_STA) {
     int G = 1;
@@ -535,14 +564,17 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   if (qblocks == 0 || bh == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
   const char* err = nullptr;
-  if (!make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) || !make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err) ||
-      !make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err))
-    return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Smem<D>::ALLOC);
+  bool maps_ok;
+  if constexpr (F8)
+    maps_ok = make_tmap_rows_u8(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows_u8(&tk, a.k, D, p.Nk, bh, p.G, &err);
+  else
+    maps_ok = make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err);
+  if (!maps_ok || !make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Smem<D, F8>::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(qblocks, (unsigned)bh);
-  attn_fwd_kernel<D><<<grid, NTHREADS, Smem<D>::ALLOC, st>>>(tq, tk, tv, p);
+  attn_fwd_kernel<D, F8><<<grid, NTHREADS, Smem<D, F8>::ALLOC, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -560,6 +592,10 @@ cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t
 }
 
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
+  if (a.qk_amax) {  // e4m3 Q*K^T: sliding tile, d = 128
+    if (g.d != 128 || mode != FWD_STA || a.kgeom) return cudaErrorInvalidValue;
+    return launch_fwd_d<128, true>(g, mode, a, st);
+  }
   if (g.d == 128) return launch_fwd_d<128>(g, mode, a, st);
   if (g.d == 64) return launch_fwd_d<64>(g, mode, a, st);
   return cudaErrorInvalidValue;

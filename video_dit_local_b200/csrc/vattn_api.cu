@@ -107,6 +107,28 @@ bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_pe
   return true;
 }
 
+// The same for rows of `d` bytes (e4m3): box = 128 bytes x box_rows x 1.
+bool make_tmap_rows_u8(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
+                       const char** err) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows_per_bh, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)rows_per_bh * d};
+  cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed";
+    return false;
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // validation
 // ---------------------------------------------------------------------------
@@ -249,6 +271,21 @@ static SymBwdWs sym_bwd_ws(const DevGeom& g) {
   w.dvp = w.dkp + pf;
   w.dqp = w.dvp + pf;
   w.total = w.dqp + pf;
+  return w;
+}
+
+// FP8 forward: e4m3 Q, K bytes and the per-batch*head absmax words.
+struct Fp8FwdWs {
+  size_t q8, k8, amax, total;
+};
+static Fp8FwdWs fp8_fwd_ws(const DevGeom& g) {
+  Fp8FwdWs w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t t = align256(bh * g.N * g.d);
+  w.q8 = 0;
+  w.k8 = t;
+  w.amax = 2 * t;
+  w.total = 2 * t + align256(bh * 2 * 4);
   return w;
 }
 
@@ -404,6 +441,7 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_STA_FWD_HOST: *bytes = host_chunk_ws(g).total; break;
     case VATTN_OP_HIER_FWD: *bytes = hier_fwd_ws(g).total; break;
     case VATTN_OP_HIER_BWD: *bytes = hier_bwd_ws(g).total; break;
+    case VATTN_OP_STA_FWD_FP8: *bytes = fp8_fwd_ws(g).total; break;
     default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
   return ok();
@@ -671,6 +709,37 @@ int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const v
   CHECK_LAUNCH(launch_bwd_dkdv_hier(g, gc, a, false, st), "hier_bwd fine dK/dV launch");
   CHECK_LAUNCH(launch_bwd_dq_hier(g, gc, a, st), "hier_bwd coarse dQ launch");
   CHECK_LAUNCH(launch_bwd_dq(g, a, true, st), "hier_bwd fine dQ launch");
+  return ok();
+}
+
+int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                      float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (g.d != 128) return fail(VATTN_ERR_UNSUPPORTED, "the FP8 forward supports head_dim 128 only");
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  const Fp8FwdWs w = fp8_fwd_ws(g);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  uint8_t* ws = (uint8_t*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  int* amax = (int*)(ws + w.amax);
+  CHECK_LAUNCH(launch_quant_qk(g, q, k, ws + w.q8, ws + w.k8, amax, st), "sta_fwd_fp8 quantise launch");
+  FwdArgs a{};
+  a.q = ws + w.q8;
+  a.k = ws + w.k8;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.scale = scale;
+  a.qk_amax = amax;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "sta_fwd_fp8 launch");
   return ok();
 }
 

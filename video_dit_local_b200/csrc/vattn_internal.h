@@ -53,6 +53,11 @@ cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void*
 // pooled grid cut into tiles (the coarse tiles of the hierarchical branch).
 cudaError_t launch_pool_kv_tiled(const DevGeom& g, const DevGeom& gc, const void* k, const void* v, void* kp,
                                  void* vp, cudaStream_t st);
+// Q and K to e4m3 bytes with one scale per batch*head and tensor: amax[2 bh]
+// (Q) and amax[2 bh + 1] (K) receive the absmax as float bits; the dequantised
+// value is byte * amax / 448.
+cudaError_t launch_quant_qk(const DevGeom& g, const void* q, const void* k, void* q8, void* k8, int* amax,
+                            cudaStream_t st);
 cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, const void* v, void* qp, void* kp,
                             void* vp, cudaStream_t st);
 cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void* o_l, const float* gvec, void* out,
@@ -81,6 +86,10 @@ struct FwdArgs {
   int cf[3];
   const void* merge_o;
   const float* merge_lse;
+  // STA only: q and k hold e4m3 bytes (Q*K^T on the f8f6f4 tensor path);
+  // qk_amax[2 bh] / [2 bh + 1] are the absmax float bits of Q / K (scale
+  // absmax / 448).  d = 128 only.
+  const int* qk_amax;
 };
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st);
@@ -136,5 +145,7 @@ cudaError_t launch_bwd_dq_hier(const DevGeom& g, const DevGeom& gc, const BwdArg
 // fills *err on failure.
 bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                     const char** err);
+bool make_tmap_rows_u8(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
+                       const char** err);
 
 }  // namespace vattn
