@@ -121,3 +121,24 @@ def test_fp8_fwd_equals_oracle_on_dequantised_inputs(V, grid, tile, window, batc
         assert_close(to_f64(o_r[b, h]), o_ex[0, 0], FP8_O_MAX_ABS, FP8_O_MEAN_ABS, f"O vs exact b{b} h{h}")
         assert_close(lse_r[b, h].cpu().numpy().astype(np.float64), lse_ex[0, 0], FP8_LSE_MAX_ABS,
                      what=f"LSE vs exact b{b} h{h}")
+
+
+def test_fp8_fwd_720p_sampled(V):
+    """The benchmarked 720p workload, all 24 heads in one launch; heads 0 and
+    23 compared on query tiles covering every boundary class, against the
+    oracle on their dequantised Q and K."""
+    from helpers import sample_tiles
+    w = S.WORKLOADS["720p"]
+    check = [(0, 0), (0, w.heads - 1)]
+    _, _, q8, k8, amax, o_r, lse_r = _run(V, w, check)
+    g = O.geom_of(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    tiles = sample_tiles(g.tiles_per_dim, 10)
+    for b, h in check:
+        i = b * w.heads + h
+        qd = O.unpermute(_dequant(q8[b, h], amax[i, 0]), g)
+        kd = O.unpermute(_dequant(k8[b, h], amax[i, 1]), g)
+        v = host_f64(w, S.V_ID, b, h)
+        ids, o_ref, lse_ref = O.sta_attention_tiles(qd, kd, v, g, scale, tiles)
+        assert_close(to_f64(o_r[b, h])[ids], o_ref, O_MAX_ABS, O_MEAN_ABS, f"O b{b} h{h}")
+        assert_close(lse_r[b, h].cpu().numpy().astype(np.float64)[ids], lse_ref, LSE_MAX_ABS, what=f"LSE b{b} h{h}")

@@ -125,3 +125,30 @@ def test_sta_fwd_host_720p_sampled(V):
     (o, lse), = _host_path(V, geom, w, qh, kh, vh, scale, 3)
     assert torch_equal_bits(o, o_ref) and torch_equal_bits(lse, lse_ref)
     torch.cuda.empty_cache()
+
+
+def test_sta_fwd_host_back_to_back_calls_from_two_streams(V):
+    """Two calls with different inputs, issued from two streams and sharing
+    one workspace: the library orders them on its own streams, so both
+    results equal the device path."""
+    import torch
+    w = S.small_workload("host_2s", 34, 1, 4, 128, (6, 16, 16), (3, 8, 8), (1, 1, 3), (1, 1, 1))
+    check = [(0, h) for h in range(4)]
+    geom = geom_for(V, w)
+    scale = 1 / math.sqrt(128)
+    qr, kr, vr = (gpu_tensor(w, i, check) for i in (S.Q_ID, S.K_ID, S.V_ID))
+    q2, k2, v2 = (x.flip(2).contiguous() for x in (qr, kr, vr))   # a second, different input set
+    ref1, _ = _device_path(V, geom, qr, kr, vr, scale)
+    ref2, _ = _device_path(V, geom, q2, k2, v2, scale)
+    one = V.make_geom(1, 2, 128, w.grid, w.tile, w.window, w.pool)
+    ws = torch.empty(2 * V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, one), dtype=torch.uint8, device="cuda")
+    ins1 = [x.cpu().pin_memory() for x in (qr, kr, vr)]
+    ins2 = [x.cpu().pin_memory() for x in (q2, k2, v2)]
+    o1 = torch.empty(qr.shape, dtype=torch.bfloat16).pin_memory()
+    o2 = torch.empty(qr.shape, dtype=torch.bfloat16).pin_memory()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    V.vattn_sta_fwd_host(geom, *ins1, scale, o1, None, 2, ws, stream=s1)
+    V.vattn_sta_fwd_host(geom, *ins2, scale, o2, None, 2, ws, stream=s2)
+    torch.cuda.synchronize()
+    assert V.vattn_get_status() == 0, V.vattn_last_error()
+    assert torch_equal_bits(o1, ref1) and torch_equal_bits(o2, ref2)

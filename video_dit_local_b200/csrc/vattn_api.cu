@@ -353,6 +353,7 @@ static HostChunkWs host_chunk_ws(const DevGeom& g) {
 struct HostPipe {
   cudaStream_t in = nullptr, comp = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+  cudaEvent_t last = nullptr;  // the previous call's end on these streams
   std::mutex mu;
   bool ready = false;
 };
@@ -368,6 +369,7 @@ static cudaError_t host_pipe_init(HostPipe& p) {
   if ((e = cudaStreamCreateWithFlags(&p.comp, cudaStreamNonBlocking)) != cudaSuccess) return e;
   if ((e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
   if ((e = cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming)) != cudaSuccess) return e;
+  if ((e = cudaEventCreateWithFlags(&p.last, cudaEventDisableTiming)) != cudaSuccess) return e;
   for (int i = 0; i < 2; ++i) {
     if ((e = cudaEventCreateWithFlags(&p.in_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&p.comp_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
@@ -553,6 +555,11 @@ int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, con
   HostPipe& p = *pp;
   cudaStream_t caller = (cudaStream_t)stream;
   CHECK_LAUNCH(cudaEventRecord(p.start, caller), "event record");
+  // the library streams also wait for the previous call's end (its caller may
+  // have used another stream): its staging slots are reused below.  Waiting
+  // on a never-recorded event is a no-op.
+  CHECK_LAUNCH(cudaStreamWaitEvent(p.in, p.last, 0), "stream wait");
+  CHECK_LAUNCH(cudaStreamWaitEvent(p.comp, p.last, 0), "stream wait");
   CHECK_LAUNCH(cudaStreamWaitEvent(p.in, p.start, 0), "stream wait");
   CHECK_LAUNCH(cudaStreamWaitEvent(p.comp, p.start, 0), "stream wait");
   CHECK_LAUNCH(cudaStreamWaitEvent(p.out, p.start, 0), "stream wait");
@@ -601,6 +608,7 @@ int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, con
   // the caller's stream waits for every copy-out (and therefore for everything)
   for (int slot = 0; slot < 2 && slot < nchunks; ++slot)
     CHECK_LAUNCH(cudaStreamWaitEvent(caller, p.out_done[slot], 0), "stream wait");
+  CHECK_LAUNCH(cudaEventRecord(p.last, p.out), "event record");
   return ok();
 }
 
