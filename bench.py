@@ -221,29 +221,23 @@ def run_ours(args, rank, world, local_rank):
     pinned = [torch.from_numpy(h).pin_memory() for h in host]
     shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
     qr, kr, vr = (p.to(dev).view(torch.bfloat16) for p in pinned)
-    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
-    o = torch.empty_like(q)
-    o_r = torch.empty_like(q)
-    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
-    lse_r = torch.empty_like(lse)
+    o_r = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    lse_r = torch.empty(shape[:3], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     kernel_events = []
 
     def step(record=False):
-        V.vattn_tile_permute(geom, qr, q)
-        V.vattn_tile_permute(geom, kr, k)
-        V.vattn_tile_permute(geom, vr, v)
+        # raster Q, K, V in, raster O and LSE out: the tile reorder is done by
+        # the kernel's tensor-map boxes and epilogue stores (one launch)
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        V.vattn_sta_fwd(geom, q, k, v, scale, o, lse)
+        V.vattn_sta_fwd_raster(geom, qr, kr, vr, scale, o_r, lse_r)
         if record:
             e1.record(stream)
             kernel_events.append((e0, e1))
-        V.vattn_tile_unpermute(geom, o, o_r)
-        V.vattn_tile_unpermute(geom, lse, lse_r, 4)
 
-    launches_per_step = 6
+    launches_per_step = 1
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -332,13 +326,13 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"720p sliding-tile fwd: B1 h{w.heads} d128, grid 30x48x80, tile 6x8x8, window 3x3x3",
                    "global_batch": w.batch * world, "seq_len": w.n_tokens, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (2.1 GB Q/K/V), no flush",
-                   "step": "permute Q,K,V + sta_fwd + unpermute O,LSE"},
+                   "step": "sta_fwd on raster Q,K,V -> raster O,LSE (tile reorder fused into the kernel)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "peak_source": f"{peak_src} bf16 (burst)", "traffic": traffic,
-                     "kernel": "attn_fwd_kernel<128> (sliding tile)", "kernel_ms": round(ms_kernel, 4),
+                     "kernel": "attn_fwd_kernel<128> (sliding tile, raster tensor-map boxes)", "kernel_ms": round(ms_kernel, 4),
                      "algorithmic_flop_per_launch": flops_local},
         "e2e": {"value": round(whole_job_tflops(flops_local, ms_e2e, world), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -161,6 +161,17 @@ int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const v
                    const float* lse, const void* dout, float scale, void* dq, void* dk, void* dv, void* workspace,
                    size_t ws_bytes, void* stream);
 
+/* Sliding-tile forward on RASTER-order tensors: the raster <-> tile-major
+ * reorder (vattn_tile_permute / unpermute) fused into the attention kernel.
+ * q, k, v [B,h,N,d] bf16 raster; o bf16 raster; lse fp32 [B,h,N] raster or
+ * NULL.  The kernel's loads are boxes of whole t-slices of a tile (5-D tensor
+ * maps), so a tile's t-slice of th*tw tokens must divide 128 and the key
+ * sub-box (the largest power of two <= 128 dividing the tile volume); else
+ * VATTN_ERR_UNSUPPORTED.  The result equals vattn_tile_permute +
+ * vattn_sta_fwd + vattn_tile_unpermute bit for bit. */
+int vattn_sta_fwd_raster(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                         float* lse, void* stream);
+
 /* Sliding-tile forward with Q*K^T in FP8 (e4m3) on the f8f6f4 tensor path,
  * P*V in bf16: an inference variant in the spirit of the 8-bit attention the
  * pages cite ("SageAttention"), which the pages do not define further.
@@ -176,8 +187,9 @@ int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, cons
 
 /* Sliding-tile forward on HOST buffers in raster order, pipelined.  The
  * batch*head range is cut into chunks of `chunk_slices` slices; for every
- * chunk the host->device copy of Q, K, V, the permute + vattn_sta_fwd +
- * unpermute, and the device->host copy of O (and LSE) run on three library
+ * chunk the host->device copy of Q, K, V, the attention (the raster kernel
+ * of vattn_sta_fwd_raster when the tile allows it, else permute +
+ * vattn_sta_fwd + unpermute), and the device->host copy of O (and LSE) run on three library
  * streams, so that copies in both directions overlap the compute of the
  * neighbouring chunks (two staging slots, reused in turn).
  *  q, k, v : host bf16 [B,h,N,d] raster; o: host bf16 raster; lse: host fp32

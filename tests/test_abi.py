@@ -93,6 +93,9 @@ def test_argument_errors(V):
     with pytest.raises(V.VattnError) as e:
         V.vattn_hier_fwd(g, 16, 16, 16, 0.1, 16, None, 32, 64)
     assert e.value.code == B.VATTN_ERR_WORKSPACE
+    with pytest.raises(V.VattnError) as e:   # t-slice of 6 x 8 = 48 tokens does not divide 128
+        V.vattn_sta_fwd_raster(_geom(V, grid=(4, 12, 16), tile=(2, 6, 8)), 16, 16, 16, 0.1, 16)
+    assert e.value.code == B.VATTN_ERR_UNSUPPORTED and "t-slice" in str(e.value)
     with pytest.raises(V.VattnError) as e:   # the FP8 forward is d = 128 only
         V.vattn_sta_fwd_fp8(_geom(V, head_dim=64), 16, 16, 16, 0.1, 16, None, 32, 1 << 30)
     assert e.value.code == B.VATTN_ERR_UNSUPPORTED

@@ -88,6 +88,7 @@ _SIGS = {
     "vattn_xwin_fwd": [_GP, _INT, _P, _P, _P, _F, _P, _P, _P],
     "vattn_hier_fwd": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_hier_bwd": [_GP, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
+    "vattn_sta_fwd_raster": [_GP, _P, _P, _P, _F, _P, _P, _P],
     "vattn_sta_fwd_fp8": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_host": [_GP, _P, _P, _P, _F, _P, _P, _I64, _P, _SZ, _P],
     "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
@@ -209,6 +210,12 @@ def vattn_hier_bwd(geom: Geom, q, k, v, o, lse, dout, scale: float, dq, dk, dv, 
         ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib.vattn_hier_bwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), scale,
                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def vattn_sta_fwd_raster(geom: Geom, q, k, v, scale: float, o, lse=None, stream=None) -> None:
+    """Sliding-tile forward on raster-order tensors (reorder fused into the kernel)."""
+    _check(lib.vattn_sta_fwd_raster(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
+                                    _stream(stream)))
 
 
 def vattn_sta_fwd_fp8(geom: Geom, q, k, v, scale: float, o, lse=None, workspace=None, ws_bytes: int = 0,

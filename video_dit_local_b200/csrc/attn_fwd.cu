@@ -78,8 +78,22 @@ struct Params {
   const __nv_bfloat16* merge_o;  // hierarchical: fine-key O and LSE to merge with (NULL = none)
   const float* merge_lse;
   const int* qk_amax;            // e4m3 Q*K^T: absmax bits of Q and K per batch*head
+  // raster (STA only): Q, K, V, O and LSE in raster token order.  The tensor
+  // maps are 5-D (d, W, H, T, batch*head); a load is a box of whole t-slices
+  // of one tile, which lands in shared memory in the tile-major row order.
+  int raster;
   DevCtl ctl;
 };
+
+__device__ __forceinline__ void tma_load_5d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], "
+      "[%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
 
 // D[tmem] (+)= A[smem] * B[smem], e4m3 x e4m3 -> f32, K = 32 per instruction
 __device__ __forceinline__ void mma_ss_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -129,6 +143,25 @@ __device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int 
   return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + o;
 }
 
+// Raster box of key stream position v (a multiple of the sub-box rows): the
+// x, y, t of its first token; past the end, t = T (a zero-filled box).
+__device__ __forceinline__ void stream_box(const Params& p, const Stream& s, int v, int L_total, int* x, int* y,
+                                           int* t) {
+  const DevGeom& g = p.g;
+  if (v >= L_total) {
+    *x = 0;
+    *y = 0;
+    *t = g.T;
+    return;
+  }
+  const int r = v / s.run_len, o = v - r * s.run_len;
+  const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
+  const int tile_in_run = o / g.s, lo = o - tile_in_run * g.s;
+  *x = (s.w0 + tile_in_run) * g.tw;
+  *y = kh * g.th;
+  *t = kt * g.tt + lo / (g.th * g.tw);
+}
+
 template <int D, bool F8 = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -164,10 +197,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   wc.err_word = p.ctl.err_word;
 
   // query block -> rows
-  int q_tile, q_row0, q_valid;
+  int q_tile, q_row0, q_valid, sub = 0;
   if (p.mode == FWD_STA) {
     q_tile = qblk / p.q_blocks_per_tile;
-    const int sub = qblk - q_tile * p.q_blocks_per_tile;
+    sub = qblk - q_tile * p.q_blocks_per_tile;
     q_row0 = q_tile * p.g.s + sub * BM;
     q_valid = min(BM, p.g.s - sub * BM);
   } else {
@@ -219,8 +252,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int issued_k = 0;
       if (!(p.ctl.debug_flags & 1)) {
         mbar_arrive_expect_tx(q_full, L::QK_BYTES);
-        for (int c = 0; c < L::QK_CHUNKS; ++c)
-          tma_load_3d(smem + L::OFF_Q + c * BOX_BYTES, &tm_q, q_full, c * L::QK_ELEMS, q_row0, bh);
+        if (p.raster) {
+          const DevGeom& g = p.g;
+          const int at = q_tile / (g.Nh * g.Nw), ah = (q_tile / g.Nw) % g.Nh, aw = q_tile % g.Nw;
+          const int t0 = at * g.tt + sub * BM / (g.th * g.tw);
+          for (int c = 0; c < L::QK_CHUNKS; ++c)
+            tma_load_5d(smem + L::OFF_Q + c * BOX_BYTES, &tm_q, q_full, c * L::QK_ELEMS, aw * g.tw, ah * g.th, t0, bh);
+        } else {
+          for (int c = 0; c < L::QK_CHUNKS; ++c)
+            tma_load_3d(smem + L::OFF_Q + c * BOX_BYTES, &tm_q, q_full, c * L::QK_ELEMS, q_row0, bh);
+        }
       }
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NK, r = j / NK;
@@ -229,9 +270,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* dst = smem + L::OFF_K + s * L::QK_BYTES;
         for (int u = 0; u < subs; ++u) {
           const int v = j * BN + u * p.G;
-          const int row = v < L_total ? stream_row(p, st, v) : p.Nk;  // past the end: zero fill
-          for (int c = 0; c < L::QK_CHUNKS; ++c)
-            tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * L::QK_ELEMS, row, bh);
+          if (p.raster) {
+            int x, y, t;
+            stream_box(p, st, v, L_total, &x, &y, &t);
+            for (int c = 0; c < L::QK_CHUNKS; ++c)
+              tma_load_5d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * L::QK_ELEMS, x, y, t, bh);
+          } else {
+            const int row = v < L_total ? stream_row(p, st, v) : p.Nk;  // past the end: zero fill
+            for (int c = 0; c < L::QK_CHUNKS; ++c)
+              tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * L::QK_ELEMS, row, bh);
+          }
         }
         ++issued_k;
       }
@@ -250,9 +298,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* dst = smem + L::OFF_V + s * L::BLOCK_BYTES;
         for (int u = 0; u < subs; ++u) {
           const int v = j * BN + u * p.G;
-          const int row = v < L_total ? stream_row(p, st, v) : p.Nk;
-          for (int c = 0; c < L::CHUNKS; ++c)
-            tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * 64, row, bh);
+          if (p.raster) {
+            int x, y, t;
+            stream_box(p, st, v, L_total, &x, &y, &t);
+            for (int c = 0; c < L::CHUNKS; ++c)
+              tma_load_5d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * 64, x, y, t, bh);
+          } else {
+            const int row = v < L_total ? stream_row(p, st, v) : p.Nk;
+            for (int c = 0; c < L::CHUNKS; ++c)
+              tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * 64, row, bh);
+          }
         }
         ++issued_v;
       }
@@ -433,7 +488,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float a1 = (w == 0 ? a_other : a_self) * inv_l;
       const bool have1 = nblk >= 2;
       const bool row_ok = row < q_valid;
-      const size_t grow = (size_t)bh * p.g.N + (size_t)(q_row0 + row);
+      size_t grow = (size_t)bh * p.g.N + (size_t)(q_row0 + row);
+      if (p.raster) {  // tile-major row -> raster token
+        const DevGeom& g = p.g;
+        const int at = q_tile / (g.Nh * g.Nw), ah = (q_tile / g.Nw) % g.Nh, aw = q_tile % g.Nw;
+        const int lr = sub * BM + row;
+        const int lt = lr / (g.th * g.tw), lh = (lr / g.tw) % g.th, lw = lr % g.tw;
+        grow = (size_t)bh * g.N + ((size_t)(at * g.tt + lt) * g.H + (ah * g.th + lh)) * g.W + (aw * g.tw + lw);
+      }
       // hierarchical merge: one softmax over the fine keys (O_f, LSE_f given)
       // and this kernel's coarse keys, in log2 units
       float wf = 0.f, wc = 1.f, lse2_out = m + __log2f(l);
@@ -535,6 +597,7 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   p.merge_o = nullptr;
   p.merge_lse = nullptr;
   p.qk_amax = a.qk_amax;
+  p.raster = a.raster ? 1 : 0;
   int qblocks;
   if (mode == FWD_STA) {
     int G = 1;
@@ -565,6 +628,19 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   CUtensorMap tq, tk, tv;
   const char* err = nullptr;
   bool maps_ok;
+  if (p.raster) {  // 5-D raster maps: boxes of whole t-slices of one tile
+    const int slice = g.th * g.tw;
+    if (F8 || mode != FWD_STA || a.kgeom || BM % slice || p.G % slice) return cudaErrorInvalidValue;
+    maps_ok = make_tmap_raster(&tq, a.q, D, g, bh, BM / slice, &err) &&
+              make_tmap_raster(&tk, a.k, D, g, bh, p.G / slice, &err) &&
+              make_tmap_raster(&tv, a.v, D, g, bh, p.G / slice, &err);
+    if (!maps_ok) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Smem<D, F8>::ALLOC);
+    if (e != cudaSuccess) return e;
+    attn_fwd_kernel<D, F8><<<dim3(qblocks, (unsigned)bh), NTHREADS, Smem<D, F8>::ALLOC, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+  }
   if constexpr (F8)
     maps_ok = make_tmap_rows_u8(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows_u8(&tk, a.k, D, p.Nk, bh, p.G, &err);
   else

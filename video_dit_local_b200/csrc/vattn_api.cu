@@ -107,6 +107,28 @@ bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_pe
   return true;
 }
 
+bool make_tmap_raster(CUtensorMap* map, const void* base, int d, const DevGeom& g, long long bh, int box_t,
+                      const char** err) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  const cuuint64_t row = (cuuint64_t)d * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T, (cuuint64_t)bh};
+  cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
+  cuuint32_t box[5] = {64, (cuuint32_t)g.tw, (cuuint32_t)g.th, (cuuint32_t)box_t, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed";
+    return false;
+  }
+  return true;
+}
+
 // The same for rows of `d` bytes (e4m3): box = 128 bytes x box_rows x 1.
 bool make_tmap_rows_u8(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                        const char** err) {
@@ -565,6 +587,10 @@ int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, con
   CHECK_LAUNCH(cudaStreamWaitEvent(p.out, p.start, 0), "stream wait");
   const size_t row = (size_t)g.N * g.d * 2, lrow = (size_t)g.N * 4;
   const int nchunks = (int)((total + chunk_slices - 1) / chunk_slices);
+  // the tile reorder fused into the kernel when the t-slice allows it
+  int G = 1;
+  while (G < 128 && g.s % (G * 2) == 0) G *= 2;
+  const bool raster = 128 % (g.th * g.tw) == 0 && G % (g.th * g.tw) == 0;
   for (int c = 0; c < nchunks; ++c) {
     const int slot = c & 1;
     const long long s0 = (long long)c * chunk_slices;
@@ -584,19 +610,31 @@ int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, con
     CHECK_LAUNCH(cudaMemcpyAsync(ws + w.vr, (const uint8_t*)v + s0 * row, bytes, cudaMemcpyHostToDevice, p.in), "H2D v");
     CHECK_LAUNCH(cudaEventRecord(p.in_done[slot], p.in), "event record");
     CHECK_LAUNCH(cudaStreamWaitEvent(p.comp, p.in_done[slot], 0), "stream wait");
-    CHECK_LAUNCH(launch_permute(gk, ws + w.qr, ws + w.qt, g.d * 2, true, p.comp), "permute q");
-    CHECK_LAUNCH(launch_permute(gk, ws + w.kr, ws + w.kt, g.d * 2, true, p.comp), "permute k");
-    CHECK_LAUNCH(launch_permute(gk, ws + w.vr, ws + w.vt, g.d * 2, true, p.comp), "permute v");
-    FwdArgs a{};
-    a.q = ws + w.qt;
-    a.k = ws + w.kt;
-    a.v = ws + w.vt;
-    a.o = ws + w.ot;
-    a.lse = lse ? (float*)(ws + w.lt) : nullptr;
-    a.scale = scale;
-    CHECK_LAUNCH(launch_attn_fwd(gk, FWD_STA, a, p.comp), "sta_fwd");
-    CHECK_LAUNCH(launch_permute(gk, ws + w.ot, ws + w.orr, g.d * 2, false, p.comp), "unpermute o");
-    if (lse) CHECK_LAUNCH(launch_permute(gk, ws + w.lt, ws + w.lr, 4, false, p.comp), "unpermute lse");
+    if (raster) {
+      FwdArgs a{};
+      a.q = ws + w.qr;
+      a.k = ws + w.kr;
+      a.v = ws + w.vr;
+      a.o = ws + w.orr;
+      a.lse = lse ? (float*)(ws + w.lr) : nullptr;
+      a.scale = scale;
+      a.raster = true;
+      CHECK_LAUNCH(launch_attn_fwd(gk, FWD_STA, a, p.comp), "sta_fwd (raster)");
+    } else {
+      CHECK_LAUNCH(launch_permute(gk, ws + w.qr, ws + w.qt, g.d * 2, true, p.comp), "permute q");
+      CHECK_LAUNCH(launch_permute(gk, ws + w.kr, ws + w.kt, g.d * 2, true, p.comp), "permute k");
+      CHECK_LAUNCH(launch_permute(gk, ws + w.vr, ws + w.vt, g.d * 2, true, p.comp), "permute v");
+      FwdArgs a{};
+      a.q = ws + w.qt;
+      a.k = ws + w.kt;
+      a.v = ws + w.vt;
+      a.o = ws + w.ot;
+      a.lse = lse ? (float*)(ws + w.lt) : nullptr;
+      a.scale = scale;
+      CHECK_LAUNCH(launch_attn_fwd(gk, FWD_STA, a, p.comp), "sta_fwd");
+      CHECK_LAUNCH(launch_permute(gk, ws + w.ot, ws + w.orr, g.d * 2, false, p.comp), "unpermute o");
+      if (lse) CHECK_LAUNCH(launch_permute(gk, ws + w.lt, ws + w.lr, 4, false, p.comp), "unpermute lse");
+    }
     CHECK_LAUNCH(cudaEventRecord(p.comp_done[slot], p.comp), "event record");
     CHECK_LAUNCH(cudaStreamWaitEvent(p.out, p.comp_done[slot], 0), "stream wait");
     CHECK_LAUNCH(cudaMemcpyAsync((uint8_t*)o + s0 * row, ws + w.orr, bytes, cudaMemcpyDeviceToHost, p.out), "D2H o");
@@ -717,6 +755,34 @@ int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const v
   CHECK_LAUNCH(launch_bwd_dkdv_hier(g, gc, a, false, st), "hier_bwd fine dK/dV launch");
   CHECK_LAUNCH(launch_bwd_dq_hier(g, gc, a, st), "hier_bwd coarse dQ launch");
   CHECK_LAUNCH(launch_bwd_dq(g, a, true, st), "hier_bwd fine dQ launch");
+  return ok();
+}
+
+int vattn_sta_fwd_raster(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
+                         float* lse, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  const int slice = g.th * g.tw;
+  int G = 1;
+  while (G < 128 && g.s % (G * 2) == 0) G *= 2;
+  if (128 % slice || G % slice)
+    return fail(VATTN_ERR_UNSUPPORTED, "tile t-slice of %d tokens must divide 128 and the key sub-box of %d rows", slice,
+                G);
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(o);
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.scale = scale;
+  a.raster = true;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, (cudaStream_t)stream), "sta_fwd_raster launch");
   return ok();
 }
 

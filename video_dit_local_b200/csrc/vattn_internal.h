@@ -90,6 +90,9 @@ struct FwdArgs {
   // qk_amax[2 bh] / [2 bh + 1] are the absmax float bits of Q / K (scale
   // absmax / 448).  d = 128 only.
   const int* qk_amax;
+  // STA only: q, k, v, o and lse in raster token order (5-D tensor maps; the
+  // tile's t-slice, th*tw rows, must divide 128 and the key sub-box)
+  bool raster;
 };
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st);
@@ -145,6 +148,10 @@ cudaError_t launch_bwd_dq_hier(const DevGeom& g, const DevGeom& gc, const BwdArg
 // fills *err on failure.
 bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                     const char** err);
+// 5-D map over a raster [bh][T][H][W][d] bf16 tensor: box = 64 elements x
+// tile-w x tile-h x box_t t-slices x 1, 128-byte swizzle.
+bool make_tmap_raster(CUtensorMap* map, const void* base, int d, const DevGeom& g, long long bh, int box_t,
+                      const char** err);
 bool make_tmap_rows_u8(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                        const char** err);
 
