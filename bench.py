@@ -388,7 +388,40 @@ def run_extras(V, dev):
     out["1080p_dual_sym_fwd"] = _bench_sym(V, dev, peaks)
     out["720p_hier_fwd_bwd"] = _bench_hier(V, dev, peaks)
     out["720p_sta_fwd_fp8"] = _bench_fp8(V, dev, peaks)
+    out["1080p_dual_fwd_fp8"] = _bench_dual_fp8(V, dev, peaks)
     return out
+
+
+def _bench_dual_fp8(V, dev, peaks):
+    """The 1080p dual forward with e4m3 Q*K^T in both branches (pooling and
+    quantisation included in the timed call); effective FLOPs as the bf16
+    dual forward, fraction of the bf16 peak."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["1080p"]
+    geom = _geom(V, w)
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 900 + i) for i in range(3))
+    gvec = torch.rand(w.heads, device=dev)
+    o = torch.empty_like(q)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD_FP8, geom), dtype=torch.uint8, device=dev)
+    fl, fg = _flops_fwd(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    for _ in range(2):
+        V.vattn_dual_fwd_fp8(geom, q, k, v, gvec, scale, o, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(4):
+        V.vattn_dual_fwd_fp8(geom, q, k, v, gvec, scale, o, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 4
+    res = {"ms": round(ms, 3), "eff_tflops": round((fl + fg) / ms / 1e9, 1),
+           "frac_of_bf16_peak": round((fl + fg) / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status()}
+    del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def _bench_fp8(V, dev, peaks):

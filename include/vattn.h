@@ -83,7 +83,8 @@ enum {
   VATTN_OP_STA_FWD_HOST = 6, /* per chunk of batch*head slices: pass heads = the chunk size in geom */
   VATTN_OP_HIER_FWD = 7,     /* geom->pool = the medium pool factor h_pool */
   VATTN_OP_HIER_BWD = 8,
-  VATTN_OP_STA_FWD_FP8 = 9
+  VATTN_OP_STA_FWD_FP8 = 9,
+  VATTN_OP_DUAL_FWD_FP8 = 10
 };
 
 /* Raster -> tile-major row gather.  Tile-major position of raster token
@@ -184,6 +185,17 @@ int vattn_sta_fwd_raster(const vattn_geom* geom, const void* q, const void* k, c
  * bits as int32 [B*h][2] (Q, K); they hold this call's values afterwards. */
 int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
                       float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/* Dual forward (inference) with both branches' Q*K^T in FP8 (e4m3), as
+ * vattn_sta_fwd_fp8: O = g*O_local + (1-g)*O_global with K_p, V_p the bf16
+ * average pools of K, V (as vattn_pool_kv), and Q, K, K_p quantised with one
+ * absmax scale per batch*head each.  Tile-major q, k, v, o; g fp32 [heads].
+ * workspace >= vattn_workspace_size(VATTN_OP_DUAL_FWD_FP8), in this order
+ * (each part starting on a 256-byte boundary): e4m3 Q, e4m3 K [B,h,N,d];
+ * e4m3 K_p [B,h,N_p,d]; absmax bits int32 [B*h][2] of (Q, K) and of (Q, K_p);
+ * bf16 O_local [B,h,N,d]; bf16 K_p, V_p [B,h,N_p,d].  d = 128 only. */
+int vattn_dual_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* g, float scale,
+                       void* o, void* workspace, size_t ws_bytes, void* stream);
 
 /* Sliding-tile forward on HOST buffers in raster order, pipelined.  The
  * batch*head range is cut into chunks of `chunk_slices` slices; for every

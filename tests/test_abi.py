@@ -124,6 +124,9 @@ def test_workspace_sizes(V):
     # hierarchical forward (pool = h_pool): pooled K, V, then fine O and LSE
     assert V.vattn_workspace_size(V.VATTN_OP_HIER_FWD, g) == (2 * a(bh * npool * d * 2) + a(bh * n * d * 2)
                                                               + a(bh * n * 4))
+    # FP8 dual forward: e4m3 Q, K, K_p; two absmax pairs; bf16 O_local, K_p, V_p
+    assert V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD_FP8, g) == (
+        2 * a(bh * n * d) + a(bh * npool * d) + 2 * a(bh * 8) + a(bh * n * d * 2) + 2 * a(bh * npool * d * 2))
     # FP8 forward: e4m3 Q and K bytes, then two absmax words per batch*head
     assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_FP8, g) == 2 * a(bh * n * d) + a(bh * 8)
     # host-buffer forward, per slot: 8 bf16 token tensors and 2 fp32 rows

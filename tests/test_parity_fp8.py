@@ -142,3 +142,69 @@ def test_fp8_fwd_720p_sampled(V):
         ids, o_ref, lse_ref = O.sta_attention_tiles(qd, kd, v, g, scale, tiles)
         assert_close(to_f64(o_r[b, h])[ids], o_ref, O_MAX_ABS, O_MEAN_ABS, f"O b{b} h{h}")
         assert_close(lse_r[b, h].cpu().numpy().astype(np.float64)[ids], lse_ref, LSE_MAX_ABS, what=f"LSE b{b} h{h}")
+
+
+def _a256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("grid,tile,window,pool,batch,heads", [
+    ((6, 16, 24), (3, 8, 8), (1, 3, 3), (1, 4, 4), 1, 2),   # tile 192, N_p = 144
+    ((6, 16, 32), (6, 8, 8), (1, 3, 3), (2, 2, 2), 2, 1),   # temporal pooling, batch 2
+])
+def test_dual_fp8_fwd(V, grid, tile, window, pool, batch, heads):
+    """vattn_dual_fwd_fp8: the K_p bytes and the shared Q scale bit-exact; the
+    blended output against the oracle on the dequantised operands (bf16 bars)
+    and against the exact dual oracle (e4m3 bars)."""
+    import torch
+    w = S.small_workload("fp8dual", 73, batch, heads, 128, grid, tile, window, pool)
+    check = [(b, h) for b in range(batch) for h in range(heads)]
+    g = O.geom_of(w)
+    geom = geom_for(V, w)
+    tiled = []
+    for tid in (S.Q_ID, S.K_ID, S.V_ID):
+        x = gpu_tensor(w, tid, check)
+        t = torch.empty_like(x)
+        V.vattn_tile_permute(geom, x, t)
+        tiled.append(t)
+    q, k, v = tiled
+    gvec = torch.from_numpy(S.blend_g(w)).cuda()
+    o = torch.empty_like(q)
+    ws = torch.zeros(V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD_FP8, geom), dtype=torch.uint8, device="cuda")
+    scale = 1 / math.sqrt(128)
+    V.vattn_dual_fwd_fp8(geom, q, k, v, gvec, scale, o, ws)
+    o_r = torch.empty_like(o)
+    V.vattn_tile_unpermute(geom, o, o_r)
+    torch.cuda.synchronize()
+    assert V.vattn_get_status() == 0, V.vattn_last_error()
+    bh, n, npl = batch * heads, g.n, g.n_pooled
+    t8, p8, am = _a256(bh * n * 128), _a256(bh * npl * 128), _a256(bh * 8)
+    off_kp8, off_al = 2 * t8, 2 * t8 + p8
+    off_ag, off_ol = off_al + am, off_al + 2 * am
+    off_kp = off_ol + _a256(bh * n * 128 * 2)
+    off_vp = off_kp + _a256(bh * npl * 128 * 2)
+    wsc = ws.cpu()
+    q8 = wsc[:bh * n * 128].view(batch, heads, n, 128)
+    k8 = wsc[t8:t8 + bh * n * 128].view(batch, heads, n, 128)
+    kp8 = wsc[off_kp8:off_kp8 + bh * npl * 128].view(batch, heads, npl, 128)
+    amax_l = wsc[off_al:off_al + 8 * bh].view(torch.int32).view(torch.float32).numpy().reshape(-1, 2)
+    amax_g = wsc[off_ag:off_ag + 8 * bh].view(torch.int32).view(torch.float32).numpy().reshape(-1, 2)
+    kp = wsc[off_kp:off_kp + bh * npl * 256].view(torch.bfloat16).view(batch, heads, npl, 128)
+    vp = wsc[off_vp:off_vp + bh * npl * 256].view(torch.bfloat16).view(batch, heads, npl, 128)
+    assert np.array_equal(amax_g[:, 0], amax_l[:, 0])
+    gv = S.blend_g(w)
+    for b, h in check:
+        i = b * heads + h
+        assert amax_g[i, 1] == float(kp[b, h].float().abs().max())
+        assert torch.equal(kp8[b, h], _e4m3_bytes(kp[b, h], amax_g[i, 1])), "K_p e4m3 bytes"
+        qd = O.unpermute(_dequant(q8[b, h], amax_l[i, 0]), g)
+        kd = O.unpermute(_dequant(k8[b, h], amax_l[i, 1]), g)
+        kpd = _dequant(kp8[b, h], amax_g[i, 1])
+        vv = host_f64(w, S.V_ID, b, h)
+        o_l, _ = O.sta_attention(qd[None, None], kd[None, None], vv[None, None], g, scale)
+        o_g, _ = O.global_attention(qd[None, None], kpd[None, None], vp[b, h].double().numpy()[None, None], scale)
+        ref = gv[h] * o_l[0, 0] + (1 - gv[h]) * o_g[0, 0]
+        assert_close(to_f64(o_r[b, h]), ref, O_MAX_ABS, O_MEAN_ABS, f"O b{b} h{h}")
+        qx, kx = host_f64(w, S.Q_ID, b, h), host_f64(w, S.K_ID, b, h)
+        ex = O.dual_forward(qx[None, None], kx[None, None], vv[None, None], gv[h:h + 1], g, scale)["O"]
+        assert_close(to_f64(o_r[b, h]), ex[0, 0], FP8_O_MAX_ABS, FP8_O_MEAN_ABS, f"O vs exact b{b} h{h}")

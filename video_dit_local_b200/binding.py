@@ -33,6 +33,7 @@ VATTN_OP_STA_FWD_HOST = 6
 VATTN_OP_HIER_FWD = 7
 VATTN_OP_HIER_BWD = 8
 VATTN_OP_STA_FWD_FP8 = 9
+VATTN_OP_DUAL_FWD_FP8 = 10
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -89,6 +90,7 @@ _SIGS = {
     "vattn_hier_fwd": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_hier_bwd": [_GP, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_raster": [_GP, _P, _P, _P, _F, _P, _P, _P],
+    "vattn_dual_fwd_fp8": [_GP, _P, _P, _P, _P, _F, _P, _P, _SZ, _P],
     "vattn_sta_fwd_fp8": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_host": [_GP, _P, _P, _P, _F, _P, _P, _I64, _P, _SZ, _P],
     "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
@@ -216,6 +218,14 @@ def vattn_sta_fwd_raster(geom: Geom, q, k, v, scale: float, o, lse=None, stream=
     """Sliding-tile forward on raster-order tensors (reorder fused into the kernel)."""
     _check(lib.vattn_sta_fwd_raster(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
                                     _stream(stream)))
+
+
+def vattn_dual_fwd_fp8(geom: Geom, q, k, v, g, scale: float, o, workspace, ws_bytes: int = 0, stream=None) -> None:
+    """Dual forward with e4m3 Q*K^T in both branches (inference)."""
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_dual_fwd_fp8(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), scale, _ptr(o),
+                                  _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def vattn_sta_fwd_fp8(geom: Geom, q, k, v, scale: float, o, lse=None, workspace=None, ws_bytes: int = 0,

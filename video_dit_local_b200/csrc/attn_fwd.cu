@@ -668,8 +668,8 @@ cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t
 }
 
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
-  if (a.qk_amax) {  // e4m3 Q*K^T: sliding tile, d = 128
-    if (g.d != 128 || mode != FWD_STA || a.kgeom) return cudaErrorInvalidValue;
+  if (a.qk_amax) {  // e4m3 Q*K^T: sliding tile or global (+ blend), d = 128
+    if (g.d != 128 || a.kgeom || a.raster) return cudaErrorInvalidValue;
     return launch_fwd_d<128, true>(g, mode, a, st);
   }
   if (g.d == 128) return launch_fwd_d<128>(g, mode, a, st);

@@ -304,22 +304,20 @@ cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, cons
 // x8 = RNE_e4m3(x * (448 / absmax)) with saturation.  e4m3 is a floating
 // format: one scale per head only has to keep values in range.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) absmax_qk_kernel(const uint4* q, const uint4* k, int* amax, uint32_t vec_per_bh) {
+// absmax of one [bh][vec_per_bh] tensor per batch*head into amax[bh * stride]
+__global__ void __launch_bounds__(256) absmax_kernel(const uint4* x, int* amax, int stride, uint32_t vec_per_bh) {
   const uint32_t bh = blockIdx.y;
-  const uint4* src[2] = {q + (size_t)bh * vec_per_bh, k + (size_t)bh * vec_per_bh};
+  const uint4* src = x + (size_t)bh * vec_per_bh;
+  float m = 0.f;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < vec_per_bh; i += gridDim.x * blockDim.x) {
+    const uint4 w = __ldg(src + i);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    float m = 0.f;
-    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < vec_per_bh; i += gridDim.x * blockDim.x) {
-      const uint4 w = __ldg(src[t] + i);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(ww[e])), fabsf(bf16hi(ww[e]))));
-    }
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    // non-negative floats order like their bit patterns
-    if ((threadIdx.x & 31) == 0) atomicMax(&amax[2 * bh + t], __float_as_int(m));
+    for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(ww[e])), fabsf(bf16hi(ww[e]))));
   }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  // non-negative floats order like their bit patterns
+  if ((threadIdx.x & 31) == 0) atomicMax(&amax[(size_t)bh * stride], __float_as_int(m));
 }
 
 __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
@@ -328,41 +326,36 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   return r;
 }
 
-__global__ void __launch_bounds__(256) quant_qk_kernel(const uint4* q, const uint4* k, const int* amax, uint2* q8,
-                                                       uint2* k8, uint32_t vec_per_bh) {
+__global__ void __launch_bounds__(256) quant_kernel(const uint4* x, const int* amax, int stride, uint2* x8,
+                                                    uint32_t vec_per_bh) {
   const uint32_t bh = blockIdx.y;
+  const float a = __int_as_float(amax[(size_t)bh * stride]);
+  const float inv = a > 0.f ? 448.f / a : 1.f;
+  const uint4* src = x + (size_t)bh * vec_per_bh;
+  uint2* dst = x8 + (size_t)bh * vec_per_bh;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < vec_per_bh; i += gridDim.x * blockDim.x) {
+    const uint4 w = __ldg(src + i);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    uint32_t b[4];
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const float a = __int_as_float(amax[2 * bh + t]);
-    const float inv = a > 0.f ? 448.f / a : 1.f;
-    const uint4* src = (t == 0 ? q : k) + (size_t)bh * vec_per_bh;
-    uint2* dst = (t == 0 ? q8 : k8) + (size_t)bh * vec_per_bh;
-    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < vec_per_bh; i += gridDim.x * blockDim.x) {
-      const uint4 w = __ldg(src + i);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-      uint32_t b[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) b[e] = e4m3x2(bf16lo(ww[e]) * inv, bf16hi(ww[e]) * inv);
-      dst[i] = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
-    }
+    for (int e = 0; e < 4; ++e) b[e] = e4m3x2(bf16lo(ww[e]) * inv, bf16hi(ww[e]) * inv);
+    dst[i] = make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
   }
 }
 
-cudaError_t launch_quant_qk(const DevGeom& g, const void* q, const void* k, void* q8, void* k8, int* amax,
-                            cudaStream_t st) {
-  const long long bh = (long long)g.B * g.heads;
-  const long long vec = (long long)g.N * g.d / 8;
+cudaError_t launch_quant_e4m3(const void* x, long long rows_per_bh, long long bh, int d, void* x8, int* amax,
+                              int amax_stride, cudaStream_t st) {
+  const long long vec = rows_per_bh * d / 8;
   if (bh == 0 || vec == 0) return cudaSuccess;
   if (vec >= (1ll << 31)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(int) * 2 * bh, st);
+  cudaError_t e = cudaMemset2DAsync(amax, sizeof(int) * amax_stride, 0, sizeof(int), bh, st);
   if (e != cudaSuccess) return e;
   const int blocks = (int)std::min<long long>((vec + 255) / 256, 128);
-  absmax_qk_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>((const uint4*)q, (const uint4*)k, amax,
-                                                               (uint32_t)vec);
+  absmax_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>((const uint4*)x, amax, amax_stride, (uint32_t)vec);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  quant_qk_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>((const uint4*)q, (const uint4*)k, amax, (uint2*)q8,
-                                                              (uint2*)k8, (uint32_t)vec);
+  quant_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>((const uint4*)x, amax, amax_stride, (uint2*)x8,
+                                                           (uint32_t)vec);
   return cudaGetLastError();
 }
 

@@ -311,6 +311,26 @@ static Fp8FwdWs fp8_fwd_ws(const DevGeom& g) {
   return w;
 }
 
+// FP8 dual forward, in the order the header documents.
+struct DualFp8Ws {
+  size_t q8, k8, kp8, amax_l, amax_g, o_l, kp, vp, total;
+};
+static DualFp8Ws dual_fp8_ws(const DevGeom& g) {
+  DualFp8Ws w;
+  const size_t bh = (size_t)g.B * g.heads;
+  const size_t t8 = align256(bh * g.N * g.d), p8 = align256(bh * g.Np * g.d), am = align256(bh * 2 * 4);
+  w.q8 = 0;
+  w.k8 = t8;
+  w.kp8 = 2 * t8;
+  w.amax_l = w.kp8 + p8;
+  w.amax_g = w.amax_l + am;
+  w.o_l = w.amax_g + am;
+  w.kp = w.o_l + align256(bh * g.N * g.d * 2);
+  w.vp = w.kp + align256(bh * g.Np * g.d * 2);
+  w.total = w.vp + align256(bh * g.Np * g.d * 2);
+  return w;
+}
+
 // Hierarchical forward: medium-pooled K, V (coarse tile-major), then the
 // fine-key O and LSE that the coarse pass merges with.
 struct HierFwdWs {
@@ -466,6 +486,7 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_HIER_FWD: *bytes = hier_fwd_ws(g).total; break;
     case VATTN_OP_HIER_BWD: *bytes = hier_bwd_ws(g).total; break;
     case VATTN_OP_STA_FWD_FP8: *bytes = fp8_fwd_ws(g).total; break;
+    case VATTN_OP_DUAL_FWD_FP8: *bytes = dual_fp8_ws(g).total; break;
     default: return fail(VATTN_ERR_INVALID_ARG, "unknown op %d", op);
   }
   return ok();
@@ -786,6 +807,57 @@ int vattn_sta_fwd_raster(const vattn_geom* geom, const void* q, const void* k, c
   return ok();
 }
 
+int vattn_dual_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* gvec, float scale,
+                       void* o, void* workspace, size_t ws_bytes, void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (g.d != 128) return fail(VATTN_ERR_UNSUPPORTED, "the FP8 forward supports head_dim 128 only");
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(gvec);
+  REQUIRE_PTR(o);
+  const DualFp8Ws w = dual_fp8_ws(g);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  uint8_t* ws = (uint8_t*)workspace;
+  cudaStream_t st = (cudaStream_t)stream;
+  const long long bh = (long long)g.B * g.heads;
+  int* amax_l = (int*)(ws + w.amax_l);
+  int* amax_g = (int*)(ws + w.amax_g);
+  CHECK_LAUNCH(launch_pool_kv(g, k, v, ws + w.kp, ws + w.vp, st), "dual_fwd_fp8 pool launch");
+  CHECK_LAUNCH(launch_quant_e4m3(q, g.N, bh, g.d, ws + w.q8, amax_l, 2, st), "dual_fwd_fp8 quantise Q launch");
+  CHECK_LAUNCH(launch_quant_e4m3(k, g.N, bh, g.d, ws + w.k8, amax_l + 1, 2, st), "dual_fwd_fp8 quantise K launch");
+  CHECK_LAUNCH(launch_quant_e4m3(ws + w.kp, g.Np, bh, g.d, ws + w.kp8, amax_g + 1, 2, st),
+               "dual_fwd_fp8 quantise K_p launch");
+  // the global pass's Q scale: the same absmax as the local pass's
+  CHECK_LAUNCH(cudaMemcpy2DAsync(amax_g, 2 * sizeof(int), amax_l, 2 * sizeof(int), sizeof(int), bh,
+                                 cudaMemcpyDeviceToDevice, st),
+               "dual_fwd_fp8 scale copy");
+  FwdArgs a{};
+  a.q = ws + w.q8;
+  a.k = ws + w.k8;
+  a.v = v;
+  a.o = ws + w.o_l;
+  a.scale = scale;
+  a.qk_amax = amax_l;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "dual_fwd_fp8 local launch");
+  FwdArgs b{};
+  b.q = ws + w.q8;
+  b.k = ws + w.kp8;
+  b.v = ws + w.vp;
+  b.scale = scale;
+  b.o_local = ws + w.o_l;
+  b.g = gvec;
+  b.blend_out = o;
+  b.qk_amax = amax_g;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_GLOBAL, b, st), "dual_fwd_fp8 global launch");
+  return ok();
+}
+
 int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
                       float* lse, void* workspace, size_t ws_bytes, void* stream) {
   DevGeom g;
@@ -804,7 +876,9 @@ int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, cons
   uint8_t* ws = (uint8_t*)workspace;
   cudaStream_t st = (cudaStream_t)stream;
   int* amax = (int*)(ws + w.amax);
-  CHECK_LAUNCH(launch_quant_qk(g, q, k, ws + w.q8, ws + w.k8, amax, st), "sta_fwd_fp8 quantise launch");
+  const long long bh = (long long)g.B * g.heads;
+  CHECK_LAUNCH(launch_quant_e4m3(q, g.N, bh, g.d, ws + w.q8, amax, 2, st), "sta_fwd_fp8 quantise Q launch");
+  CHECK_LAUNCH(launch_quant_e4m3(k, g.N, bh, g.d, ws + w.k8, amax + 1, 2, st), "sta_fwd_fp8 quantise K launch");
   FwdArgs a{};
   a.q = ws + w.q8;
   a.k = ws + w.k8;

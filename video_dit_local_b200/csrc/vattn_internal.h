@@ -53,11 +53,11 @@ cudaError_t launch_pool_kv(const DevGeom& g, const void* k, const void* v, void*
 // pooled grid cut into tiles (the coarse tiles of the hierarchical branch).
 cudaError_t launch_pool_kv_tiled(const DevGeom& g, const DevGeom& gc, const void* k, const void* v, void* kp,
                                  void* vp, cudaStream_t st);
-// Q and K to e4m3 bytes with one scale per batch*head and tensor: amax[2 bh]
-// (Q) and amax[2 bh + 1] (K) receive the absmax as float bits; the dequantised
-// value is byte * amax / 448.
-cudaError_t launch_quant_qk(const DevGeom& g, const void* q, const void* k, void* q8, void* k8, int* amax,
-                            cudaStream_t st);
+// One bf16 tensor [bh][rows_per_bh][d] to e4m3 bytes with one scale per
+// batch*head: amax[bh * amax_stride] receives the absmax as float bits; the
+// dequantised value is byte * absmax / 448.
+cudaError_t launch_quant_e4m3(const void* x, long long rows_per_bh, long long bh, int d, void* x8, int* amax,
+                              int amax_stride, cudaStream_t st);
 cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, const void* v, void* qp, void* kp,
                             void* vp, cudaStream_t st);
 cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void* o_l, const float* gvec, void* out,
