@@ -144,3 +144,53 @@ def test_kernel_geometry_matches_oracle_inverse_ranges():
             for a in range(n):
                 s = min(max(a - w // 2, 0), max(n - w, 0))
                 assert range(s, s + min(w, n)) == O.window_range(a, w, n)
+
+
+def test_header_is_plain_c_and_links(V, tmp_path):
+    """include/vattn.h compiles as C99 (no C++ or torch types in the
+    signatures) and a C program links against the library."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_vattn.c"
+    src.write_text(
+        '#include "vattn.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        "  vattn_geom g = {1, 2, 64, 4, 8, 8, {2, 4, 4}, {1, 2, 2}, {1, 1, 1}};\n"
+        "  size_t bytes = 0;\n"
+        "  int r = vattn_workspace_size(VATTN_OP_DUAL_FWD, &g, &bytes);\n"
+        '  printf("%d %zu %s\\n", r, bytes, vattn_version());\n'
+        "  return r;\n"
+        "}\n")
+    exe = tmp_path / "use_vattn"
+    lib_dir = os.path.dirname(V.binding.LIB_PATH)
+    cmd = [cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+           "-L", lib_dir, "-l:libvattn.so", f"-Wl,-rpath,{lib_dir}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stderr
+    code, nbytes, version = out.stdout.split(maxsplit=2)
+    assert code == "0" and int(nbytes) > 0 and "sm_100a" in version
+
+
+def test_null_pointers_rejected_before_any_launch(V):
+    """Every entry point checks its required pointers on the host."""
+    B = V.binding
+    g = _geom(V, head_dim=128)
+    gp = _geom(V, head_dim=128, pool=(1, 2, 2))
+    cases = [
+        lambda: V.vattn_sta_fwd_raster(g, 0, 16, 16, 0.1, 16),
+        lambda: V.vattn_sta_fwd_fp8(g, 16, 0, 16, 0.1, 16, None, 32, 1 << 30),
+        lambda: V.vattn_dual_fwd_fp8(gp, 16, 16, 16, 0, 0.1, 16, 32, 1 << 30),
+        lambda: V.vattn_hier_fwd(gp, 16, 16, 0, 0.1, 16, None, 32, 1 << 30),
+        lambda: V.vattn_hier_bwd(gp, 16, 16, 16, 16, None, 16, 0.1, 16, 16, 16, 32, 1 << 30),
+        lambda: V.vattn_sta_fwd_host(g, 16, 16, 16, 0.1, 0, None, 1, 32, 1 << 30),
+    ]
+    for f in cases:
+        with pytest.raises(V.VattnError) as e:
+            f()
+        assert e.value.code == B.VATTN_ERR_INVALID_ARG, str(e.value)
