@@ -735,3 +735,21 @@ def hier_attention_tiles(q, k, v, g: Geom, hpool: tuple, scale: float, tile_ids)
         os_.append(o)
         ls_.append(l)
     return np.concatenate(ids), np.concatenate(os_), np.concatenate(ls_)
+
+
+def hier_backward_dq_tiles(q, k, v, do, g: Geom, hpool: tuple, scale: float, tile_ids):
+    """dQ of hier_backward for the listed query tiles of one head (2-D arrays):
+    a query's dQ depends only on its own row of the joint softmax.  Returns
+    (raster query ids, dQ rows)."""
+    gh = g._replace(pool=tuple(hpool))
+    kh, vh = pool(k, gh), pool(v, gh)
+    want = set(int(t) for t in tile_ids)
+    ids, rows = [], []
+    for t, (qi, kj, kc) in enumerate(_hier_query_tiles(g, hpool)):
+        if t not in want:
+            continue
+        dq, _, _ = _softmax_attend_bwd(q[qi], np.concatenate([k[kj], kh[kc]]), np.concatenate([v[kj], vh[kc]]),
+                                       do[qi], scale)
+        ids.append(qi)
+        rows.append(dq)
+    return np.concatenate(ids), np.concatenate(rows)

@@ -632,3 +632,12 @@ def test_pins_catch_coarse_tile_without_division(monkeypatch):
     g, hp = HIER_CASES[0]
     with pytest.raises(AssertionError):
         test_hier_equals_independent_masked_softmax(g, hp)
+
+
+def test_hier_sampled_dq_equals_full_backward():
+    g, hp = HIER_CASES[0]
+    q, k, v, do = (_rand((1, 1, g.n, 8), s) for s in (58, 59, 60, 61))
+    dq, _, _ = O.hier_backward(q, k, v, do, g, hp, 0.3)
+    tiles = [0, 7, 19, 63]
+    ids, rows = O.hier_backward_dq_tiles(q[0, 0], k[0, 0], v[0, 0], do[0, 0], g, hp, 0.3, tiles)
+    np.testing.assert_allclose(rows, dq[0, 0][ids], rtol=0, atol=1e-13)
