@@ -2,7 +2,9 @@
 // of kind::f16 MMAs with M = 128 (one CTA per SM, one issuing thread), as a
 // function of N, operand source (A from shared memory or TMEM), B major-ness,
 // concurrent TMEM traffic from other warps, and the barrier operations placed
-// between groups of 16 MMAs; and the CTA-pair form (cta_group::2, M = 256).
+// between groups of 16 MMAs; the CTA-pair form (cta_group::2, M = 256); and
+// whether a second CTA per SM, with its own issuing thread, covers the pauses
+// one issuing thread leaves between MMA groups.
 //
 // Build and run on one B200:
 //   nvcc -gencode arch=compute_100a,code=sm_100a -O3 -std=c++17 \
@@ -235,6 +237,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128) pair_kernel(Res
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tm), "r"(512) : "memory");
 }
 
+// Per CTA: 256 TMEM columns (S/P at 0, O at 128) and 96 KB of shared memory,
+// so two CTAs fit on one SM.  Groups of 8 TMEM x SMEM + 8 SMEM x SMEM MMAs
+// (the attention forward's per-block pattern), then `pause` idle cycles.
+__global__ void __launch_bounds__(128, 2) two_cta_kernel(Res* out, int iters, int pause, int* err) {
+  extern __shared__ uint8_t raw[];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const uint32_t base = (smem_u32(raw) + 1023u) & ~1023u;
+  uint8_t* p = raw + (base - smem_u32(raw));
+  for (int i = threadIdx.x; i < (96 * 1024) / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(p)[i] = rand_bf16x2(i + blockIdx.x * 77777u);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tbase, 256);
+    tmem_relinquish();
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tbase;
+  {
+    uint32_t r[32];
+    for (int c = 0; c < 4; ++c) {
+      for (int i = 0; i < 32; ++i) r[i] = rand_bf16x2(threadIdx.x * 128 + c * 32 + i);
+      tmem_st32(tm + ((uint32_t)(32 * warp) << 16) + 32 * c, r);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0 && lane == 0) {
+    constexpr uint32_t IQK = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t IPV = idesc_bf16_f32(128, 128, 0, 1);
+    const uint32_t q_s = base, k_s = base + 32768, v_s = base + 65536;
+    const long long t0 = clock64();
+    const uint64_t g0 = globaltimer_ns();
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(tm + 128, tm + kk * 8, smem_desc_sw128(v_s + kk * 2048, 16384, 1024), IPV, 1);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_ss(tm, smem_desc_sw128(q_s + off, 16, 1024), smem_desc_sw128(k_s + off, 16, 1024), IQK, kk > 0);
+      }
+      const long long s0 = clock64();
+      while (clock64() - s0 < pause) {
+      }
+    }
+    tc_commit(&bar);
+    const bool ok = bounded_wait(&bar, 0);
+    const long long t1 = clock64();
+    const uint64_t g1 = globaltimer_ns();
+    if (!ok) atomicExch(err, 4);
+    out[blockIdx.x].cyc = t1 - t0;
+    out[blockIdx.x].ns = (long long)(g1 - g0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, 256);
+}
+
 void report(const char* name, const std::vector<Res>& h, double instrs, double flop_per_sm_instr, int herr) {
   std::vector<double> c;
   double ghz = 0;
@@ -311,5 +382,33 @@ int main() {
   run<128, 1, 1, 0, 1>("TMEMxSMEM N=128 + per-16 sync ops", d_out, d_err);
   run_pair<128>("CTA pair M=256 N=128 (per SM)", d_out, d_err);
   run_pair<256>("CTA pair M=256 N=256 (per SM)", d_out, d_err);
+  // one or two CTAs per SM, each pausing between 16-MMA groups
+  Res* d_out2;
+  cudaMalloc(&d_out2, 296 * sizeof(Res));
+  const int smem2 = 100 * 1024;
+  cudaFuncSetAttribute(two_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2);
+  for (int pause : {0, 400, 800}) {
+    for (int per_sm = 1; per_sm <= 2; ++per_sm) {
+      const int ctas = 148 * per_sm, iters = 256;
+      for (int rep = 0; rep < 3; ++rep) {
+        two_cta_kernel<<<ctas, 128, smem2>>>(d_out2, iters, pause, d_err);
+        const cudaError_t e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) {
+          printf("two_cta: %s\n", cudaGetErrorString(e));
+          return 1;
+        }
+      }
+      std::vector<Res> h(ctas);
+      int herr = 0;
+      cudaMemcpy(&herr, d_err, 4, cudaMemcpyDeviceToHost);
+      cudaMemcpy(h.data(), d_out2, h.size() * sizeof(Res), cudaMemcpyDeviceToHost);
+      std::vector<double> c;
+      for (const Res& r : h) c.push_back((double)r.cyc / iters);
+      std::sort(c.begin(), c.end());
+      const double med = c[c.size() / 2];
+      printf("pause %3d cycles, %d CTA(s) per SM: %6.1f cycles per 16-MMA group and CTA, tensor pipe busy %5.1f%%  err %d\n",
+             pause, per_sm, med, 100.0 * per_sm * 16 * 64.2 / med, herr);
+    }
+  }
   return 0;
 }
