@@ -210,7 +210,9 @@ int vattn_dual_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, con
  *            computed on a geometry whose heads = chunk_slices and batch = 1.
  *  The work is ordered after earlier work on `stream`, and `stream` is made
  *  to wait for all of it: synchronise `stream` before reading o / lse.
- *  Calls from several host threads on one device are serialised. */
+ *  Calls from several host threads on one device are serialised.  When a
+ *  CUDA call fails after part of the pipeline was enqueued, the library
+ *  streams are synchronised before the error returns (o / lse undefined). */
 int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale,
                        void* o, float* lse, int64_t chunk_slices, void* workspace, size_t ws_bytes,
                        void* stream);

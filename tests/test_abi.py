@@ -194,3 +194,34 @@ def test_null_pointers_rejected_before_any_launch(V):
         with pytest.raises(V.VattnError) as e:
             f()
         assert e.value.code == B.VATTN_ERR_INVALID_ARG, str(e.value)
+
+
+def test_misaligned_optional_outputs_rejected(V):
+    """Optional outputs (LSE, dg) follow the same 16-byte rule as every other
+    pointer, on every entry point that takes one."""
+    B = V.binding
+    g = _geom(V, head_dim=128)
+    cases = [
+        lambda: V.vattn_sta_fwd(g, 16, 16, 16, 0.1, 16, lse=20),
+        lambda: V.vattn_xwin_fwd(g, 0, 16, 16, 16, 0.1, 16, lse=20),
+        lambda: V.vattn_global_fwd(g, 16, 16, 16, 0.1, 16, lse=20),
+        lambda: V.vattn_sta_fwd_raster(g, 16, 16, 16, 0.1, 16, lse=20),
+        lambda: V.vattn_sta_fwd_fp8(g, 16, 16, 16, 0.1, 16, 20, 32, 1 << 30),
+        lambda: V.vattn_hier_fwd(g, 16, 16, 16, 0.1, 16, 20, 32, 1 << 30),
+        lambda: V.vattn_dual_fwd(g, 16, 16, 16, 16, 0.1, 16, o_l=16, lse_l=20, o_g=16, lse_g=16, kp=16, vp=16),
+        lambda: V.vattn_dual_bwd(g, 16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 16, 0.1, 16, 16, 16, 20, 32, 1 << 30),
+    ]
+    for f in cases:
+        with pytest.raises(V.VattnError) as e:
+            f()
+        assert e.value.code == B.VATTN_ERR_ALIGN and "aligned" in str(e.value), str(e.value)
+
+
+def test_batch_heads_limit_without_overflow(V):
+    """batch*heads >= 2^16 is unsupported, including values whose product
+    would overflow 64 bits."""
+    B = V.binding
+    for batch, heads in [(1, 65536), (256, 256), (1 << 40, 1 << 40)]:
+        with pytest.raises(V.VattnError) as e:
+            V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, _geom(V, batch=batch, heads=heads))
+        assert e.value.code == B.VATTN_ERR_UNSUPPORTED

@@ -175,7 +175,8 @@ static int build_geom(const vattn_geom* in, int need, DevGeom* g) {
   if ((need & NEED_ATTN) && in->head_dim != 64 && in->head_dim != 128)
     return fail(VATTN_ERR_UNSUPPORTED, "head_dim %lld not supported (64 or 128)", (long long)in->head_dim);
   if (in->head_dim <= 0 || in->head_dim > 4096) return fail(VATTN_ERR_INVALID_ARG, "head_dim out of range");
-  if (in->batch * in->heads >= 65536) return fail(VATTN_ERR_UNSUPPORTED, "batch*heads must be < 65536");
+  if (in->batch >= 65536 || in->heads >= 65536 || in->batch * in->heads >= 65536)
+    return fail(VATTN_ERR_UNSUPPORTED, "batch*heads must be < 65536");
   g->B = (int)in->batch;
   g->heads = (int)in->heads;
   g->d = (int)in->head_dim;
@@ -573,30 +574,13 @@ int vattn_xwin_fwd(const vattn_geom* geom, int shifted, const void* q, const voi
   return ok();
 }
 
-int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
-                       float* lse, int64_t chunk_slices, void* workspace, size_t ws_bytes, void* stream) {
-  DevGeom g;
-  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
-  if (r) return r;
-  if (empty_geom(g)) return ok();
-  if (!q || !k || !v || !o) return fail(VATTN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL host pointers");
+}  // extern "C"
+
+// Enqueues the chunk pipeline of vattn_sta_fwd_host on the library streams.
+static int sta_fwd_host_enqueue(HostPipe& p, const DevGeom& g, const DevGeom& gc, const HostChunkWs& w, const void* q,
+                                const void* k, const void* v, float scale, void* o, float* lse, long long chunk_slices,
+                                void* workspace, cudaStream_t caller) {
   const long long total = (long long)g.B * g.heads;
-  if (chunk_slices <= 0 || chunk_slices > total) return fail(VATTN_ERR_INVALID_ARG, "chunk_slices out of range");
-  DevGeom gc = g;  // one chunk: batch 1, heads = chunk_slices (the attention path has no per-head state here)
-  gc.B = 1;
-  gc.heads = (int)chunk_slices;
-  const HostChunkWs w = host_chunk_ws(gc);
-  if (!workspace || ws_bytes < 2 * w.total)
-    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", 2 * w.total, workspace ? ws_bytes : 0);
-  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
-  int dev = 0;
-  CHECK_LAUNCH(cudaGetDevice(&dev), "cudaGetDevice");
-  HostPipe* pp = host_pipe(dev);
-  if (!pp) return fail(VATTN_ERR_UNSUPPORTED, "device index out of range");
-  std::lock_guard<std::mutex> lk(pp->mu);
-  CHECK_LAUNCH(host_pipe_init(*pp), "pipeline stream/event creation");
-  HostPipe& p = *pp;
-  cudaStream_t caller = (cudaStream_t)stream;
   CHECK_LAUNCH(cudaEventRecord(p.start, caller), "event record");
   // the library streams also wait for the previous call's end (its caller may
   // have used another stream): its staging slots are reused below.  Waiting
@@ -671,6 +655,44 @@ int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, con
   return ok();
 }
 
+extern "C" int vattn_sta_fwd_host(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale,
+                                  void* o, float* lse, int64_t chunk_slices, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  if (!q || !k || !v || !o) return fail(VATTN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL host pointers");
+  const long long total = (long long)g.B * g.heads;
+  if (chunk_slices <= 0 || chunk_slices > total) return fail(VATTN_ERR_INVALID_ARG, "chunk_slices out of range");
+  DevGeom gc = g;  // one chunk: batch 1, heads = chunk_slices (the attention path has no per-head state here)
+  gc.B = 1;
+  gc.heads = (int)chunk_slices;
+  const HostChunkWs w = host_chunk_ws(gc);
+  if (!workspace || ws_bytes < 2 * w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", 2 * w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  int dev = 0;
+  CHECK_LAUNCH(cudaGetDevice(&dev), "cudaGetDevice");
+  HostPipe* pp = host_pipe(dev);
+  if (!pp) return fail(VATTN_ERR_UNSUPPORTED, "device index out of range");
+  std::lock_guard<std::mutex> lk(pp->mu);
+  CHECK_LAUNCH(host_pipe_init(*pp), "pipeline stream/event creation");
+  r = sta_fwd_host_enqueue(*pp, g, gc, w, q, k, v, scale, o, lse, chunk_slices, workspace, (cudaStream_t)stream);
+  if (r != VATTN_OK) {
+    // part of the pipeline may be in flight, and `last` does not cover it:
+    // let it finish, so that no later call reuses a staging slot under it
+    const std::string msg = t_last_error;
+    cudaStreamSynchronize(pp->in);
+    cudaStreamSynchronize(pp->comp);
+    cudaStreamSynchronize(pp->out);
+    record_error(r, msg.c_str());
+  }
+  return r;
+}
+
+extern "C" {
+
 // Fine geometry (pool = h_pool) and the coarse grid: the medium-pooled grid
 // cut into tiles of the same shape.
 static int build_hier(const vattn_geom* geom, DevGeom* g, DevGeom* gc) {
@@ -697,6 +719,7 @@ int vattn_hier_fwd(const vattn_geom* geom, const void* q, const void* k, const v
   REQUIRE_PTR(k);
   REQUIRE_PTR(v);
   REQUIRE_PTR(o);
+  if (lse && !aligned16(lse)) return fail(VATTN_ERR_ALIGN, "lse is not 16-byte aligned");
   const HierFwdWs w = hier_fwd_ws(g);
   if (!workspace || ws_bytes < w.total)
     return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
@@ -795,6 +818,7 @@ int vattn_sta_fwd_raster(const vattn_geom* geom, const void* q, const void* k, c
   REQUIRE_PTR(k);
   REQUIRE_PTR(v);
   REQUIRE_PTR(o);
+  if (lse && !aligned16(lse)) return fail(VATTN_ERR_ALIGN, "lse is not 16-byte aligned");
   FwdArgs a{};
   a.q = q;
   a.k = k;
@@ -869,6 +893,7 @@ int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, cons
   REQUIRE_PTR(k);
   REQUIRE_PTR(v);
   REQUIRE_PTR(o);
+  if (lse && !aligned16(lse)) return fail(VATTN_ERR_ALIGN, "lse is not 16-byte aligned");
   const Fp8FwdWs w = fp8_fwd_ws(g);
   if (!workspace || ws_bytes < w.total)
     return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
