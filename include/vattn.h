@@ -320,6 +320,18 @@ int vattn_get_status(void* stream);
 /* Message for the last non-OK return on this thread ("" if none). */
 const char* vattn_last_error(void);
 
+/* Releases what the library keeps between calls: the three streams and eight
+ * events of vattn_sta_fwd_host's pipeline, on every device where a call
+ * created them, after waiting for the work queued on them.  A later
+ * vattn_sta_fwd_host creates them again.  Nothing else is held: tensor-map
+ * descriptors are built per call and passed to the kernels by value, and the
+ * scratch of vattn_dual_fwd_noalloc is a static device array that lives as
+ * long as the loaded library.  Safe from any thread at any time (it waits for
+ * a vattn_sta_fwd_host call in progress); the current device is left as it
+ * was.  Returns VATTN_OK, or VATTN_ERR_CUDA if a synchronisation or a destroy
+ * failed (the handles are released all the same). */
+int vattn_shutdown(void);
+
 /* Test hook.  flags bit 0: the attention kernels' load warp skips its first
  * arrival, so the consumer's bounded wait runs out (no fault, no hang);
  * timeout_ns: the device wait limit (<= 0 restores the default, 2 s).
@@ -327,8 +339,9 @@ const char* vattn_last_error(void);
 int vattn_debug_set(int flags, int64_t timeout_ns);
 
 /* Test hook: y[i] = the library's polynomial 2^x[i] (the one the attention
- * forward uses for a quarter of its exponentials), for checking against
- * CUDA's exp2f.  x, y: device float32 [n]. */
+ * forward can run on the FMA pipe for one chunk of its exponentials; off in
+ * the default build), for checking against CUDA's exp2f.  x, y: device
+ * float32 [n]. */
 int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /* Library version string. */

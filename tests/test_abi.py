@@ -225,3 +225,11 @@ def test_batch_heads_limit_without_overflow(V):
         with pytest.raises(V.VattnError) as e:
             V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, _geom(V, batch=batch, heads=heads))
         assert e.value.code == B.VATTN_ERR_UNSUPPORTED
+
+
+def test_shutdown_without_pipeline_is_ok(V):
+    """vattn_shutdown with nothing created touches no device and succeeds,
+    and may be called repeatedly."""
+    V.vattn_shutdown()
+    V.vattn_shutdown()
+    assert V.vattn_last_error() == ""

@@ -152,3 +152,26 @@ def test_sta_fwd_host_back_to_back_calls_from_two_streams(V):
     torch.cuda.synchronize()
     assert V.vattn_get_status() == 0, V.vattn_last_error()
     assert torch_equal_bits(o1, ref1) and torch_equal_bits(o2, ref2)
+
+
+def test_shutdown_waits_for_the_pipeline_and_calls_recreate_it(V):
+    """vattn_shutdown issued right after an asynchronous host-buffer call
+    waits for that call's copies and kernels, releases the library streams,
+    and the next call builds them again with the same result."""
+    import torch
+    w = S.small_workload("host_shutdown", 35, 1, 4, 128, (6, 16, 16), (3, 8, 8), (1, 1, 3), (1, 1, 1))
+    check = [(0, h) for h in range(4)]
+    geom = geom_for(V, w)
+    scale = 1 / math.sqrt(128)
+    qr, kr, vr = (gpu_tensor(w, i, check) for i in (S.Q_ID, S.K_ID, S.V_ID))
+    ref, _ = _device_path(V, geom, qr, kr, vr, scale)
+    ins = [x.cpu().pin_memory() for x in (qr, kr, vr)]
+    one = V.make_geom(1, 1, 128, w.grid, w.tile, w.window, w.pool)
+    ws = torch.empty(2 * V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, one), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        o = torch.full(qr.shape, float("nan"), dtype=torch.bfloat16).pin_memory()
+        V.vattn_sta_fwd_host(geom, *ins, scale, o, None, 1, ws)
+        V.vattn_shutdown()          # no synchronisation before it: shutdown waits
+        torch.cuda.current_stream().synchronize()
+        assert V.vattn_get_status() == 0, V.vattn_last_error()
+        assert torch_equal_bits(o, ref)

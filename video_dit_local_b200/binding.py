@@ -99,6 +99,7 @@ _SIGS = {
     "vattn_workspace_size": [_INT, _GP, ctypes.POINTER(_SZ)],
     "vattn_get_status": [_P],
     "vattn_last_error": [],
+    "vattn_shutdown": [],
     "vattn_debug_set": [_INT, _I64],
     "vattn_debug_exp2": [_P, _P, _I64, _P],
     "vattn_version": [],
@@ -302,6 +303,11 @@ def vattn_get_status(stream=None) -> int:
 
 def vattn_last_error() -> str:
     return lib.vattn_last_error().decode()
+
+
+def vattn_shutdown() -> None:
+    """Releases the host pipeline's library streams and events on every device."""
+    _check(lib.vattn_shutdown())
 
 
 def vattn_debug_set(flags: int, timeout_ns: int = 0) -> None:

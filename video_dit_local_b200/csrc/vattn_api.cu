@@ -405,18 +405,43 @@ static HostPipe* host_pipe(int dev) {
   if (dev < 0 || dev >= 64) return nullptr;
   return &pipes[dev];
 }
+// Destroys whatever streams and events `p` holds (the caller has waited for
+// their work) and returns the first error met.
+static cudaError_t host_pipe_release(HostPipe& p) {
+  cudaError_t first = cudaSuccess;
+  auto keep = [&first](cudaError_t e) {
+    if (first == cudaSuccess) first = e;
+  };
+  for (cudaStream_t* s : {&p.in, &p.comp, &p.out}) {
+    if (*s) keep(cudaStreamDestroy(*s));
+    *s = nullptr;
+  }
+  cudaEvent_t* evs[] = {&p.start, &p.last, &p.in_done[0], &p.in_done[1], &p.comp_done[0], &p.comp_done[1],
+                        &p.out_done[0], &p.out_done[1]};
+  for (cudaEvent_t* ev : evs) {
+    if (*ev) keep(cudaEventDestroy(*ev));
+    *ev = nullptr;
+  }
+  p.ready = false;
+  return first;
+}
+
 static cudaError_t host_pipe_init(HostPipe& p) {
   if (p.ready) return cudaSuccess;
-  cudaError_t e;
-  if ((e = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking)) != cudaSuccess) return e;
-  if ((e = cudaStreamCreateWithFlags(&p.comp, cudaStreamNonBlocking)) != cudaSuccess) return e;
-  if ((e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
-  if ((e = cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming)) != cudaSuccess) return e;
-  if ((e = cudaEventCreateWithFlags(&p.last, cudaEventDisableTiming)) != cudaSuccess) return e;
-  for (int i = 0; i < 2; ++i) {
-    if ((e = cudaEventCreateWithFlags(&p.in_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&p.comp_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&p.out_done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  auto ok_so_far = [&e](cudaError_t r) { return (e = r) == cudaSuccess; };
+  bool made = ok_so_far(cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking)) &&
+              ok_so_far(cudaStreamCreateWithFlags(&p.comp, cudaStreamNonBlocking)) &&
+              ok_so_far(cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking)) &&
+              ok_so_far(cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming)) &&
+              ok_so_far(cudaEventCreateWithFlags(&p.last, cudaEventDisableTiming));
+  for (int i = 0; made && i < 2; ++i)
+    made = ok_so_far(cudaEventCreateWithFlags(&p.in_done[i], cudaEventDisableTiming)) &&
+           ok_so_far(cudaEventCreateWithFlags(&p.comp_done[i], cudaEventDisableTiming)) &&
+           ok_so_far(cudaEventCreateWithFlags(&p.out_done[i], cudaEventDisableTiming));
+  if (!made) {  // nothing was used yet: drop what was created
+    host_pipe_release(p);
+    return e;
   }
   p.ready = true;
   return cudaSuccess;
@@ -468,6 +493,36 @@ int vattn_get_status(void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
     return fail(word, "device reported status %d (a bounded wait ran out)", word);
   }
+  return ok();
+}
+
+int vattn_shutdown(void) {
+  int prev = -1;
+  int code = VATTN_OK;
+  std::string msg;
+  for (int dev = 0; dev < 64; ++dev) {
+    HostPipe& p = *host_pipe(dev);
+    std::lock_guard<std::mutex> lk(p.mu);
+    if (!p.ready) continue;
+    if (prev < 0 && cudaGetDevice(&prev) != cudaSuccess) prev = 0;
+    cudaError_t e = cudaSetDevice(dev);
+    if (e == cudaSuccess) {
+      // wait for the pipeline's copies and kernels before the handles go
+      for (cudaStream_t s : {p.in, p.comp, p.out}) {
+        const cudaError_t r = cudaStreamSynchronize(s);
+        if (e == cudaSuccess) e = r;
+      }
+      const cudaError_t r = host_pipe_release(p);
+      if (e == cudaSuccess) e = r;
+    }
+    if (e != cudaSuccess && code == VATTN_OK) {
+      code = VATTN_ERR_CUDA;
+      msg = std::string("shutdown of the host pipeline on device ") + std::to_string(dev) + ": " +
+            cudaGetErrorString(e);
+    }
+  }
+  if (prev >= 0) cudaSetDevice(prev);
+  if (code != VATTN_OK) return record_error(code, msg.c_str());
   return ok();
 }
 
