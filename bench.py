@@ -2,8 +2,10 @@
 
 Default workload: the 720p-shaped sliding-tile forward (B1 h24 d128, grid
 30x48x80, tile 6x8x8, window 3x3x3, per-head U(0.5, 2) scale).  One step =
-raster->tile-major permute of Q, K, V, the sliding-tile forward (O, LSE), and
-the tile-major->raster unpermute of O and LSE, all through the C ABI.
+one vattn_sta_fwd_raster call: raster Q, K, V in, raster O and LSE out, the
+raster <-> tile-major reorder done by the kernel's tensor-map boxes and
+epilogue stores (one launch).  `e2e` times vattn_sta_fwd_host on the same
+workload from pinned host buffers, copies included.
 Effective FLOPs count 4*d per kept query-key pair (masked work is not
 counted).  Inputs (2.1 GB of Q/K/V) are larger than the 126 MB L2, so no flush
 is needed between steps.
