@@ -2,7 +2,9 @@
 hypothesis, each oracle function against an independent token-level masked
 softmax built in the test (library SDPA in float64), and the kept-tile count
 against its closed form.  The masks come from token coordinates only; the
-oracle's tile-iteration code is not used to build them."""
+oracle's tile-iteration code is not used to build them.  Every backward
+oracle is also held to four identities of normalised softmax attention
+(below), on random geometries, pools and blend factors."""
 import math
 
 import numpy as np
@@ -119,3 +121,128 @@ def test_hier_matches_coordinate_mask(gh, seed):
     o, _ = O.hier_attention(q, k, v, g, hp, 0.5)
     np.testing.assert_allclose(o, _sdpa(q, keys, vals, 0.5, np.concatenate([fine, coarse], axis=1)), rtol=0,
                                atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Backward identities that hold for any softmax attention whose rows are
+# normalised over their key set, whatever the mask, pooling or blend:
+#   sum_tokens dK = 0          (every row of dS sums to zero; pool^T keeps sums)
+#   sum_tokens dV = sum dO     (rows of P sum to one; g + (1 - g) = 1; the
+#                               upsampling weights of an output row sum to one)
+#   <Q, dQ> = <K, dK>          (both equal scale * sum_ij dS_ij (q_i . k_j);
+#                               pooling is linear, so it holds through it)
+#   <V, dV> = <O, dO>          (both equal sum_ij P_ij (v_j . dO_i), per branch
+#                               weight, with O the blended output)
+# all per (batch, head).  They come from the mathematics, not from the
+# oracle's code, and a dropped pool^T term, a missing branch weight, a
+# transposed operand or a wrong sign in the softmax Jacobian breaks one.
+# ---------------------------------------------------------------------------
+
+def _identity_residuals(q, k, v, do, o, dq, dk, dv):
+    sk = np.abs(dk.sum(axis=2)).max()
+    sv = np.abs(dv.sum(axis=2) - do.sum(axis=2)).max()
+    qk = np.abs((q * dq).sum(axis=(2, 3)) - (k * dk).sum(axis=(2, 3))).max()
+    vo = np.abs((v * dv).sum(axis=(2, 3)) - (o * do).sum(axis=(2, 3))).max()
+    return sk, sv, qk, vo
+
+
+def _assert_identities(*a, atol=1e-9):
+    sk, sv, qk, vo = _identity_residuals(*a)
+    assert sk < atol, f"sum dK = {sk}"
+    assert sv < atol, f"sum dV - sum dO = {sv}"
+    assert qk < atol, f"<Q,dQ> - <K,dK> = {qk}"
+    assert vo < atol, f"<V,dV> - <O,dO> = {vo}"
+
+
+def _divisors(n):
+    return [p for p in range(1, n + 1) if n % p == 0]
+
+
+@st.composite
+def pooled_geoms(draw):
+    g = draw(geoms(max_tokens=192))
+    pool = tuple(draw(st.sampled_from(_divisors(n))) for n in (g.T, g.H, g.W))
+    return g._replace(pool=pool)
+
+
+def _qkvdo(n, seed, heads=2, d=4):
+    q, k, v = (_rand((1, heads, n, d), seed + i) for i in range(3))
+    return q, k, v, 0.3 * _rand((1, heads, n, d), seed + 3)
+
+
+@SETTINGS
+@given(g=geoms(max_tokens=192), seed=st.integers(0, 10_000))
+def test_sta_backward_identities(g, seed):
+    q, k, v, do = _qkvdo(g.n, seed)
+    o, _ = O.sta_attention(q, k, v, g, 0.5)
+    _assert_identities(q, k, v, do, o, *O.sta_backward(q, k, v, do, g, 0.5))
+
+
+@SETTINGS
+@given(g=geoms(max_tokens=192), shifted=st.booleans(), seed=st.integers(0, 10_000))
+def test_xwin_backward_identities(g, shifted, seed):
+    q, k, v, do = _qkvdo(g.n, seed)
+    o, _ = O.xwin_attention(q, k, v, g, 0.5, shifted)
+    _assert_identities(q, k, v, do, o, *O.xwin_backward(q, k, v, do, g, 0.5, shifted))
+
+
+@SETTINGS
+@given(g=pooled_geoms(), seed=st.integers(0, 10_000))
+def test_dual_backward_identities(g, seed):
+    q, k, v, do = _qkvdo(g.n, seed)
+    gvec = np.random.default_rng(seed).uniform(0, 1, 2)
+    o = O.dual_forward(q, k, v, gvec, g, 0.5)["O"]
+    r = O.dual_backward(q, k, v, gvec, do, g, 0.5)
+    _assert_identities(q, k, v, do, o, r["dQ"], r["dK"], r["dV"])
+
+
+@SETTINGS
+@given(g=pooled_geoms(), seed=st.integers(0, 10_000))
+def test_dual_sym_backward_identities(g, seed):
+    q, k, v, do = _qkvdo(g.n, seed)
+    gvec = np.random.default_rng(seed).uniform(0, 1, 2)
+    o = O.dual_sym_forward(q, k, v, gvec, g, 0.5)["O"]
+    r = O.dual_sym_backward(q, k, v, gvec, do, g, 0.5)
+    _assert_identities(q, k, v, do, o, r["dQ"], r["dK"], r["dV"])
+
+
+@SETTINGS
+@given(gh=hier_geoms(), seed=st.integers(0, 10_000))
+def test_hier_backward_identities(gh, seed):
+    g, hp = gh
+    q, k, v, do = _qkvdo(g.n, seed)
+    o, _ = O.hier_attention(q, k, v, g, hp, 0.5)
+    _assert_identities(q, k, v, do, o, *O.hier_backward(q, k, v, do, g, hp, 0.5))
+
+
+def test_identities_catch_planted_mistakes(monkeypatch):
+    """Mistakes planted in the oracle (on the CPU) break an identity."""
+    g = O.Geom(2, 4, 4, (1, 2, 2), (1, 1, 1), (1, 2, 2))
+    q, k, v, do = _qkvdo(g.n, 7)
+    gvec = np.array([0.3, 0.8])
+    o = O.dual_forward(q, k, v, gvec, g, 0.5)["O"]
+
+    def residuals():
+        r = O.dual_backward(q, k, v, gvec, do, g, 0.5)
+        return _identity_residuals(q, k, v, do, o, r["dQ"], r["dK"], r["dV"])
+
+    assert max(residuals()) < 1e-9
+    with monkeypatch.context() as m:   # the pooled branch's gradients not sent back through the pooling
+        m.setattr(O, "pool_transpose", lambda y, g: np.zeros(y.shape[:2] + (g.n, y.shape[3])))
+        assert max(residuals()) > 1e-3
+    true_bwd = O._softmax_attend_bwd
+
+    def no_rowsum(q_, k_, v_, do_, scale):   # dS = P * dP: the Jacobian's rank-one term dropped
+        _, _, p = O._softmax_attend(q_, k_, v_, scale)
+        ds = p * (do_ @ v_.T)
+        return scale * (ds @ k_), scale * (ds.T @ q_), p.T @ do_
+    with monkeypatch.context() as m:
+        m.setattr(O, "_softmax_attend_bwd", no_rowsum)
+        assert residuals()[0] > 1e-3
+
+    def dk_without_scale(q_, k_, v_, do_, scale):   # scale applied to dQ but not to dK
+        a, b, c = true_bwd(q_, k_, v_, do_, scale)
+        return a, b / scale, c
+    with monkeypatch.context() as m:
+        m.setattr(O, "_softmax_attend_bwd", dk_without_scale)
+        assert residuals()[2] > 1e-3
