@@ -1,6 +1,7 @@
 """Property-based pins of the oracle (CPU): random small geometries drawn by
 hypothesis, each oracle function against an independent token-level masked
-softmax built in the test (library SDPA in float64), and the kept-tile count
+softmax built in the test (library SDPA in float64 for O, torch logsumexp of
+the masked scores for LSE), and the kept-tile count
 against its closed form.  The masks come from token coordinates only; the
 oracle's tile-iteration code is not used to build them.  Every backward
 oracle is also held to four identities of normalised softmax attention
@@ -26,6 +27,13 @@ def _sdpa(q, k, v, scale, mask):
     tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(a)) for a in (q, k, v))
     return torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=torch.from_numpy(mask),
                                                             scale=scale).numpy()
+
+
+def _masked_lse(q, k, scale, mask):
+    """ln sum_j exp(scale q_i . k_j) over the mask's keys (torch logsumexp, float64)."""
+    s = torch.from_numpy(np.ascontiguousarray(q)) @ torch.from_numpy(np.ascontiguousarray(k)).transpose(-1, -2)
+    s = (scale * s).masked_fill(~torch.from_numpy(mask), float("-inf"))
+    return torch.logsumexp(s, dim=-1).numpy()
 
 
 def _window_set(a, w, n):
@@ -61,8 +69,9 @@ def test_sta_matches_coordinate_mask(g, seed):
     tile_of = [tuple(c[ax] // g.tile[ax] for ax in range(3)) for c in cs]
     mask = np.array([[all(tj[ax] in wins[ax][ti[ax]] for ax in range(3)) for tj in tile_of] for ti in tile_of])
     q, k, v = (_rand((1, 1, g.n, 4), seed + i) for i in range(3))
-    o, _ = O.sta_attention(q, k, v, g, 0.5)
+    o, lse = O.sta_attention(q, k, v, g, 0.5)
     np.testing.assert_allclose(o, _sdpa(q, k, v, 0.5, mask), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _masked_lse(q, k, 0.5, mask), rtol=0, atol=1e-12)
     # kept tiles per query tile: the closed form
     assert all(len(O.kept_tiles(g)[t]) == O.kept_count_closed_form(g) for t in range(math.prod(dims)))
 
@@ -80,8 +89,9 @@ def test_xwin_matches_coordinate_blocks(g, shifted, seed):
     lab = [tuple(block(t[ax], g.window[ax], g.tiles_per_dim[ax]) for ax in range(3)) for t in tile_of]
     mask = np.array([[li == lj for lj in lab] for li in lab])
     q, k, v = (_rand((1, 1, g.n, 4), seed + i) for i in range(3))
-    o, _ = O.xwin_attention(q, k, v, g, 0.5, shifted)
+    o, lse = O.xwin_attention(q, k, v, g, 0.5, shifted)
     np.testing.assert_allclose(o, _sdpa(q, k, v, 0.5, mask), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _masked_lse(q, k, 0.5, mask), rtol=0, atol=1e-12)
 
 
 @st.composite
@@ -118,9 +128,10 @@ def test_hier_matches_coordinate_mask(gh, seed):
 
     keys = np.concatenate([k, pool(k)], axis=2)
     vals = np.concatenate([v, pool(v)], axis=2)
-    o, _ = O.hier_attention(q, k, v, g, hp, 0.5)
-    np.testing.assert_allclose(o, _sdpa(q, keys, vals, 0.5, np.concatenate([fine, coarse], axis=1)), rtol=0,
-                               atol=1e-12)
+    o, lse = O.hier_attention(q, k, v, g, hp, 0.5)
+    joint = np.concatenate([fine, coarse], axis=1)
+    np.testing.assert_allclose(o, _sdpa(q, keys, vals, 0.5, joint), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, _masked_lse(q, keys, 0.5, joint), rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------------------
