@@ -257,3 +257,58 @@ def test_identities_catch_planted_mistakes(monkeypatch):
     with monkeypatch.context() as m:
         m.setattr(O, "_softmax_attend_bwd", dk_without_scale)
         assert residuals()[2] > 1e-3
+
+
+def _avg_pool(x, g):
+    """Raster [B, h, n, d] -> pooled raster [B, h, n_p, d] by torch avg_pool3d."""
+    B, h, _, d = x.shape
+    t = torch.from_numpy(np.ascontiguousarray(x)).reshape(B * h, g.T, g.H, g.W, d).permute(0, 4, 1, 2, 3)
+    p = torch.nn.functional.avg_pool3d(t, kernel_size=g.pool, stride=g.pool)
+    return p.permute(0, 2, 3, 4, 1).reshape(B, h, -1, d).numpy()
+
+
+def _trilinear(x, g):
+    """Pooled raster -> full grid by torch trilinear interpolation (half-pixel centres)."""
+    B, h, _, d = x.shape
+    PT, PH, PW = g.pooled_dims
+    t = torch.from_numpy(np.ascontiguousarray(x)).reshape(B * h, PT, PH, PW, d).permute(0, 4, 1, 2, 3)
+    u = torch.nn.functional.interpolate(t, size=(g.T, g.H, g.W), mode="trilinear", align_corners=False)
+    return u.permute(0, 2, 3, 4, 1).reshape(B, h, -1, d).numpy()
+
+
+def _sta_mask(g):
+    cs = _coords(g.T, g.H, g.W)
+    dims = g.tiles_per_dim
+    wins = [[_window_set(a, g.window[ax], dims[ax]) for a in range(dims[ax])] for ax in range(3)]
+    tile_of = [tuple(c[ax] // g.tile[ax] for ax in range(3)) for c in cs]
+    return np.array([[all(tj[ax] in wins[ax][ti[ax]] for ax in range(3)) for tj in tile_of] for ti in tile_of])
+
+
+@SETTINGS
+@given(g=pooled_geoms(), seed=st.integers(0, 10_000))
+def test_dual_forward_matches_library_pooling(g, seed):
+    q, k, v, _ = _qkvdo(g.n, seed)
+    gvec = np.random.default_rng(seed).uniform(0, 1, 2)
+    r = O.dual_forward(q, k, v, gvec, g, 0.5)
+    kp, vp = _avg_pool(k, g), _avg_pool(v, g)
+    np.testing.assert_allclose(r["K_p"], kp, rtol=0, atol=1e-13)
+    o_l = _sdpa(q, k, v, 0.5, _sta_mask(g))
+    o_g = _sdpa(q, kp, vp, 0.5, np.ones((g.n, g.n_pooled), dtype=bool))
+    gb = gvec[None, :, None, None]
+    np.testing.assert_allclose(r["O"], gb * o_l + (1 - gb) * o_g, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["LSE_g"], _masked_lse(q, kp, 0.5, np.ones((g.n, g.n_pooled), dtype=bool)),
+                               rtol=0, atol=1e-12)
+
+
+@SETTINGS
+@given(g=pooled_geoms(), seed=st.integers(0, 10_000))
+def test_dual_sym_forward_matches_library_pool_and_trilinear(g, seed):
+    q, k, v, _ = _qkvdo(g.n, seed)
+    gvec = np.random.default_rng(seed).uniform(0, 1, 2)
+    r = O.dual_sym_forward(q, k, v, gvec, g, 0.5)
+    qp, kp, vp = (_avg_pool(x, g) for x in (q, k, v))
+    o_p = _sdpa(qp, kp, vp, 0.5, np.ones((g.n_pooled, g.n_pooled), dtype=bool))
+    np.testing.assert_allclose(r["O_p"], o_p, rtol=0, atol=1e-12)
+    o_l = _sdpa(q, k, v, 0.5, _sta_mask(g))
+    gb = gvec[None, :, None, None]
+    np.testing.assert_allclose(r["O"], gb * o_l + (1 - gb) * _trilinear(o_p, g), rtol=0, atol=1e-12)
