@@ -96,7 +96,7 @@ def torch_equal_bits(a, b):
 
 def test_sta_fwd_host_without_lse_and_pageable_output(V):
     """LSE may be omitted, and pageable (unpinned) host buffers still give the
-    same result (the copies then stage through the driver)."""
+    same result (CUDA then stages the copies through its own pinned buffers)."""
     import torch
     w = S.small_workload("host_nolse", 33, 1, 4, 128, (6, 16, 16), (3, 8, 8), (1, 1, 3), (1, 1, 1))
     check = [(0, h) for h in range(4)]
