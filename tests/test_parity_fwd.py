@@ -292,9 +292,10 @@ def test_device_timeout_is_reported_and_context_survives(V):
 
 
 def test_polynomial_exp2_against_cuda_exp2f(V):
-    """The FMA-pipe 2^x used for a quarter of the forward's exponentials
-    against CUDA's exp2f (torch.exp2): relative error <= 1e-4 on the range the
-    forward feeds it (x <= 8); at or below the clamp the result is tiny."""
+    """The FMA-pipe 2^x that the forward can run for one chunk of its
+    exponentials (a compile-time option, off in the default build) against
+    CUDA's exp2f (torch.exp2): relative error <= 1e-4 on the range the forward
+    feeds it (x <= 8); at or below the clamp the result is tiny."""
     import torch
     x = torch.cat([torch.linspace(-124.0, 8.0, 1 << 20, device="cuda"),
                    torch.rand(1 << 20, device="cuda") * 16 - 8]).contiguous()

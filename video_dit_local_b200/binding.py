@@ -1,8 +1,10 @@
 """Thin ctypes binding over libvattn.so: argument marshalling only.
 
 Every function mirrors the C entry point of the same name in include/vattn.h.
-Tensor arguments may be torch tensors (their data_ptr() is passed) or raw
-integer device addresses; `stream` defaults to torch's current CUDA stream.
+Tensor arguments may be contiguous torch tensors (their data_ptr() is
+passed; CUDA tensors for device pointers, host tensors for the host-buffer
+entry point's q, k, v, o, lse) or raw integer addresses; `stream` defaults to
+torch's current CUDA stream.
 Every non-OK status raises VattnError.  There is no fallback: if the shared
 library is missing the import of this module fails.
 """
@@ -121,10 +123,25 @@ lib = _load()
 
 
 def _ptr(x) -> Optional[int]:
-    if x is None:
-        return None
-    if isinstance(x, int):
+    """Device pointer argument: None, a raw address, or a contiguous CUDA tensor."""
+    if x is None or isinstance(x, int):
         return x
+    if not x.is_cuda:
+        raise ValueError("a device pointer argument got a host tensor: pass a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous (the library reads them as dense arrays)")
+    return x.data_ptr()
+
+
+def _hptr(x) -> Optional[int]:
+    """Host pointer argument (vattn_sta_fwd_host's q, k, v, o, lse): None, a raw
+    address, or a contiguous host tensor."""
+    if x is None or isinstance(x, int):
+        return x
+    if x.is_cuda:
+        raise ValueError("a host pointer argument got a CUDA tensor: pass host (ideally pinned) memory")
+    if not x.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous (the library reads them as dense arrays)")
     return x.data_ptr()
 
 
@@ -244,7 +261,7 @@ def vattn_sta_fwd_host(geom: Geom, q, k, v, scale: float, o, lse, chunk_slices: 
     batch*head slices (q, k, v, o, lse: host tensors / addresses, raster)."""
     if workspace is not None and not ws_bytes:
         ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib.vattn_sta_fwd_host(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), scale, _ptr(o), _ptr(lse),
+    _check(lib.vattn_sta_fwd_host(ctypes.byref(geom), _hptr(q), _hptr(k), _hptr(v), scale, _hptr(o), _hptr(lse),
                                   int(chunk_slices), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
