@@ -64,7 +64,7 @@ def whole_job_tflops(flops_per_rank: float, ms: float, world: int) -> float:
 
 def _src_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd.cu", "common.cuh"):
+    for f in ("attn_fwd_2cta.cu", "fwd_common.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "video_dit_local_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -334,7 +334,8 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "peak_source": f"{peak_src} bf16 (burst)", "traffic": traffic,
-                     "kernel": "attn_fwd_kernel<128> (sliding tile, raster tensor-map boxes)", "kernel_ms": round(ms_kernel, 4),
+                     "kernel": "fwd2::attn_fwd_kernel<128> (two CTAs per SM; sliding tile, raster tensor-map boxes)",
+                     "kernel_ms": round(ms_kernel, 4),
                      "algorithmic_flop_per_launch": flops_local},
         "e2e": {"value": round(whole_job_tflops(flops_local, ms_e2e, world), 2), "unit": "TFLOP/s",
                 "ms_per_step": round(ms_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -369,28 +370,105 @@ def run_extras(V, dev):
 
         def call():
             V.vattn_dual_fwd(geom, q, k, v, gvec, scale, o, workspace=ws)
-        for _ in range(2):
-            call()
-        torch.cuda.synchronize()
-        n = 4
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(n):
-            call()
-        e1.record()
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / n
+        with ClockSampler(dev.index) as clk:
+            ms = _time_ms(call, 4)
         out[f"{name}_dual_fwd"] = {"ms": round(ms, 3), "eff_tflops": round((fl + fg) / ms / 1e9, 1),
                                    "frac": round((fl + fg) / ms / 1e9 / peaks["bf16_tflops"], 4),
-                                   "status": V.vattn_get_status()}
+                                   "status": V.vattn_get_status(), "clocks": clk.summary()}
         del q, k, v, o, ws
         torch.cuda.empty_cache()
-    out["train_fwd_bwd"] = _bench_train(V, dev, peaks)
-    out.update(_bench_xwin(V, dev, peaks))
-    out["1080p_dual_sym_fwd"] = _bench_sym(V, dev, peaks)
-    out["720p_hier_fwd_bwd"] = _bench_hier(V, dev, peaks)
-    out["720p_sta_fwd_fp8"] = _bench_fp8(V, dev, peaks)
-    out["1080p_dual_fwd_fp8"] = _bench_dual_fp8(V, dev, peaks)
+    def clocked(fn):
+        with ClockSampler(dev.index) as clk:
+            res = fn()
+        res["clocks"] = clk.summary()
+        return res
+
+    out["train_fwd_bwd"] = clocked(lambda: _bench_train(V, dev, peaks))
+    with ClockSampler(dev.index) as clk:
+        xw = _bench_xwin(V, dev, peaks)
+    for name, res in xw.items():
+        res["clocks"] = clk.summary()
+        out[name] = res
+    out["1080p_dual_sym_fwd"] = clocked(lambda: _bench_sym(V, dev, peaks))
+    out["720p_hier_fwd_bwd"] = clocked(lambda: _bench_hier(V, dev, peaks))
+    out["720p_sta_fwd_fp8"] = clocked(lambda: _bench_fp8(V, dev, peaks))
+    out["1080p_dual_fwd_fp8"] = clocked(lambda: _bench_dual_fp8(V, dev, peaks))
+    out["720p_sta_fwd_one_cta_design"] = clocked(lambda: _bench_one_cta(V, dev, peaks))
+    out["memory_bound"] = clocked(lambda: _bench_memory_bound(V, dev, peaks))
+    return out
+
+
+def _time_ms(fn, n, warm=2):
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def _bench_one_cta(V, dev, peaks):
+    """The 720p sliding-tile forward (raster) with the one-CTA-per-SM kernel
+    (two softmax groups on alternate key blocks), for comparison with the
+    default two-CTA kernel of the main line."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["720p"]
+    geom = _geom(V, w)
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 700 + i) for i in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    fl, _ = _flops_fwd(w)
+    V.vattn_debug_set(V.binding.VATTN_DEBUG_ONE_CTA_FWD, 0)
+    try:
+        ms = _time_ms(lambda: V.vattn_sta_fwd_raster(geom, q, k, v, 1 / math.sqrt(w.head_dim), o, lse), 5)
+    finally:
+        V.vattn_debug_set(0, 0)
+    res = {"ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
+           "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status()}
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return res
+
+
+def _bench_memory_bound(V, dev, peaks):
+    """The HBM-bound kernels on their own, algorithmic bytes over time: the
+    tile permute of one 720p tensor (read + write of every row) and the K/V
+    pooling at 1080p and 4K (K and V read, K_p and V_p written)."""
+    import torch
+    from synth import inputs as S
+    out = {}
+    w = S.WORKLOADS["720p"]
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    x = _device_randn(shape, 600)
+    y = torch.empty_like(x)
+    geom = _geom(V, w)
+    ms = _time_ms(lambda: V.vattn_tile_permute(geom, x, y), 10)
+    nbytes = 2 * x.numel() * 2
+    out["permute_720p"] = {"ms": round(ms, 4), "gbs": round(nbytes / ms / 1e6, 1),
+                           "frac_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    del x, y
+    for name in ("1080p", "4k"):
+        w = S.WORKLOADS[name]
+        geom = _geom(V, w)
+        shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+        k, v = (_device_randn(shape, 610 + i) for i in range(2))
+        npool = w.n_tokens // (w.pool[0] * w.pool[1] * w.pool[2])
+        kp = torch.empty((w.batch, w.heads, npool, w.head_dim), dtype=torch.bfloat16, device=dev)
+        vp = torch.empty_like(kp)
+        ms = _time_ms(lambda: V.vattn_pool_kv(geom, k, v, kp, vp), 10)
+        nbytes = 2 * k.numel() * 2 + 2 * kp.numel() * 2
+        out[f"pool_kv_{name}"] = {"ms": round(ms, 4), "gbs": round(nbytes / ms / 1e6, 1),
+                                  "frac_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+        del k, v, kp, vp
+        torch.cuda.empty_cache()
+    out["status"] = V.vattn_get_status()
     return out
 
 

@@ -70,7 +70,9 @@ typedef enum {
   VATTN_ERR_ALIGN = -4,
   VATTN_ERR_CUDA = -5,
   VATTN_ERR_DEVICE_TIMEOUT = -6,
-  VATTN_ERR_WORKSPACE = -7
+  VATTN_ERR_WORKSPACE = -7,
+  VATTN_ERR_DEVICE_BOUNDS = -8   /* debug build only: a kernel computed an out-of-range row, tile or
+                                    coordinate, skipped the access and stopped (vattn_get_status) */
 } vattn_status;
 
 /* Operation ids for vattn_workspace_size. */
@@ -173,27 +175,37 @@ int vattn_hier_bwd(const vattn_geom* geom, const void* q, const void* k, const v
 int vattn_sta_fwd_raster(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
                          float* lse, void* stream);
 
-/* Sliding-tile forward with Q*K^T in FP8 (e4m3) on the f8f6f4 tensor path,
- * P*V in bf16: an inference variant in the spirit of the 8-bit attention the
- * pages cite ("SageAttention"), which the pages do not define further.
- * Q and K are quantised per batch*head: scale s = absmax / 448 (the largest
- * finite e4m3), byte = round-to-nearest-even e4m3 of x * (448 / absmax) with
- * saturation; S = bytes(Q) bytes(K)^T * s_Q * s_K * scale in fp32.  Same
- * arguments and layouts as vattn_sta_fwd; d = 128 only.
- * workspace >= vattn_workspace_size(VATTN_OP_STA_FWD_FP8): e4m3 Q [B,h,N,d]
- * bytes at offset 0, e4m3 K at offset align256(B*h*N*d), then the absmax
- * bits as int32 [B*h][2] (Q, K); they hold this call's values afterwards. */
+/* Sliding-tile forward in FP8 (e4m3) on the f8f6f4 tensor path, for
+ * inference: both products, Q*K^T and P*V, take e4m3 operands, in the spirit
+ * of the 8-bit attention the pages cite ("SageAttention"), which the pages do
+ * not define further.
+ *  - Q, K and V are quantised per batch*head: scale s = absmax / 448 (the
+ *    largest finite e4m3), byte = round-to-nearest-even e4m3 of
+ *    x * (448 / absmax) with saturation; S = bytes(Q) bytes(K)^T * s_Q * s_K *
+ *    scale in fp32.
+ *  - P is rounded to e4m3 in the units 2^(S*log2(e) - m + 6), where the
+ *    running row maximum m is moved whenever a row's maximum grows by more
+ *    than a factor 4, so the largest P is at most 2^8 and probabilities down
+ *    to about 2^-15 of the row maximum keep a normal e4m3 value; the row sum
+ *    is accumulated in fp32 from the unrounded P; O = P_e4m3 bytes(V) * s_V /
+ *    row sum.
+ * Same arguments and layouts as vattn_sta_fwd; d = 128 only.
+ * workspace >= vattn_workspace_size(VATTN_OP_STA_FWD_FP8), in this order
+ * (each part starting on a 256-byte boundary): e4m3 Q, K, V [B,h,N,d]; the
+ * absmax bits as int32 [B*h][2] (Q, K); the absmax bits of V, int32 [B*h].
+ * They hold this call's values afterwards. */
 int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, float scale, void* o,
                       float* lse, void* workspace, size_t ws_bytes, void* stream);
 
-/* Dual forward (inference) with both branches' Q*K^T in FP8 (e4m3), as
+/* Dual forward (inference) with both branches in FP8 (e4m3), as
  * vattn_sta_fwd_fp8: O = g*O_local + (1-g)*O_global with K_p, V_p the bf16
- * average pools of K, V (as vattn_pool_kv), and Q, K, K_p quantised with one
- * absmax scale per batch*head each.  Tile-major q, k, v, o; g fp32 [heads].
- * workspace >= vattn_workspace_size(VATTN_OP_DUAL_FWD_FP8), in this order
- * (each part starting on a 256-byte boundary): e4m3 Q, e4m3 K [B,h,N,d];
- * e4m3 K_p [B,h,N_p,d]; absmax bits int32 [B*h][2] of (Q, K) and of (Q, K_p);
- * bf16 O_local [B,h,N,d]; bf16 K_p, V_p [B,h,N_p,d].  d = 128 only. */
+ * average pools of K, V (as vattn_pool_kv), and Q, K, V, K_p, V_p quantised
+ * with one absmax scale per batch*head each.  Tile-major q, k, v, o; g fp32
+ * [heads].  workspace >= vattn_workspace_size(VATTN_OP_DUAL_FWD_FP8), in this
+ * order (each part starting on a 256-byte boundary): e4m3 Q, K, V [B,h,N,d];
+ * e4m3 K_p, V_p [B,h,N_p,d]; absmax bits int32 [B*h][2] of (Q, K) and of
+ * (Q, K_p); absmax bits int32 [B*h] of V and of V_p; bf16 O_local [B,h,N,d];
+ * bf16 K_p, V_p [B,h,N_p,d].  d = 128 only. */
 int vattn_dual_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, const void* v, const float* g, float scale,
                        void* o, void* workspace, size_t ws_bytes, void* stream);
 
@@ -254,9 +266,11 @@ int vattn_dual_fwd(const vattn_geom* geom, const void* q, const void* k, const v
  *  - Geometries whose dual-forward workspace (vattn_workspace_size
  *    (VATTN_OP_DUAL_FWD)) exceeds VATTN_NOALLOC_SCRATCH_BYTES are rejected
  *    with VATTN_ERR_WORKSPACE before anything is launched.
- *  - The first call on each device resolves the scratch's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - The scratch has one device address per CUDA context.  The first call
+ *    in each context (the current device's primary context, or whichever
+ *    context the caller made current) resolves it with cudaGetSymbolAddress
+ *    and caches it under the context's unique id; make that first call before
+ *    any stream capture.
  *  - All calls on a device share the one scratch array and it keeps the last
  *    call's contents (nothing in it has to start at zero).  Calls whose work
  *    overlaps on the GPU (other streams, other host threads) race on it:
@@ -332,11 +346,23 @@ const char* vattn_last_error(void);
  * failed (the handles are released all the same). */
 int vattn_shutdown(void);
 
-/* Test hook.  flags bit 0: the attention kernels' load warp skips its first
- * arrival, so the consumer's bounded wait runs out (no fault, no hang);
- * timeout_ns: the device wait limit (<= 0 restores the default, 2 s).
- * Affects calls made after it on any thread. */
+/* Flags of vattn_debug_set. */
+#define VATTN_DEBUG_SKIP_ARRIVAL 1  /* the attention kernels' load warp skips its first arrival */
+#define VATTN_DEBUG_ONE_CTA_FWD 2   /* forwards run the one-CTA-per-SM kernel instead of the default
+                                       kernel with two co-resident CTAs per SM (same results) */
+
+/* Test hook.  flags: VATTN_DEBUG_SKIP_ARRIVAL makes the consumer's bounded
+ * wait run out (no fault, no hang); VATTN_DEBUG_ONE_CTA_FWD selects the other
+ * forward kernel design (for comparisons).  timeout_ns: the device wait limit
+ * (<= 0 restores the default, 2 s).  Affects calls made after it on any
+ * thread. */
 int vattn_debug_set(int flags, int64_t timeout_ns);
+
+/* Resident CTAs per SM of the default (two-CTA) forward kernel for head_dim
+ * (64 or 128) and e4m3 Q*K^T (fp8 != 0, head_dim 128 only), as the CUDA
+ * occupancy calculator reports it on the current device; the design needs 2.
+ * Returns the count, or a negative vattn_status. */
+int vattn_debug_fwd_ctas_per_sm(int head_dim, int fp8);
 
 /* Test hook: y[i] = the library's polynomial 2^x[i] (the one the attention
  * forward can run on the FMA pipe for one chunk of its exponentials; off in

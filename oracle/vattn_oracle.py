@@ -753,3 +753,43 @@ def hier_backward_dq_tiles(q, k, v, do, g: Geom, hpool: tuple, scale: float, til
         ids.append(qi)
         rows.append(dq)
     return np.concatenate(ids), np.concatenate(rows)
+
+
+def hier_backward_dkdv_tiles(q, k, v, do, g: Geom, hpool: tuple, scale: float, k_tiles):
+    """dK and dV of hier_backward for the tokens of the listed fine key tiles
+    of one head (2-D arrays).  A fine key token receives gradient twice: as a
+    fine key of every query tile whose sliding window holds its tile, and
+    through the medium pooling, as 1/|block| of the gradient of the pooled key
+    holding it, which every query tile whose coarse window holds that pooled
+    key contributes to.  Only the query tiles that see a wanted fine or pooled
+    key are evaluated; each is the full joint-softmax row of the definition.
+    Returns (raster key ids, dK rows, dV rows)."""
+    gh = g._replace(pool=tuple(hpool))
+    kh, vh = pool(k, gh), pool(v, gh)
+    u = pooled_index(gh)
+    cnt = hpool[0] * hpool[1] * hpool[2]
+    want = np.concatenate([_tile_token_box(g, tile_coords_of(g, int(t)), tuple(c + 1 for c in tile_coords_of(g, int(t))))
+                           for t in k_tiles])
+    want_set = set(int(x) for x in want)
+    coarse_set = set(int(x) for x in u[want])
+    dk_f = {t: np.zeros(q.shape[1]) for t in want_set}
+    dv_f = {t: np.zeros(q.shape[1]) for t in want_set}
+    dk_c = {c: np.zeros(q.shape[1]) for c in coarse_set}
+    dv_c = {c: np.zeros(q.shape[1]) for c in coarse_set}
+    for qi, kj, kc in _hier_query_tiles(g, hpool):
+        hit_f = [i for i, t in enumerate(kj) if int(t) in want_set]
+        hit_c = [i for i, c in enumerate(kc) if int(c) in coarse_set]
+        if not hit_f and not hit_c:
+            continue
+        _, dkeys, dvals = _softmax_attend_bwd(q[qi], np.concatenate([k[kj], kh[kc]]),
+                                              np.concatenate([v[kj], vh[kc]]), do[qi], scale)
+        nf = len(kj)
+        for i in hit_f:
+            dk_f[int(kj[i])] += dkeys[i]
+            dv_f[int(kj[i])] += dvals[i]
+        for i in hit_c:
+            dk_c[int(kc[i])] += dkeys[nf + i]
+            dv_c[int(kc[i])] += dvals[nf + i]
+    dk = np.stack([dk_f[int(t)] + dk_c[int(u[t])] / cnt for t in want])
+    dv = np.stack([dv_f[int(t)] + dv_c[int(u[t])] / cnt for t in want])
+    return want, dk, dv

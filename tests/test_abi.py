@@ -124,11 +124,13 @@ def test_workspace_sizes(V):
     # hierarchical forward (pool = h_pool): pooled K, V, then fine O and LSE
     assert V.vattn_workspace_size(V.VATTN_OP_HIER_FWD, g) == (2 * a(bh * npool * d * 2) + a(bh * n * d * 2)
                                                               + a(bh * n * 4))
-    # FP8 dual forward: e4m3 Q, K, K_p; two absmax pairs; bf16 O_local, K_p, V_p
+    # FP8 dual forward: e4m3 Q, K, V, K_p, V_p; two absmax pairs and two single
+    # absmax words per batch*head; bf16 O_local, K_p, V_p
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD_FP8, g) == (
-        2 * a(bh * n * d) + a(bh * npool * d) + 2 * a(bh * 8) + a(bh * n * d * 2) + 2 * a(bh * npool * d * 2))
-    # FP8 forward: e4m3 Q and K bytes, then two absmax words per batch*head
-    assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_FP8, g) == 2 * a(bh * n * d) + a(bh * 8)
+        3 * a(bh * n * d) + 2 * a(bh * npool * d) + 2 * a(bh * 8) + 2 * a(bh * 4) + a(bh * n * d * 2)
+        + 2 * a(bh * npool * d * 2))
+    # FP8 forward: e4m3 Q, K and V bytes, the (Q, K) absmax pairs, V's absmax
+    assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_FP8, g) == 3 * a(bh * n * d) + a(bh * 8) + a(bh * 4)
     # host-buffer forward, per slot: 8 bf16 token tensors and 2 fp32 rows
     assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, g) == 8 * a(bh * n * d * 2) + 2 * a(bh * n * 4)
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == (4 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)
@@ -148,7 +150,8 @@ def test_kernel_geometry_matches_oracle_inverse_ranges():
 
 def test_header_is_plain_c_and_links(V, tmp_path):
     """include/vattn.h compiles as C99 (no C++ or torch types in the
-    signatures) and a C program links against the library."""
+    signatures) and a C program links against the library; the constants the
+    binding copies from the header agree with it."""
     import shutil
     import subprocess
     cc = shutil.which("gcc") or shutil.which("cc")
@@ -163,6 +166,7 @@ def test_header_is_plain_c_and_links(V, tmp_path):
         "  size_t bytes = 0;\n"
         "  int r = vattn_workspace_size(VATTN_OP_DUAL_FWD, &g, &bytes);\n"
         '  printf("%d %zu %s\\n", r, bytes, vattn_version());\n'
+        '  printf("%llu\\n", (unsigned long long)VATTN_NOALLOC_SCRATCH_BYTES);\n'
         "  return r;\n"
         "}\n")
     exe = tmp_path / "use_vattn"
@@ -173,8 +177,11 @@ def test_header_is_plain_c_and_links(V, tmp_path):
     assert r.returncode == 0, r.stderr
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
-    code, nbytes, version = out.stdout.split(maxsplit=2)
+    first, second = out.stdout.strip().split("\n")
+    code, nbytes, version = first.split(maxsplit=2)
     assert code == "0" and int(nbytes) > 0 and "sm_100a" in version
+    # the binding's copy of the header's scratch limit
+    assert int(second) == V.binding.VATTN_NOALLOC_SCRATCH_BYTES
 
 
 def test_null_pointers_rejected_before_any_launch(V):

@@ -641,3 +641,17 @@ def test_hier_sampled_dq_equals_full_backward():
     tiles = [0, 7, 19, 63]
     ids, rows = O.hier_backward_dq_tiles(q[0, 0], k[0, 0], v[0, 0], do[0, 0], g, hp, 0.3, tiles)
     np.testing.assert_allclose(rows, dq[0, 0][ids], rtol=0, atol=1e-13)
+
+
+def test_hier_sampled_dkdv_equals_full_backward():
+    """The key-tile restriction of the hierarchical backward returns exactly
+    the rows of the full definition, for tiles at the grid's corners and in
+    its interior (so both the fine and the pooled contributions are met)."""
+    for g, hp in HIER_CASES:
+        q, k, v, do = (_rand((1, 1, g.n, 8), s) for s in (62, 63, 64, 65))
+        _, dk, dv = O.hier_backward(q, k, v, do, g, hp, 0.3)
+        n_tiles = math.prod(g.tiles_per_dim)
+        tiles = sorted({0, 3, n_tiles // 2, n_tiles - 1})
+        ids, rk, rv = O.hier_backward_dkdv_tiles(q[0, 0], k[0, 0], v[0, 0], do[0, 0], g, hp, 0.3, tiles)
+        np.testing.assert_allclose(rk, dk[0, 0][ids], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(rv, dv[0, 0][ids], rtol=0, atol=1e-13)

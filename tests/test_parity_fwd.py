@@ -261,10 +261,67 @@ def test_dual_fwd_1080p_sampled(V):
 
 
 def test_dual_fwd_4k_sampled(V):
+    """The 4K-shaped launch with its saved outputs.  Head 23 starts past 2^31
+    elements of every [B, h, N, d] tensor (23 * 725760 * 128 > 2^31), so its
+    rows are addressed only through 64-bit offsets: O, O_l, O_g, LSE_l and
+    LSE_g of heads 0 and 23 are compared on query tiles covering every
+    boundary class."""
     w = S.WORKLOADS["4k"]
-    check = [(0, 0)]
-    out = _dual_gpu(V, w, check, saved=False)
+    check = [(0, 0), (0, w.heads - 1)]
+    assert (w.heads - 1) * w.n_tokens * w.head_dim > 2 ** 31
+    out = _dual_gpu(V, w, check, saved=True)
     _check_dual(w, out, check, sample_tiles(O.geom_of(w).tiles_per_dim, 4))
+
+
+def _global_gpu(V, w, check, kp_bits, vp_bits):
+    """vattn_global_fwd on raster Q (the global branch has no tile order: every
+    query sees every pooled key) and host-pooled K_p, V_p given as bf16 bits
+    [B, h, N_p, d]."""
+    import torch
+    from helpers import bits_to_gpu
+    geom = geom_for(V, w)
+    q = gpu_tensor(w, S.Q_ID, check)
+    kp, vp = bits_to_gpu(kp_bits), bits_to_gpu(vp_bits)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:3], float("nan"), dtype=torch.float32, device="cuda")
+    V.vattn_global_fwd(geom, q, kp, vp, 1 / math.sqrt(w.head_dim), o, lse)
+    torch.cuda.synchronize()
+    assert V.vattn_get_status() == 0, V.vattn_last_error()
+    return o, lse
+
+
+@pytest.mark.parametrize("grid,tile,pool,d,batch,heads", [
+    ((3, 20, 24), (3, 4, 4), (1, 2, 2), 128, 2, 3),   # N = 1440, N_p = 360: both ragged against 128
+    ((4, 8, 24), (2, 4, 4), (2, 4, 3), 64, 1, 2),     # temporal pooling, N_p = 32 (one partial key block)
+    ((2, 8, 16), (1, 4, 4), (1, 1, 1), 128, 1, 2),    # pool 1: the global branch is full attention
+])
+def test_global_fwd_direct(V, grid, tile, pool, d, batch, heads):
+    """vattn_global_fwd called on its own, with K_p and V_p pooled on the host
+    (the exact block mean rounded to bf16), against the oracle's dense softmax
+    attention over those pooled keys; with pool 1 also against full attention
+    over the unpooled K, V."""
+    w = S.small_workload("global", 17, batch, heads, d, grid, tile, (1, 1, 1), pool)
+    g = O.geom_of(w)
+    check = [(b, h) for b in range(batch) for h in range(heads)]
+    kp_bits = np.empty((batch, heads, g.n_pooled, d), dtype=np.uint16)
+    vp_bits = np.empty_like(kp_bits)
+    for b, h in check:
+        kp_bits[b, h] = S.bf16_round_bits(O.pool(host_f64(w, S.K_ID, b, h), g).astype(np.float32))
+        vp_bits[b, h] = S.bf16_round_bits(O.pool(host_f64(w, S.V_ID, b, h), g).astype(np.float32))
+    o, lse = _global_gpu(V, w, check, kp_bits, vp_bits)
+    scale = 1 / math.sqrt(d)
+    for b, h in check:
+        q = host_f64(w, S.Q_ID, b, h)
+        kp, vp = S.bf16_bits_to_f64(kp_bits[b, h]), S.bf16_bits_to_f64(vp_bits[b, h])
+        o_ref, lse_ref = O.global_attention(q[None, None], kp[None, None], vp[None, None], scale)
+        assert_close(to_f64(o[b, h]), o_ref[0, 0], O_MAX_ABS, O_MEAN_ABS, f"O b{b} h{h}")
+        assert_close(lse[b, h].cpu().numpy().astype(np.float64), lse_ref[0, 0], LSE_MAX_ABS, what=f"LSE b{b} h{h}")
+        if pool == (1, 1, 1):
+            k, v = host_f64(w, S.K_ID, b, h), host_f64(w, S.V_ID, b, h)
+            o_full, lse_full = O.full_attention(q[None, None], k[None, None], v[None, None], scale)
+            assert_close(to_f64(o[b, h]), o_full[0, 0], O_MAX_ABS, O_MEAN_ABS, f"full O b{b} h{h}")
+            assert_close(lse[b, h].cpu().numpy().astype(np.float64), lse_full[0, 0], LSE_MAX_ABS,
+                         what=f"full LSE b{b} h{h}")
 
 
 # ------------------------------------------------------------------ failure detection
@@ -308,3 +365,42 @@ def test_polynomial_exp2_against_cuda_exp2f(V):
     yz = torch.empty_like(z)
     V.vattn_debug_exp2(z, yz)
     assert (yz >= 0).all() and (yz <= 2.0 ** -124).all()
+
+
+# ------------------------------------------------------------------ the two forward kernel designs
+
+def test_default_forward_kernel_runs_two_ctas_per_sm(V):
+    """The default forward puts two CTAs on every SM (each with its own
+    tcgen05 issuing thread); the occupancy calculator must agree for every
+    instantiation."""
+    for d, fp8 in ((128, False), (64, False), (128, True)):
+        assert V.vattn_debug_fwd_ctas_per_sm(d, fp8) == 2, (d, fp8)
+
+
+@pytest.mark.parametrize("case", ["tiny", "small_192", "small_384_d64", "720p"])
+def test_one_cta_forward_design_matches_oracle(V, case):
+    """The one-CTA-per-SM forward (two softmax groups on alternate key blocks,
+    kept for comparison, selected by VATTN_DEBUG_ONE_CTA_FWD) against the
+    oracle, and against the default kernel within the output bars."""
+    if case == "tiny":
+        w, check, tiles = S.WORKLOADS["tiny"], [(0, 0), (0, 1)], None
+    elif case == "small_192":
+        w = S.small_workload("sta", 11, 1, 2, 128, (6, 16, 24), (3, 8, 8), (1, 1, 3), (1, 1, 1))
+        check, tiles = [(0, 0), (0, 1)], None
+    elif case == "small_384_d64":
+        w = S.small_workload("sta", 11, 2, 1, 64, (6, 16, 32), (6, 8, 8), (1, 3, 3), (1, 1, 1))
+        check, tiles = [(0, 0), (1, 0)], None
+    else:
+        w = S.WORKLOADS["720p"]
+        check, tiles = [(0, 0)], sample_tiles(O.geom_of(w).tiles_per_dim, 4)
+    if tiles is None:
+        tiles = range(math.prod(O.geom_of(w).tiles_per_dim))
+    o2, l2 = _sta_gpu(V, w, check)
+    V.vattn_debug_set(V.binding.VATTN_DEBUG_ONE_CTA_FWD, 0)
+    try:
+        o1, l1 = _sta_gpu(V, w, check)
+    finally:
+        V.vattn_debug_set(0, 0)
+    _check_sta(w, o1, l1, check, tiles)
+    for b, h in check:
+        assert_close(to_f64(o1[b, h]), to_f64(o2[b, h]), O_MAX_ABS, O_MEAN_ABS, f"designs b{b} h{h}")

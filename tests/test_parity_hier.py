@@ -145,16 +145,26 @@ def test_hier_bwd_small_full(V, grid, tile, window, hpool, d, batch, heads):
             assert_close(to_f64(got[b, h]), ref[b, h], O_MAX_ABS, O_MEAN_ABS, f"{name} b{b} h{h}")
 
 
-def test_hier_bwd_720p_sampled_dq(V):
+def test_hier_bwd_720p_sampled(V):
     """The 720p shape (24 heads, h_pool 1x2x2) through forward and backward:
-    dQ of heads 0 and 23 on query tiles covering every boundary class."""
+    dQ of heads 0 and 23 on query tiles covering every boundary class, and
+    dK, dV of head 0 on a corner and an interior key tile.  A key's
+    gradient has a fine part (query tiles whose sliding window holds its tile)
+    and a coarse part through the medium pooling (query tiles whose coarse
+    window holds its pooled key), which the coarse-key pass computes."""
     w = S.small_workload("hier_720p_bwd", 64, 1, 24, 128, (30, 48, 80), (6, 8, 8), (3, 3, 3), (1, 2, 2))
     check = [(0, 0), (0, 23)]
-    dq, _, _ = _hier_fwd_bwd(V, w, check)
+    dq, dk, dv = _hier_fwd_bwd(V, w, check)
     g = O.geom_of(w)._replace(pool=(1, 1, 1))
     scale = 1 / math.sqrt(w.head_dim)
     tiles = sample_tiles(g.tiles_per_dim, 8)
+    nt, nh, nw = g.tiles_per_dim
+    k_tiles = [0, ((nt // 2) * nh + nh // 2) * nw + nw // 2]
     for b, h in check:
         q, k, v, do = (host_f64(w, i, b, h) for i in (S.Q_ID, S.K_ID, S.V_ID, S.DO_ID))
         ids, ref = O.hier_backward_dq_tiles(q, k, v, do, g, (1, 2, 2), scale, tiles)
         assert_close(to_f64(dq[b, h])[ids], ref, O_MAX_ABS, O_MEAN_ABS, f"dQ b{b} h{h}")
+        if h == 0:  # each key tile takes the oracle about a hundred query tiles of the joint softmax
+            kid, rk, rv = O.hier_backward_dkdv_tiles(q, k, v, do, g, (1, 2, 2), scale, k_tiles)
+            assert_close(to_f64(dk[b, h])[kid], rk, O_MAX_ABS, O_MEAN_ABS, f"dK b{b} h{h}")
+            assert_close(to_f64(dv[b, h])[kid], rv, O_MAX_ABS, O_MEAN_ABS, f"dV b{b} h{h}")

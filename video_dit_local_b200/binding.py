@@ -15,7 +15,9 @@ import os
 from typing import Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libvattn.so")
+# VATTN_DEBUG_BUILD=1 loads the debug build (device-side bounds checks; see
+# build.py) instead of the default library.
+LIB_PATH = os.path.join(_HERE, "libvattn_debug.so" if os.environ.get("VATTN_DEBUG_BUILD") == "1" else "libvattn.so")
 
 VATTN_OK = 0
 VATTN_ERR_INVALID_ARG = -1
@@ -25,6 +27,7 @@ VATTN_ERR_ALIGN = -4
 VATTN_ERR_CUDA = -5
 VATTN_ERR_DEVICE_TIMEOUT = -6
 VATTN_ERR_WORKSPACE = -7
+VATTN_ERR_DEVICE_BOUNDS = -8
 
 VATTN_OP_DUAL_FWD = 1
 VATTN_OP_STA_BWD = 2
@@ -37,6 +40,9 @@ VATTN_OP_HIER_BWD = 8
 VATTN_OP_STA_FWD_FP8 = 9
 VATTN_OP_DUAL_FWD_FP8 = 10
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+VATTN_DEBUG_SKIP_ARRIVAL = 1
+VATTN_DEBUG_ONE_CTA_FWD = 2
 
 
 class VattnError(RuntimeError):
@@ -104,6 +110,7 @@ _SIGS = {
     "vattn_shutdown": [],
     "vattn_debug_set": [_INT, _I64],
     "vattn_debug_exp2": [_P, _P, _I64, _P],
+    "vattn_debug_fwd_ctas_per_sm": [_INT, _INT],
     "vattn_version": [],
 }
 
@@ -333,6 +340,13 @@ def vattn_debug_set(flags: int, timeout_ns: int = 0) -> None:
 
 def vattn_debug_exp2(x, y, n: Optional[int] = None, stream=None) -> None:
     _check(lib.vattn_debug_exp2(_ptr(x), _ptr(y), x.numel() if n is None else n, _stream(stream)))
+
+
+def vattn_debug_fwd_ctas_per_sm(head_dim: int, fp8: bool = False) -> int:
+    """Resident CTAs per SM of the default forward kernel (the design needs 2)."""
+    n = lib.vattn_debug_fwd_ctas_per_sm(head_dim, 1 if fp8 else 0)
+    _check(min(n, 0))
+    return n
 
 
 def vattn_version() -> str:

@@ -58,6 +58,16 @@ __device__ __forceinline__ RowStream flat_stream(int n) {
   return s;
 }
 
+// Debug build: the rows [v, v + G) of stream position v lie inside the
+// stream's tensor (n rows per batch*head): a tiled stream's sub-box never
+// straddles a tile, a flat stream's only past its end; past the end of the
+// stream the zero-filled row n is loaded.
+__device__ __forceinline__ bool stream_box_ok(const RowStream& st, const DevGeom& g, int v, int G, int len, int n) {
+  if (v >= len) return true;
+  const int row = st.row(g, v);
+  return row >= 0 && (st.tiled ? row + G <= n : row < n);
+}
+
 // Key tiles kept by query tile q (its window).  The keys are the tiles of gk:
 // the query grid itself for the sliding tile (cf = 1); the coarse grid of the
 // hierarchical branch, whose window is centred on q's tile index / cf.  Rows
@@ -336,7 +346,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == WARP_LOAD_A || warp == WARP_LOAD_B) {
     if (lane == 0) {
       const bool is_a = warp == WARP_LOAD_A;  // A: K, V tiles, Q and LSE; B: dO and D
-      if (is_a) {
+      if (is_a && dcheck(key_row0 >= 0 && key_row0 < p.Nk, p.ctl.err_word)) {
         mbar_arrive_expect_tx(kv_full, 2 * L::KV_BYTES);
         for (int c = 0; c < L::CHUNKS; ++c) {
           tma_load_3d(smem + L::OFF_K + c * KBOX, &tm_k, kv_full, c * 64, key_row0, bh);
@@ -350,9 +360,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       float* vec_s = is_a ? lse_s : del_s;
       const uint32_t off_x = is_a ? L::OFF_Q : L::OFF_DO;
       int issued = 0;
-      for (int i = 0; i < nblk; ++i) {
+      if (is_a && !dcheck(key_row0 >= 0 && key_valid > 0 && key_row0 + key_valid <= p.Nk, p.ctl.err_word))
+        *abort_flag = 1;
+      for (int i = 0; i < nblk && !*abort_flag; ++i) {
         const int s = i % NQ, r = i / NQ;
         if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
+        if constexpr (kDebugChecks) {
+          bool good = true;
+          for (int u = 0; u < subs; ++u) good = good && stream_box_ok(qs, g, i * 64 + u * p.Gq, p.Gq, Lq, g.N);
+          if (!dcheck(good, p.ctl.err_word)) {
+            *abort_flag = 1;
+            break;
+          }
+        }
         // LSE / D rows: whole 16-byte groups by bulk copy when the source is
         // 16-byte aligned; a ragged tail (end of a flat query stream) or an
         // unaligned source (a pooled grid used as the token sequence, N_p not
@@ -514,7 +534,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float inv_cnt = 0.f;
         if (add && row_ok) {
           const int prow = p.hier_add ? coarse_of_tiled(g, p.gadd, (int)tok) : pooled_of_tiled(g, (int)tok);
-          add_row = add + ((size_t)bh * g.Np + prow) * D;
+          if (dcheck(prow >= 0 && prow < g.Np, p.ctl.err_word)) add_row = add + ((size_t)bh * g.Np + prow) * D;
           inv_cnt = 1.f / (float)(g.pt * g.ph * g.pw);
         }
         __nv_bfloat16* dst = (w == 0 ? p.dv : p.dk) + ((size_t)bh * g.N + tok) * D;
@@ -684,7 +704,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == WARP_LOAD_A || warp == WARP_LOAD_B) {
     if (lane == 0) {
       const bool is_k = warp == WARP_LOAD_A;
-      if (is_k) {
+      if (is_k && !dcheck(q_row0 >= 0 && q_valid > 0 && q_row0 + q_valid <= g.N, p.ctl.err_word)) *abort_flag = 1;
+      if (is_k && !*abort_flag) {
         mbar_arrive_expect_tx(qdo_full, 2 * L::QB_BYTES);
         for (int c = 0; c < L::CHUNKS; ++c) {
           tma_load_3d(smem + L::OFF_Q + c * QBOX, &tm_q, qdo_full, c * 64, q_row0, bh);
@@ -699,10 +720,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NS, r = j / NS;
         if (!mbar_wait(&empty[s], (r & 1) ^ 1, wc)) break;
-        mbar_arrive_expect_tx(&full[s], L::KB_BYTES);
         const int G = glob ? DQ_BN : p.G0;
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
         const int oob = glob ? g.Np : p.gk.N;
+        if constexpr (kDebugChecks) {
+          bool good = true;
+          for (int u = 0; u < DQ_BN / G; ++u) good = good && stream_box_ok(ks, p.gk, j * DQ_BN + u * G, G, Lk, oob);
+          if (!dcheck(good, p.ctl.err_word)) {
+            *abort_flag = 1;
+            break;
+          }
+        }
+        mbar_arrive_expect_tx(&full[s], L::KB_BYTES);
         for (int u = 0; u < DQ_BN / G; ++u) {
           const int v = j * DQ_BN + u * G;
           const int row = v < Lk ? ks.row(p.gk, v) : oob;
@@ -821,8 +850,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_float4(f[4 * v4], f[4 * v4 + 1], f[4 * v4 + 2], f[4 * v4 + 3]);
           } else {
             if (p.acc_in) {
-              const size_t arow =
-                  p.acc_pooled ? (size_t)bh * g.Np + pooled_of_tiled(g, q_row0 + row) : grow;
+              const int prow = p.acc_pooled ? pooled_of_tiled(g, q_row0 + row) : 0;
+              if (!dcheck(prow >= 0 && prow < g.Np, p.ctl.err_word)) continue;
+              const size_t arow = p.acc_pooled ? (size_t)bh * g.Np + prow : grow;
               const float w = p.acc_pooled ? 1.f / (float)(g.pt * g.ph * g.pw) : 1.f;
               const float4* src = reinterpret_cast<const float4*>(p.acc_in + arow * D + c0);
 #pragma unroll

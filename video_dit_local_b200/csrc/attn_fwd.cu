@@ -17,14 +17,12 @@
 // straight from TMEM.  The running max is only moved (and O rescaled) when a
 // row's max grows by more than 2^8; otherwise P may reach 2^8, which bf16 and
 // the fp32 accumulators carry without loss of relative precision.
-#include "common.cuh"
+#include "fwd_common.cuh"
 
 namespace vattn {
 
 namespace fwd {
 
-constexpr int BM = 128;
-constexpr int BN = 128;
 constexpr int NTHREADS = 352;
 constexpr int WARP_QK_LOAD = 8;
 constexpr int WARP_V_LOAD = 9;
@@ -59,108 +57,6 @@ struct Smem {
   static constexpr int TOTAL = OFF_XCH + 2 * 128 * 2 * 4;
   static constexpr int ALLOC = TOTAL + 1024;
 };
-
-struct Params {
-  DevGeom g;
-  int mode;
-  int G;             // rows per TMA sub-box of a key block (divides the tile volume)
-  int q_blocks_per_tile;
-  int Nk;            // key rows per batch*head in the K/V tensors
-  float scale_log2;  // scale * log2(e)
-  __nv_bfloat16* o;
-  float* lse;
-  const __nv_bfloat16* o_local;
-  const float* gvec;
-  __nv_bfloat16* blend_out;
-  // key-side tile grid and coarse factor (STA): the sliding tile has the query
-  // grid and factor 1; the hierarchical branch the coarse grid and h_pool
-  int kNt, kNh, kNw, cft, cfh, cfw;
-  const __nv_bfloat16* merge_o;  // hierarchical: fine-key O and LSE to merge with (NULL = none)
-  const float* merge_lse;
-  const int* qk_amax;            // e4m3 Q*K^T: absmax bits of Q and K per batch*head
-  // raster (STA only): Q, K, V, O and LSE in raster token order.  The tensor
-  // maps are 5-D (d, W, H, T, batch*head); a load is a box of whole t-slices
-  // of one tile, which lands in shared memory in the tile-major row order.
-  int raster;
-  DevCtl ctl;
-};
-
-__device__ __forceinline__ void tma_load_5d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2, int c3, int c4) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], "
-      "[%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-      : "memory");
-}
-
-
-// D[tmem] (+)= A[smem] * B[smem], e4m3 x e4m3 -> f32, K = 32 per instruction
-__device__ __forceinline__ void mma_ss_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Instruction descriptor, kind::f8f6f4: A, B e4m3 (format 0), K-major; D f32.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// Key stream of one CTA: `runs` runs of `run_len` contiguous rows.
-struct Stream {
-  int runs, run_len, eh, t0, h0, w0;
-  __device__ __forceinline__ int length() const { return runs * run_len; }
-};
-
-__device__ __forceinline__ Stream make_stream(const Params& p, int q_tile) {
-  Stream s;
-  if (p.mode == FWD_STA) {
-    const DevGeom& g = p.g;
-    const int at = q_tile / (g.Nh * g.Nw), ah = (q_tile / g.Nw) % g.Nh, aw = q_tile % g.Nw;
-    int et, ew;
-    tile_range(at / p.cft, g.wt, p.kNt, g.wmode, &s.t0, &et);
-    tile_range(ah / p.cfh, g.wh, p.kNh, g.wmode, &s.h0, &s.eh);
-    tile_range(aw / p.cfw, g.ww, p.kNw, g.wmode, &s.w0, &ew);
-    s.runs = et * s.eh;
-    s.run_len = ew * g.s;
-  } else {
-    s.runs = 1;
-    s.run_len = p.Nk;
-    s.eh = 1;
-    s.t0 = s.h0 = s.w0 = 0;
-  }
-  return s;
-}
-
-// Key row (within the batch*head slice) of stream position v < length().
-__device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int v) {
-  if (p.mode != FWD_STA) return v;
-  const int r = v / s.run_len, o = v - r * s.run_len;
-  const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
-  return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + o;
-}
-
-// Raster box of key stream position v (a multiple of the sub-box rows): the
-// x, y, t of its first token; past the end, t = T (a zero-filled box).
-__device__ __forceinline__ void stream_box(const Params& p, const Stream& s, int v, int L_total, int* x, int* y,
-                                           int* t) {
-  const DevGeom& g = p.g;
-  if (v >= L_total) {
-    *x = 0;
-    *y = 0;
-    *t = g.T;
-    return;
-  }
-  const int r = v / s.run_len, o = v - r * s.run_len;
-  const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
-  const int tile_in_run = o / g.s, lo = o - tile_in_run * g.s;
-  *x = (s.w0 + tile_in_run) * g.tw;
-  *y = kh * g.th;
-  *t = kt * g.tt + lo / (g.th * g.tw);
-}
 
 template <int D, bool F8 = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -250,7 +146,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == WARP_QK_LOAD) {
     if (lane == 0) {
       int issued_k = 0;
-      if (!(p.ctl.debug_flags & 1)) {
+      if (!dcheck(query_block_ok(p, q_row0, q_valid), p.ctl.err_word)) *abort_flag = 1;
+      if (!(p.ctl.debug_flags & 1) && !*abort_flag) {
         mbar_arrive_expect_tx(q_full, L::QK_BYTES);
         if (p.raster) {
           const DevGeom& g = p.g;
@@ -266,6 +163,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NK, r = j / NK;
         if (!mbar_wait(&qk_done[s], (r & 1) ^ 1, wc)) break;
+        if (!dcheck(key_block_ok(p, st, j, L_total), p.ctl.err_word)) {
+          *abort_flag = 1;
+          break;
+        }
         mbar_arrive_expect_tx(&k_full[s], L::QK_BYTES);
         uint8_t* dst = smem + L::OFF_K + s * L::QK_BYTES;
         for (int u = 0; u < subs; ++u) {
@@ -294,6 +195,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NV, r = j / NV;
         if (!mbar_wait(&v_empty[s], (r & 1) ^ 1, wc)) break;
+        if (!dcheck(key_block_ok(p, st, j, L_total), p.ctl.err_word)) {
+          *abort_flag = 1;
+          break;
+        }
         mbar_arrive_expect_tx(&v_full[s], L::BLOCK_BYTES);
         uint8_t* dst = smem + L::OFF_V + s * L::BLOCK_BYTES;
         for (int u = 0; u < subs; ++u) {
@@ -487,7 +392,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float a0 = (w == 0 ? a_self : a_other) * inv_l;
       const float a1 = (w == 0 ? a_other : a_self) * inv_l;
       const bool have1 = nblk >= 2;
-      const bool row_ok = row < q_valid;
+      bool row_ok = row < q_valid;
       size_t grow = (size_t)bh * p.g.N + (size_t)(q_row0 + row);
       if (p.raster) {  // tile-major row -> raster token
         const DevGeom& g = p.g;
@@ -496,6 +401,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int lt = lr / (g.th * g.tw), lh = (lr / g.tw) % g.th, lw = lr % g.tw;
         grow = (size_t)bh * g.N + ((size_t)(at * g.tt + lt) * g.H + (ah * g.th + lh)) * g.W + (aw * g.tw + lw);
       }
+      if (row_ok && !dcheck(out_row_ok(p, bh, grow), p.ctl.err_word)) row_ok = false;
       // hierarchical merge: one softmax over the fine keys (O_f, LSE_f given)
       // and this kernel's coarse keys, in log2 units
       float wf = 0.f, wc = 1.f, lse2_out = m + __log2f(l);
@@ -574,8 +480,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace fwd
 
-bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
-                    const char** err);
+template <int D, bool F8, bool F8V>
+cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fwd::Params& p,
+                        dim3 grid, cudaStream_t st);
 
 template <int D, bool F8 = false>
 static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
@@ -597,6 +504,7 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   p.merge_o = nullptr;
   p.merge_lse = nullptr;
   p.qk_amax = a.qk_amax;
+  p.v_amax = a.v_amax;
   p.raster = a.raster ? 1 : 0;
   int qblocks;
   if (mode == FWD_STA) {
@@ -635,6 +543,8 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
               make_tmap_raster(&tk, a.k, D, g, bh, p.G / slice, &err) &&
               make_tmap_raster(&tv, a.v, D, g, bh, p.G / slice, &err);
     if (!maps_ok) return cudaErrorInvalidValue;
+    if (!(p.ctl.debug_flags & VATTN_DEBUG_ONE_CTA_FWD))
+      return launch_fwd2<D, F8, false>(tq, tk, tv, p, dim3(qblocks, (unsigned)bh), st);
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Smem<D, F8>::ALLOC);
     if (e != cudaSuccess) return e;
@@ -645,7 +555,15 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
     maps_ok = make_tmap_rows_u8(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows_u8(&tk, a.k, D, p.Nk, bh, p.G, &err);
   else
     maps_ok = make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err);
+  if constexpr (F8) {
+    if (a.v_amax) {  // e4m3 P*V: V bytes, only the two-CTA kernel has this mode
+      if (!maps_ok || !make_tmap_rows_u8(&tv, a.v, D, p.Nk, bh, p.G, &err)) return cudaErrorInvalidValue;
+      return launch_fwd2<D, true, true>(tq, tk, tv, p, dim3(qblocks, (unsigned)bh), st);
+    }
+  }
   if (!maps_ok || !make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err)) return cudaErrorInvalidValue;
+  if (!(p.ctl.debug_flags & VATTN_DEBUG_ONE_CTA_FWD))
+    return launch_fwd2<D, F8, false>(tq, tk, tv, p, dim3(qblocks, (unsigned)bh), st);
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Smem<D, F8>::ALLOC);
   if (e != cudaSuccess) return e;
@@ -668,6 +586,7 @@ cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t
 }
 
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
+  if (a.v_amax && !a.qk_amax) return cudaErrorInvalidValue;  // e4m3 P*V comes with e4m3 Q*K^T
   if (a.qk_amax) {  // e4m3 Q*K^T: sliding tile or global (+ blend), d = 128
     if (g.d != 128 || a.kgeom || a.raster) return cudaErrorInvalidValue;
     return launch_fwd_d<128, true>(g, mode, a, st);

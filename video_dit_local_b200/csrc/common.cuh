@@ -31,6 +31,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // ---------------------------------------------------------------------------
+// Debug build (-DVATTN_DEBUG=1): bounds checks on the rows, tiles and TMA
+// coordinates the kernels compute.  A failed check records
+// VATTN_ERR_DEVICE_BOUNDS in the status word (first writer wins) and the
+// caller skips the access and stops; in the default build every check is the
+// constant `true` and compiles away.
+// ---------------------------------------------------------------------------
+#ifndef VATTN_DEBUG
+#define VATTN_DEBUG 0
+#endif
+constexpr bool kDebugChecks = VATTN_DEBUG != 0;
+
+__device__ __forceinline__ bool dcheck(bool ok, int* err_word) {
+  if constexpr (kDebugChecks) {
+    if (!ok) report_error(err_word, VATTN_ERR_DEVICE_BOUNDS);
+    return ok;
+  } else {
+    (void)err_word;
+    return true;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -187,6 +209,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // UMMA descriptors
 // ---------------------------------------------------------------------------
@@ -280,8 +308,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Two floats to e4m3 (round to nearest even, saturating): lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));  // first operand -> upper byte
+  return r;
+}
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Per-warpgroup register budgets (sm_100 setmaxnreg): every warp of a
+// warpgroup executes the same instruction.  An increase draws on the
+// registers the CTA was launched with, so the shares of all warpgroups must
+// add up to at most threads x registers-per-thread at launch.
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -14,7 +14,6 @@
 // holds on every GPU that loads it, until the process exits.  It allocates
 // nothing itself.
 #include <cstdio>
-#include <mutex>
 
 #include "common.cuh"
 
@@ -30,27 +29,19 @@ constexpr size_t kNoAllocScratchBytes = VATTN_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
-
-// Set-up, once per device, with that device current: resolve the device
-// address of the scratch array.
+// Set-up, once per CUDA context (the current device's primary context unless
+// the caller made another one current): resolve the scratch array's device
+// address with cudaGetSymbolAddress.  Later calls in the same context reuse
+// the cached address, so the first call in a context must come before any
+// stream capture.
 int scratch_address(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return record_error(VATTN_ERR_CUDA, "vattn_dual_fwd_noalloc: cudaGetDevice failed");
-  if (dev < 0 || dev >= kMaxDevices)
-    return record_error(VATTN_ERR_UNSUPPORTED, "vattn_dual_fwd_noalloc: device index out of range");
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return record_error(VATTN_ERR_CUDA, "vattn_dual_fwd_noalloc: cudaGetSymbolAddress of the scratch failed");
-    g_scratch_addr[dev] = p;
+  const cudaError_t e = context_symbol_address(reinterpret_cast<const void*>(&g_noalloc_scratch), out);
+  if (e != cudaSuccess) {
+    char msg[192];
+    snprintf(msg, sizeof(msg), "vattn_dual_fwd_noalloc: cudaGetSymbolAddress of the scratch failed: %s",
+             cudaGetErrorString(e));
+    return record_error(VATTN_ERR_CUDA, msg);
   }
-  *out = g_scratch_addr[dev];
   return VATTN_OK;
 }
 }  // namespace

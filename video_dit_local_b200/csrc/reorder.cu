@@ -89,7 +89,7 @@ static ReorderParams make_params(const DevGeom& g) {
 template <bool TO_TILED, typename U>
 __global__ void __launch_bounds__(256) permute_kernel(ReorderParams p, FastDiv per_row, FastDiv n_rows,
                                                        const U* __restrict__ src, U* __restrict__ dst,
-                                                       uint32_t total) {
+                                                       uint32_t total, int* err) {
   const uint32_t stride = gridDim.x * blockDim.x;
   for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
     const uint32_t row = per_row.div(i);
@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(256) permute_kernel(ReorderParams p, FastDiv p
     const uint32_t bh = n_rows.div(row);
     const uint32_t r = row - bh * n_rows.d;
     const uint32_t sr = TO_TILED ? tiled_to_raster(p, r) : raster_to_tiled(p, r);
+    if (!dcheck(sr < n_rows.d, err)) continue;
     const U v = __ldg(src + ((size_t)bh * n_rows.d + sr) * per_row.d + c);
     __stcs(dst + i, v);
   }
@@ -116,6 +117,7 @@ template <typename U>
 static cudaError_t permute_typed(const DevGeom& g, const void* src, void* dst, uint32_t units, bool to_tiled,
                                  cudaStream_t st) {
   const ReorderParams p = make_params(g);
+  int* err = current_ctl().err_word;
   const long long per_bh = (long long)g.N * units;
   const long long bh_total = (long long)g.B * g.heads;
   long long chunk = ((1ll << 31) - 1) / per_bh;
@@ -127,9 +129,9 @@ static cudaError_t permute_typed(const DevGeom& g, const void* src, void* dst, u
     U* d = (U*)dst + b0 * per_bh;
     const int grid = grid_for(total, 256);
     if (to_tiled)
-      permute_kernel<true, U><<<grid, 256, 0, st>>>(p, FastDiv(units), FastDiv(g.N), s, d, total);
+      permute_kernel<true, U><<<grid, 256, 0, st>>>(p, FastDiv(units), FastDiv(g.N), s, d, total, err);
     else
-      permute_kernel<false, U><<<grid, 256, 0, st>>>(p, FastDiv(units), FastDiv(g.N), s, d, total);
+      permute_kernel<false, U><<<grid, 256, 0, st>>>(p, FastDiv(units), FastDiv(g.N), s, d, total, err);
   }
   return cudaGetLastError();
 }
@@ -188,8 +190,12 @@ struct PoolTensors {
 // One thread produces one 16-byte vector (8 bf16) of one pooled row: the fp32
 // sum of the block's tokens in (t, y, x) order, divided by the block size
 // (one correctly rounded fp32 division), one round-to-nearest-even to bf16.
+// PWC > 0 is the pool width known at compile time: the PWC loads of one
+// (t, y) row of the block are issued together before they are summed (in the
+// same x order), so more loads are in flight per thread.
+template <int PWC>
 __global__ void __launch_bounds__(256) pool_kv_kernel(PoolParams p, FastDiv per_row, FastDiv n_prow,
-                                                       FastDiv rows_per_tensor, PoolTensors ts) {
+                                                       FastDiv rows_per_tensor, PoolTensors ts, int* err) {
   const uint32_t total = (uint32_t)ts.count * rows_per_tensor.d * p.vpr;
   const uint32_t stride = gridDim.x * blockDim.x;
   const float cnt = (float)(p.pt * p.ph * p.pw);
@@ -209,23 +215,44 @@ __global__ void __launch_bounds__(256) pool_kv_kernel(PoolParams p, FastDiv per_
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
     for (uint32_t a = 0; a < p.pt; ++a)
-      for (uint32_t b = 0; b < p.ph; ++b)
-        for (uint32_t x = 0; x < p.pw; ++x) {
-          const uint32_t m = coords_to_tiled(p.rp, ut * p.pt + a, uy * p.ph + b, ux * p.pw + x);
-          const uint4 w = __ldg(src + (size_t)m * p.vpr);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      for (uint32_t b = 0; b < p.ph; ++b) {
+        if constexpr (PWC > 0) {
+          uint4 w[PWC];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            acc[2 * e] += bf16lo(ww[e]);
-            acc[2 * e + 1] += bf16hi(ww[e]);
+          for (int x = 0; x < PWC; ++x) {
+            const uint32_t m = coords_to_tiled(p.rp, ut * p.pt + a, uy * p.ph + b, ux * PWC + x);
+            w[x] = dcheck(m < p.N, err) ? __ldg(src + (size_t)m * p.vpr) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int x = 0; x < PWC; ++x) {
+            const uint32_t ww[4] = {w[x].x, w[x].y, w[x].z, w[x].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc[2 * e] += bf16lo(ww[e]);
+              acc[2 * e + 1] += bf16hi(ww[e]);
+            }
+          }
+        } else {
+          for (uint32_t x = 0; x < p.pw; ++x) {
+            const uint32_t m = coords_to_tiled(p.rp, ut * p.pt + a, uy * p.ph + b, ux * p.pw + x);
+            if (!dcheck(m < p.N, err)) continue;
+            const uint4 w = __ldg(src + (size_t)m * p.vpr);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc[2 * e] += bf16lo(ww[e]);
+              acc[2 * e + 1] += bf16hi(ww[e]);
+            }
           }
         }
+      }
     uint4 o;
     o.x = pack_bf16(acc[0] / cnt, acc[1] / cnt);
     o.y = pack_bf16(acc[2] / cnt, acc[3] / cnt);
     o.z = pack_bf16(acc[4] / cnt, acc[5] / cnt);
     o.w = pack_bf16(acc[6] / cnt, acc[7] / cnt);
     const uint32_t uo = p.out_tiled ? coords_to_tiled(p.rpo, ut, uy, ux) : u;
+    if (!dcheck(uo < p.Np, err)) continue;
     ts.dst[which][((size_t)bh * p.Np + uo) * p.vpr + c] = o;
   }
 }
@@ -272,8 +299,16 @@ static cudaError_t pool_tensors(const DevGeom& g, int count, const void* const* 
       ts.src[i] = (const uint4*)src[j] + in_off;
       ts.dst[i] = (uint4*)dst[j] + out_off;
     }
-    pool_kv_kernel<<<grid_for((long long)count * rows * p.vpr, 256), 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np),
-                                                                                 FastDiv(rows), ts);
+    const int grid = grid_for((long long)count * rows * p.vpr, 256);
+    int* err = current_ctl().err_word;
+    if (g.pw == 4)
+      pool_kv_kernel<4><<<grid, 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np), FastDiv(rows), ts, err);
+    else if (g.pw == 8)
+      pool_kv_kernel<8><<<grid, 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np), FastDiv(rows), ts, err);
+    else if (g.pw == 2)
+      pool_kv_kernel<2><<<grid, 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np), FastDiv(rows), ts, err);
+    else
+      pool_kv_kernel<0><<<grid, 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np), FastDiv(rows), ts, err);
   }
   return cudaGetLastError();
 }

@@ -15,21 +15,87 @@ namespace vattn {
 __device__ int g_error_word = 0;
 
 static thread_local std::string t_last_error;
-static std::atomic<int> s_debug_flags{0};
+static std::atomic<int> s_debug_flags{0};  // VATTN_DEBUG_* bits
 static std::atomic<long long> s_timeout_ns{2000000000ll};
 
-// Address of this device's status word (cached per device).
-static int* error_word_ptr() {
-  static int* cache[64] = {nullptr};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!cache[dev]) {
+// ---------------------------------------------------------------------------
+// Device addresses of the library's __device__ variables, per CUDA context.
+// A variable has one address per context that loaded the module, so a cache
+// keyed on the device index would hand out a dangling address once the
+// caller makes another context current (a framework's own context, or the
+// primary context recreated after cudaDeviceReset).  The key is the context's
+// unique id (cuCtxGetId, never reused within the process), fetched through
+// the driver entry points like the tensor-map encoder.
+// ---------------------------------------------------------------------------
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_error_word) == cudaSuccess) cache[dev] = (int*)p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+cudaError_t context_symbol_address(const void* symbol, void** out) {
+  struct Entry {
+    unsigned long long ctx;
+    const void* symbol;
+    void* addr;
+  };
+  constexpr int kEntries = 64;
+  static Entry table[kEntries] = {};
+  static int used = 0, next = 0;
+  static std::mutex mu;
+  unsigned long long id = 0;
+  if (current_context_id(&id)) {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i)
+      if (table[i].ctx == id && table[i].symbol == symbol) {
+        *out = table[i].addr;
+        return cudaSuccess;
+      }
   }
-  return cache[dev];
+  // Miss (or no context yet): resolve, which also creates the primary
+  // context when none is current, then record under the now-current id.
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, symbol);
+  if (e != cudaSuccess) return e;
+  if (p == nullptr) return cudaErrorInvalidSymbol;
+  if (current_context_id(&id)) {
+    std::lock_guard<std::mutex> lk(mu);
+    int slot;
+    if (used < kEntries) {
+      slot = used++;
+    } else {  // full: overwrite round robin (an evicted entry is resolved again)
+      slot = next;
+      next = (next + 1) % kEntries;
+    }
+    table[slot] = Entry{id, symbol, p};
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
+// Address of the current context's status word.
+static int* error_word_ptr() {
+  void* p = nullptr;
+  if (context_symbol_address(reinterpret_cast<const void*>(&g_error_word), &p) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
 }
 
 DevCtl current_ctl() {
@@ -299,7 +365,7 @@ static SymBwdWs sym_bwd_ws(const DevGeom& g) {
 
 // FP8 forward: e4m3 Q, K bytes and the per-batch*head absmax words.
 struct Fp8FwdWs {
-  size_t q8, k8, amax, total;
+  size_t q8, k8, v8, amax, vamax, total;
 };
 static Fp8FwdWs fp8_fwd_ws(const DevGeom& g) {
   Fp8FwdWs w;
@@ -307,25 +373,32 @@ static Fp8FwdWs fp8_fwd_ws(const DevGeom& g) {
   const size_t t = align256(bh * g.N * g.d);
   w.q8 = 0;
   w.k8 = t;
-  w.amax = 2 * t;
-  w.total = 2 * t + align256(bh * 2 * 4);
+  w.v8 = 2 * t;
+  w.amax = 3 * t;
+  w.vamax = w.amax + align256(bh * 2 * 4);
+  w.total = w.vamax + align256(bh * 4);
   return w;
 }
 
 // FP8 dual forward, in the order the header documents.
 struct DualFp8Ws {
-  size_t q8, k8, kp8, amax_l, amax_g, o_l, kp, vp, total;
+  size_t q8, k8, v8, kp8, vp8, amax_l, amax_g, vamax_l, vamax_g, o_l, kp, vp, total;
 };
 static DualFp8Ws dual_fp8_ws(const DevGeom& g) {
   DualFp8Ws w;
   const size_t bh = (size_t)g.B * g.heads;
-  const size_t t8 = align256(bh * g.N * g.d), p8 = align256(bh * g.Np * g.d), am = align256(bh * 2 * 4);
+  const size_t t8 = align256(bh * g.N * g.d), p8 = align256(bh * g.Np * g.d), am = align256(bh * 2 * 4),
+               av = align256(bh * 4);
   w.q8 = 0;
   w.k8 = t8;
-  w.kp8 = 2 * t8;
-  w.amax_l = w.kp8 + p8;
+  w.v8 = 2 * t8;
+  w.kp8 = 3 * t8;
+  w.vp8 = w.kp8 + p8;
+  w.amax_l = w.vp8 + p8;
   w.amax_g = w.amax_l + am;
-  w.o_l = w.amax_g + am;
+  w.vamax_l = w.amax_g + am;
+  w.vamax_g = w.vamax_l + av;
+  w.o_l = w.vamax_g + av;
   w.kp = w.o_l + align256(bh * g.N * g.d * 2);
   w.vp = w.kp + align256(bh * g.Np * g.d * 2);
   w.total = w.vp + align256(bh * g.Np * g.d * 2);
@@ -468,6 +541,16 @@ int vattn_debug_set(int flags, int64_t timeout_ns) {
   s_debug_flags.store(flags);
   s_timeout_ns.store(timeout_ns > 0 ? (long long)timeout_ns : 2000000000ll);
   return ok();
+}
+
+int vattn_debug_fwd_ctas_per_sm(int head_dim, int fp8) {
+  if (!(head_dim == 64 || head_dim == 128) || (fp8 && head_dim != 128))
+    return fail(VATTN_ERR_UNSUPPORTED, "vattn_debug_fwd_ctas_per_sm: head_dim %d%s unsupported", head_dim,
+                fp8 ? " with fp8" : "");
+  const int n = fwd2_ctas_per_sm(head_dim, fp8 != 0);
+  if (n < 0) return fail(VATTN_ERR_CUDA, "vattn_debug_fwd_ctas_per_sm: occupancy query failed");
+  ok();
+  return n;
 }
 
 int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream) {
@@ -907,11 +990,16 @@ int vattn_dual_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, con
   const long long bh = (long long)g.B * g.heads;
   int* amax_l = (int*)(ws + w.amax_l);
   int* amax_g = (int*)(ws + w.amax_g);
+  int* vamax_l = (int*)(ws + w.vamax_l);
+  int* vamax_g = (int*)(ws + w.vamax_g);
   CHECK_LAUNCH(launch_pool_kv(g, k, v, ws + w.kp, ws + w.vp, st), "dual_fwd_fp8 pool launch");
   CHECK_LAUNCH(launch_quant_e4m3(q, g.N, bh, g.d, ws + w.q8, amax_l, 2, st), "dual_fwd_fp8 quantise Q launch");
   CHECK_LAUNCH(launch_quant_e4m3(k, g.N, bh, g.d, ws + w.k8, amax_l + 1, 2, st), "dual_fwd_fp8 quantise K launch");
+  CHECK_LAUNCH(launch_quant_e4m3(v, g.N, bh, g.d, ws + w.v8, vamax_l, 1, st), "dual_fwd_fp8 quantise V launch");
   CHECK_LAUNCH(launch_quant_e4m3(ws + w.kp, g.Np, bh, g.d, ws + w.kp8, amax_g + 1, 2, st),
                "dual_fwd_fp8 quantise K_p launch");
+  CHECK_LAUNCH(launch_quant_e4m3(ws + w.vp, g.Np, bh, g.d, ws + w.vp8, vamax_g, 1, st),
+               "dual_fwd_fp8 quantise V_p launch");
   // the global pass's Q scale: the same absmax as the local pass's
   CHECK_LAUNCH(cudaMemcpy2DAsync(amax_g, 2 * sizeof(int), amax_l, 2 * sizeof(int), sizeof(int), bh,
                                  cudaMemcpyDeviceToDevice, st),
@@ -919,20 +1007,22 @@ int vattn_dual_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, con
   FwdArgs a{};
   a.q = ws + w.q8;
   a.k = ws + w.k8;
-  a.v = v;
+  a.v = ws + w.v8;
   a.o = ws + w.o_l;
   a.scale = scale;
   a.qk_amax = amax_l;
+  a.v_amax = vamax_l;
   CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "dual_fwd_fp8 local launch");
   FwdArgs b{};
   b.q = ws + w.q8;
   b.k = ws + w.kp8;
-  b.v = ws + w.vp;
+  b.v = ws + w.vp8;
   b.scale = scale;
   b.o_local = ws + w.o_l;
   b.g = gvec;
   b.blend_out = o;
   b.qk_amax = amax_g;
+  b.v_amax = vamax_g;
   CHECK_LAUNCH(launch_attn_fwd(g, FWD_GLOBAL, b, st), "dual_fwd_fp8 global launch");
   return ok();
 }
@@ -959,14 +1049,17 @@ int vattn_sta_fwd_fp8(const vattn_geom* geom, const void* q, const void* k, cons
   const long long bh = (long long)g.B * g.heads;
   CHECK_LAUNCH(launch_quant_e4m3(q, g.N, bh, g.d, ws + w.q8, amax, 2, st), "sta_fwd_fp8 quantise Q launch");
   CHECK_LAUNCH(launch_quant_e4m3(k, g.N, bh, g.d, ws + w.k8, amax + 1, 2, st), "sta_fwd_fp8 quantise K launch");
+  int* vamax = (int*)(ws + w.vamax);
+  CHECK_LAUNCH(launch_quant_e4m3(v, g.N, bh, g.d, ws + w.v8, vamax, 1, st), "sta_fwd_fp8 quantise V launch");
   FwdArgs a{};
   a.q = ws + w.q8;
   a.k = ws + w.k8;
-  a.v = v;
+  a.v = ws + w.v8;
   a.o = o;
   a.lse = lse;
   a.scale = scale;
   a.qk_amax = amax;
+  a.v_amax = vamax;
   CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "sta_fwd_fp8 launch");
   return ok();
 }

@@ -36,13 +36,19 @@ enum { WIN_SLIDING = 0, WIN_PARTITION = 1, WIN_SHIFTED = 2 };
 struct DevCtl {
   unsigned long long timeout_ns;
   int* err_word;            // device status word (first writer wins)
-  int debug_flags;          // bit 0: skip the first producer arrival
+  int debug_flags;          // VATTN_DEBUG_* bits (vattn.h)
 };
 
 DevCtl current_ctl();
 
 // Records `msg` as this thread's last error and returns `code`.
 int record_error(int code, const char* msg);
+
+// Device address of the library's __device__ variable `symbol` in the calling
+// thread's current CUDA context (the primary context of the current device
+// is created when none is current).  Cached per context: the first lookup in
+// a context calls cudaGetSymbolAddress, so make it before any stream capture.
+cudaError_t context_symbol_address(const void* symbol, void** out);
 
 // -- reorder / pooling (reorder.cu) --
 cudaError_t launch_permute(const DevGeom& g, const void* src, void* dst, int64_t row_bytes, bool to_tiled,
@@ -90,11 +96,16 @@ struct FwdArgs {
   // qk_amax[2 bh] / [2 bh + 1] are the absmax float bits of Q / K (scale
   // absmax / 448).  d = 128 only.
   const int* qk_amax;
+  // with qk_amax: v holds e4m3 bytes too (P*V on the f8f6f4 tensor path, P
+  // rounded to e4m3); v_amax[bh] is V's absmax float bits (scale absmax / 448)
+  const int* v_amax;
   // STA only: q, k, v, o and lse in raster token order (5-D tensor maps; the
   // tile's t-slice, th*tw rows, must divide 128 and the key sub-box)
   bool raster;
 };
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
+// Resident CTAs per SM of the two-CTA forward kernel (-1 on error).
+int fwd2_ctas_per_sm(int d, bool f8);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st);
 
 // -- attention backward (attn_bwd.cu) --
