@@ -64,7 +64,7 @@ def whole_job_tflops(flops_per_rank: float, ms: float, world: int) -> float:
 
 def _src_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_fwd_2cta.cu", "fwd_common.cuh", "common.cuh"):
+    for f in ("attn_fwd.cu", "fwd_common.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "video_dit_local_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -334,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "frac_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "peak_source": f"{peak_src} bf16 (burst)", "traffic": traffic,
-                     "kernel": "fwd2::attn_fwd_kernel<128> (two CTAs per SM; sliding tile, raster tensor-map boxes)",
+                     "kernel": "fwd::attn_fwd_kernel<128> (sliding tile, raster tensor-map boxes)",
                      "kernel_ms": round(ms_kernel, 4),
                      "algorithmic_flop_per_launch": flops_local},
         "e2e": {"value": round(whole_job_tflops(flops_local, ms_e2e, world), 2), "unit": "TFLOP/s",
@@ -393,7 +393,6 @@ def run_extras(V, dev):
     out["720p_hier_fwd_bwd"] = clocked(lambda: _bench_hier(V, dev, peaks))
     out["720p_sta_fwd_fp8"] = clocked(lambda: _bench_fp8(V, dev, peaks))
     out["1080p_dual_fwd_fp8"] = clocked(lambda: _bench_dual_fp8(V, dev, peaks))
-    out["720p_sta_fwd_one_cta_design"] = clocked(lambda: _bench_one_cta(V, dev, peaks))
     out["memory_bound"] = clocked(lambda: _bench_memory_bound(V, dev, peaks))
     return out
 
@@ -410,31 +409,6 @@ def _time_ms(fn, n, warm=2):
     e1.record()
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / n
-
-
-def _bench_one_cta(V, dev, peaks):
-    """The 720p sliding-tile forward (raster) with the one-CTA-per-SM kernel
-    (two softmax groups on alternate key blocks), for comparison with the
-    default two-CTA kernel of the main line."""
-    import torch
-    from synth import inputs as S
-    w = S.WORKLOADS["720p"]
-    geom = _geom(V, w)
-    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
-    q, k, v = (_device_randn(shape, 700 + i) for i in range(3))
-    o = torch.empty_like(q)
-    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
-    fl, _ = _flops_fwd(w)
-    V.vattn_debug_set(V.binding.VATTN_DEBUG_ONE_CTA_FWD, 0)
-    try:
-        ms = _time_ms(lambda: V.vattn_sta_fwd_raster(geom, q, k, v, 1 / math.sqrt(w.head_dim), o, lse), 5)
-    finally:
-        V.vattn_debug_set(0, 0)
-    res = {"ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
-           "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status()}
-    del q, k, v, o, lse
-    torch.cuda.empty_cache()
-    return res
 
 
 def _bench_memory_bound(V, dev, peaks):

@@ -348,21 +348,13 @@ int vattn_shutdown(void);
 
 /* Flags of vattn_debug_set. */
 #define VATTN_DEBUG_SKIP_ARRIVAL 1  /* the attention kernels' load warp skips its first arrival */
-#define VATTN_DEBUG_ONE_CTA_FWD 2   /* forwards run the one-CTA-per-SM kernel instead of the default
-                                       kernel with two co-resident CTAs per SM (same results) */
 
 /* Test hook.  flags: VATTN_DEBUG_SKIP_ARRIVAL makes the consumer's bounded
- * wait run out (no fault, no hang); VATTN_DEBUG_ONE_CTA_FWD selects the other
- * forward kernel design (for comparisons).  timeout_ns: the device wait limit
+ * wait run out (no fault, no hang).  timeout_ns: the device wait limit
  * (<= 0 restores the default, 2 s).  Affects calls made after it on any
  * thread. */
 int vattn_debug_set(int flags, int64_t timeout_ns);
 
-/* Resident CTAs per SM of the default (two-CTA) forward kernel for head_dim
- * (64 or 128) and e4m3 Q*K^T (fp8 != 0, head_dim 128 only), as the CUDA
- * occupancy calculator reports it on the current device; the design needs 2.
- * Returns the count, or a negative vattn_status. */
-int vattn_debug_fwd_ctas_per_sm(int head_dim, int fp8);
 
 /* Test hook: y[i] = the library's polynomial 2^x[i] (the one the attention
  * forward can run on the FMA pipe for one chunk of its exponentials; off in

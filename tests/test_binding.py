@@ -86,7 +86,6 @@ def _calls(B):
         "vattn_shutdown": lambda: B.vattn_shutdown(),
         "vattn_debug_set": lambda: B.vattn_debug_set(0, 0),
         "vattn_debug_exp2": lambda: B.vattn_debug_exp2(t(), t()),
-        "vattn_debug_fwd_ctas_per_sm": lambda: B.vattn_debug_fwd_ctas_per_sm(128),
     }
 
 

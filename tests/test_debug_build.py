@@ -7,7 +7,8 @@ default library and once with the debug build, each in its own process.  In
 both, every call must leave the status word at VATTN_OK (the debug build
 would report VATTN_ERR_DEVICE_BOUNDS for any out-of-range row, tile or TMA
 coordinate it computed) and every canary intact; the two builds' outputs must
-be bit-identical (the checks add branches, not arithmetic).
+be bit-identical (the checks add branches, not arithmetic), except dg, whose
+per-block partials are summed with atomics in a varying order.
 """
 import os
 import subprocess
@@ -43,4 +44,7 @@ def test_debug_build_checks_pass_and_match_the_default_build(tmp_path):
     dbg = _run(tmp_path, debug=True)
     assert sorted(ref.files) == sorted(dbg.files)
     for name in ref.files:
-        assert np.array_equal(ref[name], dbg[name]), name
+        if name == "dg":  # sums per-block partials with atomics: the order of the adds varies
+            np.testing.assert_allclose(ref[name], dbg[name], rtol=1e-5, atol=1e-6)
+        else:
+            assert np.array_equal(ref[name], dbg[name]), name

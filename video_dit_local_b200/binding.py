@@ -42,7 +42,6 @@ VATTN_OP_DUAL_FWD_FP8 = 10
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 VATTN_DEBUG_SKIP_ARRIVAL = 1
-VATTN_DEBUG_ONE_CTA_FWD = 2
 
 
 class VattnError(RuntimeError):
@@ -110,7 +109,6 @@ _SIGS = {
     "vattn_shutdown": [],
     "vattn_debug_set": [_INT, _I64],
     "vattn_debug_exp2": [_P, _P, _I64, _P],
-    "vattn_debug_fwd_ctas_per_sm": [_INT, _INT],
     "vattn_version": [],
 }
 
@@ -340,13 +338,6 @@ def vattn_debug_set(flags: int, timeout_ns: int = 0) -> None:
 
 def vattn_debug_exp2(x, y, n: Optional[int] = None, stream=None) -> None:
     _check(lib.vattn_debug_exp2(_ptr(x), _ptr(y), x.numel() if n is None else n, _stream(stream)))
-
-
-def vattn_debug_fwd_ctas_per_sm(head_dim: int, fp8: bool = False) -> int:
-    """Resident CTAs per SM of the default forward kernel (the design needs 2)."""
-    n = lib.vattn_debug_fwd_ctas_per_sm(head_dim, 1 if fp8 else 0)
-    _check(min(n, 0))
-    return n
 
 
 def vattn_version() -> str:

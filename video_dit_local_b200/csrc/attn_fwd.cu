@@ -17,6 +17,12 @@
 // straight from TMEM.  The running max is only moved (and O rescaled) when a
 // row's max grows by more than 2^8; otherwise P may reach 2^8, which bf16 and
 // the fp32 accumulators carry without loss of relative precision.
+//
+// FP8 variant (inference): F8 takes Q and K as e4m3 bytes (Q*K^T on the
+// f8f6f4 tensor path, the dequantisation folded into the softmax constant);
+// F8V also takes V as e4m3 bytes and rounds P to e4m3 (packed four to a TMEM
+// column), so P*V is four K = 32 instructions per key block instead of
+// eight; V's scale is applied in the epilogue.
 #include "fwd_common.cuh"
 
 namespace vattn {
@@ -30,27 +36,29 @@ constexpr int WARP_MMA = 10;
 constexpr int NK = 3;  // K ring stages
 constexpr int NV = 2;  // V ring stages
 constexpr float RESCALE_LOG2_THRESHOLD = 8.0f;
-// 32-column chunk (of 4) whose exp2 runs on the FMA pipe (exp2_poly) instead
-// of the MUFU unit; -1 = none.  Measured on B200 at 720p: the MUFU unit is
-// not the limiter of this kernel (removing every ex2 leaves the time
-// unchanged), so the default keeps all exponentials on the MUFU unit.
-#ifndef VATTN_POLY_CHUNK
-#define VATTN_POLY_CHUNK -1
+// Bit b set: the exponentials of the b-th group of 16 columns (of 8) run on
+// the FMA pipe (exp2_poly) instead of the MUFU unit, shortening the MUFU part
+// of a softmax phase at the cost of FMA-pipe instructions.
+#ifndef VATTN_FWD_POLY_MASK
+#define VATTN_FWD_POLY_MASK 0x00
 #endif
-constexpr int POLY_CHUNK = VATTN_POLY_CHUNK;
+constexpr int POLY_MASK = VATTN_FWD_POLY_MASK;
 
-// F8: Q and K are e4m3 bytes (one 128-byte box per row at d = 128), V bf16.
-template <int D, bool F8 = false>
+// F8: Q and K are e4m3 bytes (one 128-byte box per row at d = 128); F8V: V
+// too (P*V on e4m3 operands, P rounded to e4m3).
+template <int D, bool F8 = false, bool F8V = false>
 struct Smem {
   static constexpr int CHUNKS = D / 64;                 // 64-column (128-byte) swizzle boxes
-  static constexpr int BLOCK_BYTES = CHUNKS * 128 * 128; // 128 rows x D bf16
   static constexpr int QK_CHUNKS = F8 ? D / 128 : CHUNKS;   // 128-byte boxes per Q / K row
   static constexpr int QK_ELEMS = F8 ? 128 : 64;            // elements per box row
   static constexpr int QK_BYTES = QK_CHUNKS * 128 * 128;    // 128 rows of Q or K
+  static constexpr int V_CHUNKS = F8V ? D / 128 : CHUNKS;   // 128-byte boxes per V row
+  static constexpr int V_ELEMS = F8V ? 128 : 64;
+  static constexpr int V_BYTES = V_CHUNKS * 128 * 128;      // 128 rows of V
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QK_BYTES;
   static constexpr int OFF_V = OFF_K + NK * QK_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NV * BLOCK_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NV * V_BYTES;
   static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_XCH = OFF_MISC + 16;
@@ -58,11 +66,12 @@ struct Smem {
   static constexpr int ALLOC = TOTAL + 1024;
 };
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool F8V = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  using L = Smem<D, F8>;
+  static_assert(!F8V || (F8 && D == 128), "e4m3 P*V comes with e4m3 Q*K^T at d = 128");
+  using L = Smem<D, F8, F8V>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -199,19 +208,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&v_full[s], L::BLOCK_BYTES);
-        uint8_t* dst = smem + L::OFF_V + s * L::BLOCK_BYTES;
+        mbar_arrive_expect_tx(&v_full[s], L::V_BYTES);
+        uint8_t* dst = smem + L::OFF_V + s * L::V_BYTES;
         for (int u = 0; u < subs; ++u) {
           const int v = j * BN + u * p.G;
           if (p.raster) {
             int x, y, t;
             stream_box(p, st, v, L_total, &x, &y, &t);
-            for (int c = 0; c < L::CHUNKS; ++c)
-              tma_load_5d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * 64, x, y, t, bh);
+            for (int c = 0; c < L::V_CHUNKS; ++c)
+              tma_load_5d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * L::V_ELEMS, x, y, t, bh);
           } else {
             const int row = v < L_total ? stream_row(p, st, v) : p.Nk;
-            for (int c = 0; c < L::CHUNKS; ++c)
-              tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * 64, row, bh);
+            for (int c = 0; c < L::V_CHUNKS; ++c)
+              tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * L::V_ELEMS, row, bh);
           }
         }
         ++issued_v;
@@ -257,14 +266,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int s = j % NV;
         if (!mbar_wait(&v_full[s], (j / NV) & 1, wc)) break;
         tc_fence_after();
-        const uint32_t vb = v_base + s * L::BLOCK_BYTES;
+        const uint32_t vb = v_base + s * L::V_BYTES;
         const uint32_t o_tmem = tmem + 256 + (uint32_t)(w * 128);
         const uint32_t p_tmem = tmem + (uint32_t)(w * 128);
+        if constexpr (F8V) {
+          // e4m3: four K = 32 steps; A = P packed four to a TMEM column; B = V
+          // block (keys x d, one 128-byte row per key), MN-major, SBO = next 8 keys
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // B = V block (keys x d), MN-major: LBO = next 64-column box, SBO = next 8 keys
-          mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, BOX_BYTES, 1024), IDESC_PV,
-                 (j >= 2 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 32; ++kk)
+            mma_ts_e4m3(o_tmem, p_tmem + kk * 8, smem_desc_sw128(vb + kk * 4096, BOX_BYTES, 1024),
+                        idesc_e4m3_f32_bmn(BM, D), (j >= 2 || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // B = V block (keys x d), MN-major: LBO = next 64-column box, SBO = next 8 keys
+            mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, BOX_BYTES, 1024), IDESC_PV,
+                   (j >= 2 || kk > 0) ? 1u : 0u);
+          }
         }
         tc_commit(&v_empty[s]);
         if (j + 2 < nblk) ok = issue_qk(j + 2);
@@ -286,6 +304,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float aq = __int_as_float(p.qk_amax[2 * bh]), ak = __int_as_float(p.qk_amax[2 * bh + 1]);
       c2 *= (aq > 0.f ? aq / 448.f : 1.f) * (ak > 0.f ? ak / 448.f : 1.f);
     }
+    // e4m3 P: the running max moves when a row's max grows by more than 2^2,
+    // so P <= 2^2 and P * 2^6 <= 2^8 < 448 (the largest e4m3); the factor 2^6
+    // (folded into the exponent) keeps small probabilities out of e4m3's
+    // subnormal range and cancels against the row sum, accumulated in the
+    // same units.
+    constexpr float THRESH = F8V ? 2.0f : RESCALE_LOG2_THRESHOLD;
+    constexpr float PSHIFT = F8V ? 6.0f : 0.0f;
     float m_ref = -INFINITY, l_sum = 0.f;
     int qs = w;          // qk_done stage of this group's next block (j % NK) ...
     uint32_t qph = 0;    // ... and its phase parity ((j / NK) & 1)
@@ -326,7 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool need = false;
       if (i == 0) {
         m_ref = mx2;
-      } else if (mx2 > m_ref + RESCALE_LOG2_THRESHOLD) {
+      } else if (mx2 > m_ref + THRESH) {
         need = true;
       }
       float alpha = 1.f;
@@ -335,18 +360,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         m_ref = mx2;
         l_sum *= alpha;
       }
-      // P = 2^(S*scale*log2(e) - m) two lanes at a time (packed fp32x2)
-      const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(-m_ref, -m_ref);
+      // P = 2^(S*scale*log2(e) - m (+ PSHIFT)) two lanes at a time (packed fp32x2)
+      const float2 c2x2 = make_float2(c2, c2), negm2 = make_float2(PSHIFT - m_ref, PSHIFT - m_ref);
       float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pk[16];
+        uint32_t p8[8];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const float2 x = ffma2(make_float2(__uint_as_float(sr[q4][2 * c]), __uint_as_float(sr[q4][2 * c + 1])),
                                  c2x2, negm2);
           float2 pp;
-          if (q4 == POLY_CHUNK) {  // FMA-pipe exponentials for this chunk (see POLY_CHUNK)
+          if ((POLY_MASK >> (q4 * 2 + (c >> 3))) & 1) {  // FMA-pipe exponentials for this group of 16
             pp.x = exp2_poly(x.x);
             pp.y = exp2_poly(x.y);
           } else {
@@ -354,9 +380,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pp.y = ex2(x.y);
           }
           s2[c & 1] = fadd2(s2[c & 1], pp);
-          pk[c] = pack_bf16(pp.x, pp.y);
+          if constexpr (F8V) {
+            const uint32_t h = pack_e4m3x2(pp.x, pp.y);
+            p8[c >> 1] = (c & 1) ? (p8[c >> 1] | (h << 16)) : h;
+          } else {
+            pk[c] = pack_bf16(pp.x, pp.y);
+          }
         }
-        tmem_st16(tS + q4 * 16, pk);
+        if constexpr (F8V)
+          tmem_st8(tS + q4 * 8, p8);
+        else
+          tmem_st16(tS + q4 * 16, pk);
       }
       l_sum += (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
       if (__any_sync(0xffffffffu, need)) {
@@ -388,7 +422,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float m = fmaxf(m_ref, other.x);
       const float a_self = ex2(m_ref - m), a_other = ex2(other.x - m);
       const float l = l_sum * a_self + other.y * a_other;
-      const float inv_l = 1.f / l;
+      float inv_l = 1.f / l;
+      if constexpr (F8V) {  // O = P V with V = bytes(V) * absmax_V / 448
+        const float av = __int_as_float(p.v_amax[bh]);
+        inv_l *= av > 0.f ? av / 448.f : 1.f;
+      }
       const float a0 = (w == 0 ? a_self : a_other) * inv_l;
       const float a1 = (w == 0 ? a_other : a_self) * inv_l;
       const bool have1 = nblk >= 2;
@@ -404,7 +442,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (row_ok && !dcheck(out_row_ok(p, bh, grow), p.ctl.err_word)) row_ok = false;
       // hierarchical merge: one softmax over the fine keys (O_f, LSE_f given)
       // and this kernel's coarse keys, in log2 units
-      float wf = 0.f, wc = 1.f, lse2_out = m + __log2f(l);
+      float wf = 0.f, wc = 1.f, lse2_out = m - PSHIFT + __log2f(l);
       if (p.merge_o && row_ok) {
         const float lf2 = p.merge_lse[grow] * 1.4426950408889634f;
         const float mm = fmaxf(lf2, lse2_out);
@@ -481,8 +519,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace fwd
 
 template <int D, bool F8, bool F8V>
-cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fwd::Params& p,
-                        dim3 grid, cudaStream_t st);
+static cudaError_t launch_fwd1(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const fwd::Params& p, dim3 grid, cudaStream_t st) {
+  using namespace fwd;
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8, F8V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Smem<D, F8, F8V>::ALLOC);
+  if (e != cudaSuccess) return e;
+  attn_fwd_kernel<D, F8, F8V><<<grid, NTHREADS, Smem<D, F8, F8V>::ALLOC, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
 
 template <int D, bool F8 = false>
 static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st) {
@@ -536,40 +581,27 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   CUtensorMap tq, tk, tv;
   const char* err = nullptr;
   bool maps_ok;
+  const bool f8v = F8 && a.v_amax != nullptr;  // e4m3 P*V: V bytes
   if (p.raster) {  // 5-D raster maps: boxes of whole t-slices of one tile
     const int slice = g.th * g.tw;
     if (F8 || mode != FWD_STA || a.kgeom || BM % slice || p.G % slice) return cudaErrorInvalidValue;
     maps_ok = make_tmap_raster(&tq, a.q, D, g, bh, BM / slice, &err) &&
               make_tmap_raster(&tk, a.k, D, g, bh, p.G / slice, &err) &&
               make_tmap_raster(&tv, a.v, D, g, bh, p.G / slice, &err);
-    if (!maps_ok) return cudaErrorInvalidValue;
-    if (!(p.ctl.debug_flags & VATTN_DEBUG_ONE_CTA_FWD))
-      return launch_fwd2<D, F8, false>(tq, tk, tv, p, dim3(qblocks, (unsigned)bh), st);
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Smem<D, F8>::ALLOC);
-    if (e != cudaSuccess) return e;
-    attn_fwd_kernel<D, F8><<<dim3(qblocks, (unsigned)bh), NTHREADS, Smem<D, F8>::ALLOC, st>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+  } else if constexpr (F8) {
+    maps_ok = make_tmap_rows_u8(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows_u8(&tk, a.k, D, p.Nk, bh, p.G, &err) &&
+              (f8v ? make_tmap_rows_u8(&tv, a.v, D, p.Nk, bh, p.G, &err)
+                   : make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err));
+  } else {
+    maps_ok = make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err) &&
+              make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err);
   }
-  if constexpr (F8)
-    maps_ok = make_tmap_rows_u8(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows_u8(&tk, a.k, D, p.Nk, bh, p.G, &err);
-  else
-    maps_ok = make_tmap_rows(&tq, a.q, D, g.N, bh, BM, &err) && make_tmap_rows(&tk, a.k, D, p.Nk, bh, p.G, &err);
+  if (!maps_ok) return cudaErrorInvalidValue;
+  const dim3 grid(qblocks, (unsigned)bh);
   if constexpr (F8) {
-    if (a.v_amax) {  // e4m3 P*V: V bytes, only the two-CTA kernel has this mode
-      if (!maps_ok || !make_tmap_rows_u8(&tv, a.v, D, p.Nk, bh, p.G, &err)) return cudaErrorInvalidValue;
-      return launch_fwd2<D, true, true>(tq, tk, tv, p, dim3(qblocks, (unsigned)bh), st);
-    }
+    if (f8v) return launch_fwd1<D, true, true>(tq, tk, tv, p, grid, st);
   }
-  if (!maps_ok || !make_tmap_rows(&tv, a.v, D, p.Nk, bh, p.G, &err)) return cudaErrorInvalidValue;
-  if (!(p.ctl.debug_flags & VATTN_DEBUG_ONE_CTA_FWD))
-    return launch_fwd2<D, F8, false>(tq, tk, tv, p, dim3(qblocks, (unsigned)bh), st);
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Smem<D, F8>::ALLOC);
-  if (e != cudaSuccess) return e;
-  dim3 grid(qblocks, (unsigned)bh);
-  attn_fwd_kernel<D, F8><<<grid, NTHREADS, Smem<D, F8>::ALLOC, st>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  return launch_fwd1<D, F8, false>(tq, tk, tv, p, grid, st);
 }
 
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {

@@ -1,7 +1,6 @@
-// Definitions shared by the two forward kernels (attn_fwd.cu: one CTA per SM
-// with two softmax groups; attn_fwd_2cta.cu: two CTAs per SM, one softmax
-// group each): launch parameters, the key stream of a query block, the 5-D
-// raster TMA load and the e4m3 tensor-core instruction.
+// Definitions of the forward kernel (attn_fwd.cu): launch parameters, the key
+// stream of a query block, the 5-D raster TMA load, the e4m3 tensor-core
+// instructions and the debug-build bounds checks.
 #pragma once
 
 #include "common.cuh"
@@ -30,7 +29,7 @@ struct Params {
   const __nv_bfloat16* merge_o;  // hierarchical: fine-key O and LSE to merge with (NULL = none)
   const float* merge_lse;
   const int* qk_amax;            // e4m3 Q*K^T: absmax bits of Q and K per batch*head
-  const int* v_amax;             // e4m3 P*V (two-CTA kernel): absmax bits of V per batch*head
+  const int* v_amax;             // e4m3 P*V: absmax bits of V per batch*head
   // raster (STA only): Q, K, V, O and LSE in raster token order.  The tensor
   // maps are 5-D (d, W, H, T, batch*head); a load is a box of whole t-slices
   // of one tile, which lands in shared memory in the tile-major row order.

@@ -543,16 +543,6 @@ int vattn_debug_set(int flags, int64_t timeout_ns) {
   return ok();
 }
 
-int vattn_debug_fwd_ctas_per_sm(int head_dim, int fp8) {
-  if (!(head_dim == 64 || head_dim == 128) || (fp8 && head_dim != 128))
-    return fail(VATTN_ERR_UNSUPPORTED, "vattn_debug_fwd_ctas_per_sm: head_dim %d%s unsupported", head_dim,
-                fp8 ? " with fp8" : "");
-  const int n = fwd2_ctas_per_sm(head_dim, fp8 != 0);
-  if (n < 0) return fail(VATTN_ERR_CUDA, "vattn_debug_fwd_ctas_per_sm: occupancy query failed");
-  ok();
-  return n;
-}
-
 int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream) {
   if (n < 0) return fail(VATTN_ERR_INVALID_ARG, "n must be >= 0");
   if (n == 0) return ok();

@@ -104,8 +104,6 @@ struct FwdArgs {
   bool raster;
 };
 cudaError_t launch_attn_fwd(const DevGeom& g, FwdMode mode, const FwdArgs& a, cudaStream_t st);
-// Resident CTAs per SM of the two-CTA forward kernel (-1 on error).
-int fwd2_ctas_per_sm(int d, bool f8);
 cudaError_t launch_exp2_poly(const float* x, float* y, long long n, cudaStream_t st);
 
 // -- attention backward (attn_bwd.cu) --
