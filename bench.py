@@ -202,6 +202,70 @@ def run_train_only(args, rank, world, local_rank):
                                    "window 3x3x3, pool 1x4x4"}, "train": res}
 
 
+def run_fp8_only(args, rank, world, local_rank):
+    """Profiling mode: the FP8 sliding-tile forward (e4m3 Q*K^T and P*V, the
+    quantisation included) of the 720p workload alone (optionally with fewer
+    heads), timed with CUDA events."""
+    import dataclasses
+
+    import torch
+
+    import video_dit_local_b200 as V
+    from synth import inputs as S
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = S.WORKLOADS["720p"]
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads)
+    geom = _geom(V, w)
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 800 + i) for i in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty(shape[:3], dtype=torch.float32, device=dev)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_STA_FWD_FP8, geom), dtype=torch.uint8, device=dev)
+    fl, _ = _flops_fwd(w)
+    ms = _time_ms(lambda: V.vattn_sta_fwd_fp8(geom, q, k, v, 1 / math.sqrt(w.head_dim), o, lse, ws), args.steps,
+                  warm=args.warmup)
+    return {"metric": METRIC, "value": round(fl / ms / 1e9, 1), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3", "data": "synthetic (seeded torch N(0,1))",
+            "config": {"workload": f"720p sliding-tile fwd, FP8: B1 h{w.heads} d128, grid 30x48x80, tile 6x8x8, "
+                                   "window 3x3x3"}, "status": V.vattn_get_status()}
+
+
+def run_dual_only(args, rank, world, local_rank):
+    """Profiling mode: the inference dual forward (pool, sliding-tile branch,
+    global branch with the blend) of the 1080p or 4K workload alone (optionally
+    with fewer heads), timed with CUDA events."""
+    import dataclasses
+
+    import torch
+
+    import video_dit_local_b200 as V
+    from synth import inputs as S
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = S.WORKLOADS[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads)
+    geom = _geom(V, w)
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 100 * w.seed + i) for i in range(3))
+    gvec = torch.rand(w.heads, device=dev)
+    o = torch.empty_like(q)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_DUAL_FWD, geom), dtype=torch.uint8, device=dev)
+    fl, fg = _flops_fwd(w)
+    ms = _time_ms(lambda: V.vattn_dual_fwd(geom, q, k, v, gvec, 1 / math.sqrt(w.head_dim), o, workspace=ws),
+                  args.steps, warm=args.warmup)
+    T, H, W = w.grid
+    return {"metric": METRIC, "value": round((fl + fg) / ms / 1e9, 1), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch N(0,1))",
+            "config": {"workload": f"{w.name} dual fwd: B{w.batch} h{w.heads} d{w.head_dim}, grid {T}x{H}x{W}, "
+                                   f"tile {'x'.join(map(str, w.tile))}, window {'x'.join(map(str, w.window))}, "
+                                   f"pool {'x'.join(map(str, w.pool))}"}, "status": V.vattn_get_status()}
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -787,8 +851,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-chunk", type=int, default=1, help="batch*head slices per host-copy chunk (e2e)")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: fewer heads than the workload")
-    ap.add_argument("--workload", choices=["720p", "train"], default="720p",
-                    help="720p: the benchmark line; train: profiling of the training step alone")
+    ap.add_argument("--workload", choices=["720p", "train", "fp8", "1080p", "4k"], default="720p",
+                    help="720p: the benchmark line; train, fp8, 1080p, 4k: profiling of the training step, the FP8 "
+                         "forward or the 1080p / 4K dual forward alone")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -811,6 +876,10 @@ def main():
     try:
         if args.workload == "train":
             result = run_train_only(args, rank, world, local_rank)
+        elif args.workload == "fp8":
+            result = run_fp8_only(args, rank, world, local_rank)
+        elif args.workload in ("1080p", "4k"):
+            result = run_dual_only(args, rank, world, local_rank)
         else:
             result = run_ours(args, rank, world, local_rank)
         if rank == 0:

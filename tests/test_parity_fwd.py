@@ -177,6 +177,12 @@ def test_sta_fwd_720p_sampled(V):
     ((6, 16, 32), (6, 8, 8), (1, 3, 3), 64, 2, 1),       # tile 384, d = 64, batch 2
     ((4, 8, 16), (2, 4, 4), (1, 1, 1), 128, 1, 3),       # window of one tile
     ((2, 8, 8), (2, 4, 4), (3, 5, 7), 128, 1, 1),        # window wider than the grid in every dim
+    # tiles of 192 and 64 rows: adjacent tiles along w share query blocks, the
+    # straddling block over windows that coincide (edges) or start a tile apart
+    ((3, 16, 40), (3, 8, 8), (1, 3, 3), 128, 1, 2),      # 5 tiles along w: two pairs and a tile of its own
+    ((2, 16, 48), (1, 8, 8), (1, 1, 3), 64, 1, 2),       # tile 64: every query block straddles two tiles
+    ((3, 8, 64), (3, 8, 8), (1, 1, 5), 128, 1, 1),       # window of 5 along w: interior pairs a tile apart
+    ((3, 8, 48), (3, 8, 8), (1, 2, 2), 128, 1, 1),       # even window
 ])
 def test_sta_fwd_small_full(V, grid, tile, window, d, batch, heads):
     w = S.small_workload("sta", 11, batch, heads, d, grid, tile, window, (1, 1, 1))
@@ -241,6 +247,8 @@ def _check_dual(w, out, check, tiles):
     ((4, 8, 8), (2, 4, 4), (1, 2, 2), (1, 2, 2), 64, 1, 2),
     ((3, 20, 24), (3, 4, 4), (1, 3, 3), (1, 2, 2), 128, 2, 3),    # N, N_p not multiples of 128
     ((3, 8, 8), (1, 4, 4), (3, 1, 1), (1, 1, 1), 128, 1, 2),      # pool 1: global = full attention
+    ((3, 24, 16), (3, 8, 8), (1, 3, 1), (1, 2, 2), 128, 1, 2),    # 192-token tiles: 5 local, 3 pooled key blocks
+    ((3, 16, 40), (3, 8, 8), (1, 3, 3), (1, 2, 2), 128, 1, 2),    # 192-token tiles paired along w
 ])
 def test_dual_fwd_small_full(V, grid, tile, window, pool, d, batch, heads):
     w = S.small_workload("dual", 13, batch, heads, d, grid, tile, window, pool)

@@ -66,7 +66,9 @@ struct Smem {
   static constexpr int ALLOC = TOTAL + 1024;
 };
 
-template <int D, bool F8 = false, bool F8V = false>
+// PAIR: query blocks of adjacent tiles paired along w (tile volumes an odd
+// multiple of BM/2); see QueryBlock.
+template <int D, bool F8 = false, bool F8V = false, bool PAIR = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -101,19 +103,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   wc.timeout_ns = p.ctl.timeout_ns;
   wc.err_word = p.ctl.err_word;
 
-  // query block -> rows
-  int q_tile, q_row0, q_valid, sub = 0;
-  if (p.mode == FWD_STA) {
-    q_tile = qblk / p.q_blocks_per_tile;
-    sub = qblk - q_tile * p.q_blocks_per_tile;
-    q_row0 = q_tile * p.g.s + sub * BM;
-    q_valid = min(BM, p.g.s - sub * BM);
-  } else {
-    q_tile = 0;
-    q_row0 = qblk * BM;
-    q_valid = min(BM, p.g.N - q_row0);
-  }
-  const Stream st = make_stream(p, q_tile);
+  // query block -> rows and key stream
+  const QueryBlock qb = query_block<PAIR>(p, qblk);
+  const int q_tile = qb.tile, q_row0 = qb.row0, q_valid = qb.valid, sub = qb.sub;
+  const Stream st = make_block_stream<PAIR>(p, qb);
   const int L_total = st.length();
   const int nblk = (L_total + BN - 1) / BN;
 
@@ -339,6 +332,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int c = 0; c < 32; ++c)
             if (q4 * 32 + c >= valid) sr[q4][c] = __float_as_uint(-INFINITY);
       }
+      if (PAIR && st.rot) {
+        // straddling block over windows one tile apart: the first tile's rows
+        // (quads 0, 1) see run tiles 0 .. ew-1 (w0+1 .. w0+ew), the second's
+        // (quads 2, 3) run tiles 0 .. ew-2 and ew (w0+1 .. w0+ew-1, then w0);
+        // 32-column groups never cross a tile (s is a multiple of 64)
+        const int x0 = (quad >> 1 ? st.ew : st.ew - 1) * p.g.s;  // excluded run offsets [x0, x0 + s)
+        const int o = (j * BN) % st.run_len;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          int oq = o + q4 * 32;
+          if (oq >= st.run_len) oq -= st.run_len;
+          if ((unsigned)(oq - x0) < (unsigned)p.g.s) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) sr[q4][c] = __float_as_uint(-INFINITY);
+          }
+        }
+      }
       // row max: four independent chains of three-input max
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -518,14 +528,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 }  // namespace fwd
 
-template <int D, bool F8, bool F8V>
+template <int D, bool F8, bool F8V, bool PAIR>
 static cudaError_t launch_fwd1(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                const fwd::Params& p, dim3 grid, cudaStream_t st) {
   using namespace fwd;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F8, F8V>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Smem<D, F8, F8V>::ALLOC);
+  auto kernel = attn_fwd_kernel<D, F8, F8V, PAIR>;
+  constexpr int smem = Smem<D, F8, F8V>::ALLOC;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  attn_fwd_kernel<D, F8, F8V><<<grid, NTHREADS, Smem<D, F8, F8V>::ALLOC, st>>>(tq, tk, tv, p);
+  kernel<<<grid, NTHREADS, smem, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -552,11 +563,16 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   p.v_amax = a.v_amax;
   p.raster = a.raster ? 1 : 0;
   int qblocks;
+  bool pair = false;
   if (mode == FWD_STA) {
     int G = 1;
     while (G < BN && g.s % (G * 2) == 0) G *= 2;
     p.G = G;
     p.q_blocks_per_tile = (g.s + BM - 1) / BM;
+    p.pair_k = 0;
+    p.pair_nw = 1;
+    p.pair_np = 0;
+    p.pair_bpr = p.q_blocks_per_tile;
     p.Nk = g.N;
     if (a.kgeom) {  // hierarchical: coarse tiles of the medium-pooled grid (same tile volume)
       p.kNt = a.kgeom->Nt;
@@ -570,9 +586,23 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
       p.merge_lse = a.merge_lse;
     }
     qblocks = g.n_tiles * p.q_blocks_per_tile;
+    // tiles of an odd multiple of BM/2 rows: pair adjacent tiles along w so
+    // that no query block is half empty (tile-major rows; sliding windows of
+    // at least two tiles along w, so a straddling block's first key tile is in
+    // both windows)
+    if (!p.raster && g.s % BM == BM / 2 && g.wmode == WIN_SLIDING && win_extent(g.ww, p.kNw) >= 2 && g.Nw >= 2) {
+      p.pair_k = g.s / BM;
+      p.pair_nw = g.Nw;
+      p.pair_np = g.Nw / 2;
+      p.pair_bpr = p.pair_np * (2 * p.pair_k + 1) + (g.Nw % 2) * (p.pair_k + 1);
+      qblocks = g.Nt * g.Nh * p.pair_bpr;
+      pair = true;
+    }
   } else {
     p.G = BN;
     p.q_blocks_per_tile = 1;
+    p.pair_k = p.pair_np = 0;
+    p.pair_nw = p.pair_bpr = 1;
     p.Nk = g.Np;
     qblocks = (g.N + BM - 1) / BM;
   }
@@ -599,9 +629,13 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
   if (!maps_ok) return cudaErrorInvalidValue;
   const dim3 grid(qblocks, (unsigned)bh);
   if constexpr (F8) {
-    if (f8v) return launch_fwd1<D, true, true>(tq, tk, tv, p, grid, st);
+    if (!f8v) return cudaErrorInvalidValue;  // the FP8 forward takes e4m3 V as well
+    if (pair) return launch_fwd1<D, true, true, true>(tq, tk, tv, p, grid, st);
+    return launch_fwd1<D, true, true, false>(tq, tk, tv, p, grid, st);
+  } else {
+    if (pair) return launch_fwd1<D, false, false, true>(tq, tk, tv, p, grid, st);
+    return launch_fwd1<D, false, false, false>(tq, tk, tv, p, grid, st);
   }
-  return launch_fwd1<D, F8, false>(tq, tk, tv, p, grid, st);
 }
 
 __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {

@@ -16,11 +16,20 @@ struct Params {
   int mode;
   int G;             // rows per TMA sub-box of a key block (divides the tile volume)
   int q_blocks_per_tile;
+  // STA query blocks.  With a tile volume an odd multiple of BM/2 (e.g. 192
+  // rows), adjacent tiles of a tile row (w = 2i, 2i+1) share their query
+  // blocks: pair_k = s / BM whole blocks of each and one block straddling the
+  // two; an odd last tile of the row takes pair_k + 1 blocks of its own.  Then
+  // pair_nw = Nw tiles and pair_np = Nw / 2 pairs per tile row, pair_bpr query
+  // blocks per tile row.  Unpaired: pair_nw = 1, pair_np = 0 and pair_bpr =
+  // q_blocks_per_tile (each tile a row of its own).
+  int pair_k, pair_nw, pair_np, pair_bpr;
   int Nk;            // key rows per batch*head in the K/V tensors
   float scale_log2;  // scale * log2(e)
   __nv_bfloat16* o;
   float* lse;
   const __nv_bfloat16* o_local;
+  __nv_bfloat16* o_local_out;    // fused dual forward: where the local pass leaves O_local (read back by the blend)
   const float* gvec;
   __nv_bfloat16* blend_out;
   // key-side tile grid and coarse factor (STA): the sliding tile has the query
@@ -76,6 +85,11 @@ __device__ __forceinline__ void mma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, ui
 // Key stream of one CTA: `runs` runs of `run_len` contiguous rows.
 struct Stream {
   int runs, run_len, eh, t0, h0, w0;
+  int ew;   // window tiles along w (sliding tile)
+  // straddling query block whose two tiles' windows start one tile apart: each
+  // run holds the union, ew + 1 tiles, streamed from the second (w0 + 1, in
+  // both windows) to w0 + ew and then w0 (only in the first tile's window)
+  int rot;
   __device__ __forceinline__ int length() const { return runs * run_len; }
 };
 
@@ -90,11 +104,74 @@ __device__ __forceinline__ Stream make_stream(const Params& p, int q_tile) {
     tile_range(aw / p.cfw, g.ww, p.kNw, g.wmode, &s.w0, &ew);
     s.runs = et * s.eh;
     s.run_len = ew * g.s;
+    s.ew = ew;
   } else {
     s.runs = 1;
     s.run_len = p.Nk;
     s.eh = 1;
     s.t0 = s.h0 = s.w0 = 0;
+    s.ew = 1;
+  }
+  s.rot = 0;
+  return s;
+}
+
+// Query block -> its rows and the key stream it attends to.  Sliding tile:
+// the block's tile (or, for a straddling block, the union of the windows of
+// tiles a and a + 1, which share t and h and whose windows along w start at
+// most one tile apart); global: every pooled key.
+struct QueryBlock {
+  int tile;      // anchor tile of the key stream (STA)
+  int row0;      // first row (tile-major)
+  int valid;     // rows of the block that exist
+  int sub;       // block within its tile (raster loads)
+  int straddle;  // rows [0, BM/2) in tile `tile`, [BM/2, BM) in tile `tile` + 1
+};
+
+template <bool PAIR>
+__device__ __forceinline__ QueryBlock query_block(const Params& p, int qblk) {
+  QueryBlock b;
+  const DevGeom& g = p.g;
+  if (!PAIR && p.mode == FWD_STA) {
+    b.tile = qblk / p.q_blocks_per_tile;
+    b.sub = qblk - b.tile * p.q_blocks_per_tile;
+    b.row0 = b.tile * g.s + b.sub * BM;
+    b.valid = min(BM, g.s - b.sub * BM);
+    b.straddle = 0;
+  } else if (p.mode == FWD_STA) {
+    // tile row r (or, unpaired, tile r), block i of it; pair pi (npair: the
+    // row's odd last tile), block sb of the pair
+    const int r = qblk / p.pair_bpr, i = qblk - r * p.pair_bpr;
+    const int span = 2 * p.pair_k + 1;
+    const int pi = min(i / span, p.pair_np);
+    const int a = r * p.pair_nw + 2 * pi, sb = i - pi * span;
+    const bool in_pair = pi < p.pair_np;
+    b.row0 = a * g.s + sb * BM;
+    b.valid = min(BM, (in_pair ? 2 * g.s : g.s) - sb * BM);
+    b.tile = a + (in_pair && sb > p.pair_k ? 1 : 0);
+    b.straddle = in_pair && sb == p.pair_k;
+    b.sub = sb;
+  } else {
+    b.tile = 0;
+    b.row0 = qblk * BM;
+    b.valid = min(BM, g.N - b.row0);
+    b.sub = 0;
+    b.straddle = 0;
+  }
+  return b;
+}
+
+template <bool PAIR>
+__device__ __forceinline__ Stream make_block_stream(const Params& p, const QueryBlock& b) {
+  Stream s = make_stream(p, b.tile);
+  if (PAIR && b.straddle) {
+    const DevGeom& g = p.g;
+    int w0b, ewb;
+    tile_range((b.tile % g.Nw + 1) / p.cfw, g.ww, p.kNw, g.wmode, &w0b, &ewb);
+    if (w0b != s.w0) {  // one tile apart (sliding windows of equal extent)
+      s.rot = 1;
+      s.run_len += g.s;
+    }
   }
   return s;
 }
@@ -104,6 +181,11 @@ __device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int 
   if (p.mode != FWD_STA) return v;
   const int r = v / s.run_len, o = v - r * s.run_len;
   const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
+  if (s.rot) {  // run order w0 + 1, ..., w0 + ew, w0
+    const int ti = o / p.g.s, lo = o - ti * p.g.s;
+    const int wt = ti < s.ew ? ti + 1 : 0;
+    return ((kt * p.kNh + kh) * p.kNw + s.w0 + wt) * p.g.s + lo;
+  }
   return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + o;
 }
 
