@@ -66,6 +66,7 @@ def _run_dual(V, w, check):
     ((3, 20, 24), (3, 4, 4), (1, 3, 3), (1, 2, 2), 128, 2, 3),    # ragged N, N_p; tile 48
     ((6, 16, 24), (3, 8, 8), (1, 1, 3), (1, 4, 4), 128, 1, 2),     # tile 192: half-empty second block
     ((6, 16, 32), (6, 8, 8), (1, 3, 3), (3, 4, 4), 64, 1, 1),      # tile 384, temporal pooling
+    ((3, 16, 40), (3, 8, 8), (1, 3, 3), (1, 2, 2), 128, 1, 2),     # tile 192, 5 along w: paired dQ query blocks
 ])
 def test_dual_bwd_small_full(V, grid, tile, window, pool, d, batch, heads):
     w = S.small_workload("dbwd", 17, batch, heads, d, grid, tile, window, pool)
@@ -84,6 +85,8 @@ def test_dual_bwd_small_full(V, grid, tile, window, pool, d, batch, heads):
 @pytest.mark.parametrize("grid,tile,window,d", [
     ((4, 8, 8), (2, 4, 4), (1, 2, 2), 64),
     ((6, 16, 24), (3, 8, 8), (3, 1, 3), 128),
+    ((2, 16, 48), (1, 8, 8), (1, 1, 3), 64),      # tile 64: every dQ query block straddles two tiles
+    ((3, 8, 64), (3, 8, 8), (1, 1, 5), 128),      # window of 5 along w: interior pairs a tile apart
 ])
 def test_sta_bwd_small_full(V, grid, tile, window, d):
     import torch

@@ -172,7 +172,7 @@ CASES = [
     ((6, 16, 24), (3, 8, 8), (1, 3, 3), 1, 2),     # tile 192: a ragged second query block
     ((6, 16, 32), (6, 8, 8), (1, 3, 3), 2, 1),     # tile 384, batch 2
     ((4, 8, 16), (2, 4, 4), (1, 1, 3), 1, 3),      # tile 32
-    ((3, 16, 40), (3, 8, 8), (1, 3, 3), 1, 2),     # tile 192, adjacent tiles along w sharing query blocks
+    ((3, 16, 40), (3, 8, 8), (1, 3, 3), 1, 2),     # tile 192, 5 tiles along w, interior windows a tile apart
 ]
 
 

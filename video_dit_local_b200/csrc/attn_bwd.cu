@@ -474,7 +474,7 @@ struct DqSmem {
   static constexpr int ALLOC = TOTAL + 1024;
 };
 
-template <int D>
+template <int D, bool PAIR = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -507,16 +507,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const bool glob = p.mode == DQ_GLOBAL;
   int q_row0, q_valid, q_tile = 0;
+  bool straddle = false;
   if (glob) {
     q_row0 = blockIdx.x * 128;
     q_valid = min(128, g.N - q_row0);
+  } else if (PAIR) {  // w-adjacent tiles share their query blocks (PairPlan)
+    const QueryBlock qb = paired_query_block(g, p.pair, blockIdx.x);
+    q_tile = qb.tile;
+    q_row0 = qb.row0;
+    q_valid = qb.valid;
+    straddle = qb.straddle;
   } else {
     q_tile = blockIdx.x / p.q_blocks_per_tile;
     const int sub = blockIdx.x - q_tile * p.q_blocks_per_tile;
     q_row0 = q_tile * g.s + sub * 128;
     q_valid = min(128, g.s - sub * 128);
   }
-  const RowStream ks = glob ? flat_stream(g.Np) : window_stream(g, p.gk, p.cft, p.cfh, p.cfw, q_tile);
+  RowStream ks = glob ? flat_stream(g.Np) : window_stream(g, p.gk, p.cft, p.cfh, p.cfw, q_tile);
+  if (PAIR && straddle && straddle_shift(g, p.gk.Nw, p.cfw, q_tile) != 0) {
+    ks.rot = 1;
+    ks.run_len += p.gk.s;
+  }
   const int Lk = ks.length();
   const int nblk = (Lk + DQ_BN - 1) / DQ_BN;
 
@@ -646,8 +657,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       const int valid = Lk - j * DQ_BN;
       const bool full_blk = valid >= DQ_BN;
+      // straddling block over windows one tile apart (PAIR): 32-column chunks
+      // of the key tile outside this warp's rows' window get dS = 0 (a chunk
+      // never crosses a tile: s is a multiple of 64)
+      unsigned drop = 0;
+      if (PAIR && ks.rot) {
+        const int x0 = straddle_excluded_start(p.gk.s, ks.ew, quad >> 1);
+        int oq = (j * DQ_BN) % ks.run_len;
+#pragma unroll
+        for (int hh = 0; hh < DQ_BN / 32; ++hh) {
+          if ((unsigned)(oq - x0) < (unsigned)p.gk.s) drop |= 1u << hh;
+          oq += 32;
+          if (oq >= ks.run_len) oq -= ks.run_len;
+        }
+      }
 #pragma unroll
       for (int hh = 0; hh < DQ_BN / 32; ++hh) {
+        const bool dropped = (drop >> hh) & 1u;
         // one 32-column chunk at a time: S, dP and the packed dS stay in registers
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + hh * 32, sv);
@@ -664,6 +690,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (cc >= valid) o2.x = 0.f;
             if (cc + 1 >= valid) o2.y = 0.f;
           }
+          if (dropped) o2 = make_float2(0.f, 0.f);
           dk[c] = pack_bf16(o2.x, o2.y);
         }
         tmem_st16(tP + hh * 16, dk);
@@ -812,6 +839,10 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   while (G0 > 8 && (DQ_BN % G0 != 0 || g.s % G0 != 0)) G0 -= 8;
   p.G0 = G0;
   p.q_blocks_per_tile = (g.s + 127) / 128;
+  // local and hierarchical passes: w-adjacent tiles of an odd multiple of 64
+  // rows share their query blocks (PairPlan), as in the forward
+  p.pair = make_pair_plan(g, p.gk.Nw, !global);
+  const bool pair = p.pair.np > 0;
   p.scale = a.scale;
   p.c2 = a.scale * LOG2E;
   p.nlse2 = global ? a.nlse2_g : a.nlse2_l;
@@ -822,7 +853,7 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   p.dq = (__nv_bfloat16*)a.dq;
   p.ctl = current_ctl();
   const long long bh = (long long)g.B * g.heads;
-  const int blocks = global ? (g.N + 127) / 128 : g.n_tiles * p.q_blocks_per_tile;
+  const int blocks = global ? (g.N + 127) / 128 : (int)pair_plan_blocks(g, p.pair);
   if (bh == 0 || blocks == 0) return cudaSuccess;
   CUtensorMap tq, tdo, tk, tv;
   const char* err = nullptr;
@@ -833,9 +864,10 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   if (!make_tmap_rows(&tq, a.q, D, g.N, bh, 128, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, 128, &err) ||
       !make_tmap_rows(&tk, kk, D, nk, bh, G, &err) || !make_tmap_rows(&tv, vv, D, nk, bh, G, &err))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_smem(dq_kernel<D>, DqSmem<D>::ALLOC);
+  auto kernel = pair ? dq_kernel<D, true> : dq_kernel<D, false>;
+  cudaError_t e = set_smem(kernel, DqSmem<D>::ALLOC);
   if (e != cudaSuccess) return e;
-  dq_kernel<D><<<dim3(blocks, (unsigned)bh), NTHREADS, DqSmem<D>::ALLOC, st>>>(tq, tdo, tk, tv, p);
+  kernel<<<dim3(blocks, (unsigned)bh), NTHREADS, DqSmem<D>::ALLOC, st>>>(tq, tdo, tk, tv, p);
   return cudaGetLastError();
 }
 

@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == WARP_QK_LOAD) {
     if (lane == 0) {
       int issued_k = 0;
+      KeyCursor kc = key_cursor(p, st, L_total);  // e4m3 instance (see KeyCursor)
+      const int tiles_per_run = p.mode == FWD_STA ? st.run_len / p.g.s : 1;
       if (!dcheck(query_block_ok(p, q_row0, q_valid), p.ctl.err_word)) *abort_flag = 1;
       if (!(p.ctl.debug_flags & 1) && !*abort_flag) {
         mbar_arrive_expect_tx(q_full, L::QK_BYTES);
@@ -173,13 +175,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* dst = smem + L::OFF_K + s * L::QK_BYTES;
         for (int u = 0; u < subs; ++u) {
           const int v = j * BN + u * p.G;
-          if (p.raster) {
+          if (!F8 && p.raster) {
             int x, y, t;
             stream_box(p, st, v, L_total, &x, &y, &t);
             for (int c = 0; c < L::QK_CHUNKS; ++c)
               tma_load_5d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * L::QK_ELEMS, x, y, t, bh);
           } else {
-            const int row = v < L_total ? stream_row(p, st, v) : p.Nk;  // past the end: zero fill
+            int row;  // past the end: row Nk, zero fill
+            if constexpr (F8) {
+              row = cursor_row(p, st, kc);
+              cursor_next(p, st, kc, tiles_per_run);
+            } else {
+              row = v < L_total ? stream_row(p, st, v) : p.Nk;
+            }
             for (int c = 0; c < L::QK_CHUNKS; ++c)
               tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_k, &k_full[s], c * L::QK_ELEMS, row, bh);
           }
@@ -194,6 +202,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == WARP_V_LOAD) {
     if (lane == 0) {
       int issued_v = 0;
+      KeyCursor vc = key_cursor(p, st, L_total);
+      const int tiles_per_run = p.mode == FWD_STA ? st.run_len / p.g.s : 1;
       for (int j = 0; j < nblk; ++j) {
         const int s = j % NV, r = j / NV;
         if (!mbar_wait(&v_empty[s], (r & 1) ^ 1, wc)) break;
@@ -205,13 +215,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* dst = smem + L::OFF_V + s * L::V_BYTES;
         for (int u = 0; u < subs; ++u) {
           const int v = j * BN + u * p.G;
-          if (p.raster) {
+          if (!F8 && p.raster) {
             int x, y, t;
             stream_box(p, st, v, L_total, &x, &y, &t);
             for (int c = 0; c < L::V_CHUNKS; ++c)
               tma_load_5d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * L::V_ELEMS, x, y, t, bh);
           } else {
-            const int row = v < L_total ? stream_row(p, st, v) : p.Nk;
+            int row;
+            if constexpr (F8) {
+              row = cursor_row(p, st, vc);
+              cursor_next(p, st, vc, tiles_per_run);
+            } else {
+              row = v < L_total ? stream_row(p, st, v) : p.Nk;
+            }
             for (int c = 0; c < L::V_CHUNKS; ++c)
               tma_load_3d(dst + c * BOX_BYTES + u * sub_bytes, &tm_v, &v_full[s], c * L::V_ELEMS, row, bh);
           }
@@ -308,6 +324,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int qs = w;          // qk_done stage of this group's next block (j % NK) ...
     uint32_t qph = 0;    // ... and its phase parity ((j / NK) & 1)
     bool ok = true;
+    int o_blk = (F8 && PAIR && st.rot) ? (w * BN) % st.run_len : 0;  // run offset of this group's next block
     for (int i = 0;; ++i) {
       const int j = 2 * i + w;
       if (j >= nblk) break;
@@ -337,8 +354,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // (quads 0, 1) see run tiles 0 .. ew-1 (w0+1 .. w0+ew), the second's
         // (quads 2, 3) run tiles 0 .. ew-2 and ew (w0+1 .. w0+ew-1, then w0);
         // 32-column groups never cross a tile (s is a multiple of 64)
-        const int x0 = (quad >> 1 ? st.ew : st.ew - 1) * p.g.s;  // excluded run offsets [x0, x0 + s)
-        const int o = (j * BN) % st.run_len;
+        const int x0 = straddle_excluded_start(p.g.s, st.ew, quad >> 1);  // excluded run offsets [x0, x0 + s)
+        int o;
+        if constexpr (F8) {  // no division in the e4m3 kernel (see KeyCursor)
+          o = o_blk;
+          o_blk += 2 * BN;  // this group's next block
+          while (o_blk >= st.run_len) o_blk -= st.run_len;
+        } else {
+          o = (j * BN) % st.run_len;
+        }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           int oq = o + q4 * 32;
@@ -569,10 +593,6 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
     while (G < BN && g.s % (G * 2) == 0) G *= 2;
     p.G = G;
     p.q_blocks_per_tile = (g.s + BM - 1) / BM;
-    p.pair_k = 0;
-    p.pair_nw = 1;
-    p.pair_np = 0;
-    p.pair_bpr = p.q_blocks_per_tile;
     p.Nk = g.N;
     if (a.kgeom) {  // hierarchical: coarse tiles of the medium-pooled grid (same tile volume)
       p.kNt = a.kgeom->Nt;
@@ -590,19 +610,15 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
     // that no query block is half empty (tile-major rows; sliding windows of
     // at least two tiles along w, so a straddling block's first key tile is in
     // both windows)
-    if (!p.raster && g.s % BM == BM / 2 && g.wmode == WIN_SLIDING && win_extent(g.ww, p.kNw) >= 2 && g.Nw >= 2) {
-      p.pair_k = g.s / BM;
-      p.pair_nw = g.Nw;
-      p.pair_np = g.Nw / 2;
-      p.pair_bpr = p.pair_np * (2 * p.pair_k + 1) + (g.Nw % 2) * (p.pair_k + 1);
-      qblocks = g.Nt * g.Nh * p.pair_bpr;
+    p.pair = make_pair_plan(g, p.kNw, !p.raster);
+    if (p.pair.np > 0) {
+      qblocks = (int)pair_plan_blocks(g, p.pair);
       pair = true;
     }
   } else {
     p.G = BN;
     p.q_blocks_per_tile = 1;
-    p.pair_k = p.pair_np = 0;
-    p.pair_nw = p.pair_bpr = 1;
+    p.pair = make_pair_plan(g, g.Nw, false);
     p.Nk = g.Np;
     qblocks = (g.N + BM - 1) / BM;
   }

@@ -13,12 +13,17 @@ constexpr float LOG2E = 1.4426950408889634f;
 // A row stream over a box of tiles (see TileBox) or a flat range.
 struct RowStream {
   int runs, run_len, eh, t0, h0, w0;
+  int ew;    // window tiles along w (window_stream)
+  int rot;   // straddling query block over windows one tile apart (see rotated_offset)
   bool tiled;
   __device__ __forceinline__ int length() const { return runs * run_len; }
   __device__ __forceinline__ int row(const DevGeom& g, int v) const {
     if (!tiled) return v;
     const int r = v / run_len, o = v - r * run_len;
     const int kt = t0 + r / eh, kh = h0 + r % eh;
+    // a branch, not a select, so that the rotation's division is not
+    // evaluated for every sub-box (XU pipe, shared with exp2)
+    if (rot) return ((kt * g.Nh + kh) * g.Nw + w0) * g.s + rotated_offset(o, g.s, ew);
     return ((kt * g.Nh + kh) * g.Nw + w0) * g.s + o;
   }
 };
@@ -29,6 +34,8 @@ __device__ __forceinline__ RowStream flat_stream(int n) {
   s.run_len = n;
   s.eh = 1;
   s.t0 = s.h0 = s.w0 = 0;
+  s.ew = 1;
+  s.rot = 0;
   s.tiled = false;
   return s;
 }
@@ -57,6 +64,8 @@ __device__ __forceinline__ RowStream window_stream(const DevGeom& g, const DevGe
   tile_range(aw / cfw, g.ww, gk.Nw, g.wmode, &s.w0, &ew);
   s.runs = et * s.eh;
   s.run_len = ew * g.s;
+  s.ew = ew;
+  s.rot = 0;
   s.tiled = true;
   return s;
 }
@@ -78,6 +87,8 @@ __device__ __forceinline__ RowStream inverse_stream(const DevGeom& g, const DevG
   s.eh = (hh - lh + 1) * cfh;
   s.runs = (ht - lt + 1) * cft * s.eh;
   s.run_len = (hw - lw + 1) * cfw * g.s;
+  s.ew = (hw - lw + 1) * cfw;
+  s.rot = 0;
   s.tiled = true;
   return s;
 }
@@ -125,6 +136,7 @@ struct DqParams {
   int mode;          // DQ_LOCAL / DQ_GLOBAL / DQ_HIER
   int G0;            // key sub-box rows of the local stream
   int q_blocks_per_tile;
+  PairPlan pair;     // LOCAL / HIER query blocks (see PairPlan; used by the PAIR instance)
   float c2;
   float scale;
   const float* nlse2;    // log2(gamma) - LSE*log2(e) of this branch

@@ -389,4 +389,93 @@ struct TileBox {
   int et, eh, ew;   // extent in tiles
 };
 
+// ---------------------------------------------------------------------------
+// 128-row query blocks over the tile-major rows of the sliding tile.  A tile
+// volume that is an odd multiple of 64 rows (192 at 1080p and 4K) would leave
+// one half-empty block per tile; instead w-adjacent tiles of a tile row
+// (w = 2i, 2i+1) share their blocks: k = s / 128 whole blocks of each and one
+// block straddling the two (the first tile's last 64 rows, the second's first
+// 64).  An odd last tile of the row takes k + 1 blocks of its own.  The
+// straddling block attends to the union of the two windows, which along w
+// start at most one tile apart (sliding windows); the rows of each tile mask
+// the key tile outside their own window.
+// ---------------------------------------------------------------------------
+struct PairPlan {
+  int k;    // whole 128-row blocks per tile (pairing only)
+  int nw;   // tiles per tile row (Nw); 1 unpaired (each tile a row of its own)
+  int np;   // pairs per tile row (Nw / 2); 0 unpaired
+  int bpr;  // query blocks per tile row
+};
+
+// key_nw: tiles of the key grid along w (the query grid's, or the coarse grid
+// of the hierarchical branch).  A straddling block's first key tile must lie
+// in both windows, which needs windows of at least two tiles along w.
+inline PairPlan make_pair_plan(const DevGeom& g, int key_nw, bool allow) {
+  PairPlan pp;
+  pp.k = 0;
+  pp.nw = 1;
+  pp.np = 0;
+  pp.bpr = (g.s + 127) / 128;
+  if (allow && g.s % 128 == 64 && g.wmode == WIN_SLIDING && win_extent(g.ww, key_nw) >= 2 && g.Nw >= 2) {
+    pp.k = g.s / 128;
+    pp.nw = g.Nw;
+    pp.np = g.Nw / 2;
+    pp.bpr = pp.np * (2 * pp.k + 1) + (g.Nw % 2) * (pp.k + 1);
+  }
+  return pp;
+}
+inline long long pair_plan_blocks(const DevGeom& g, const PairPlan& pp) {
+  return (long long)(g.n_tiles / pp.nw) * pp.bpr;
+}
+
+struct QueryBlock {
+  int tile;      // tile whose window the key stream starts from
+  int row0;      // first row (tile-major)
+  int valid;     // rows of the block that exist
+  int sub;       // block within its tile (unpaired)
+  int straddle;  // rows [0, 64) in tile `tile`, [64, 128) in tile `tile` + 1
+};
+
+__device__ __forceinline__ QueryBlock paired_query_block(const DevGeom& g, const PairPlan& pp, int qblk) {
+  QueryBlock b;
+  // tile row r (unpaired: tile r), block i of it; pair pi (np: the row's odd
+  // last tile), block sb of the pair
+  const int r = qblk / pp.bpr, i = qblk - r * pp.bpr;
+  const int span = 2 * pp.k + 1;
+  const int pi = min(i / span, pp.np);
+  const int a = r * pp.nw + 2 * pi, sb = i - pi * span;
+  const bool in_pair = pi < pp.np;
+  b.row0 = a * g.s + sb * 128;
+  b.valid = min(128, (in_pair ? 2 * g.s : g.s) - sb * 128);
+  b.tile = a + (in_pair && sb > pp.k ? 1 : 0);
+  b.straddle = in_pair && sb == pp.k;
+  b.sub = sb;
+  return b;
+}
+
+// Straddling block of tiles a, a + 1: how far (0 or 1 tiles) the second
+// tile's window along w starts after the first's.
+__device__ __forceinline__ int straddle_shift(const DevGeom& g, int key_nw, int cfw, int a) {
+  const int aw = a % g.Nw;
+  int s0, e0, s1, e1;
+  tile_range(aw / cfw, g.ww, key_nw, g.wmode, &s0, &e0);
+  tile_range((aw + 1) / cfw, g.ww, key_nw, g.wmode, &s1, &e1);
+  return s1 - s0;
+}
+
+// A straddling block over windows one tile apart streams each run of ew + 1
+// key tiles from its second tile (w0 + 1, in both windows) to w0 + ew and then
+// w0: run offset o -> offset in the unrotated run (tiles of s rows).
+__device__ __forceinline__ int rotated_offset(int o, int s, int ew) {
+  const int ti = o / s;
+  return (ti < ew ? ti + 1 : 0) * s + (o - ti * s);
+}
+
+// Run offsets [x0, x0 + s) that the rows of the first tile (second = false:
+// the tile w0 + ew) or of the second tile (second = true: the tile w0) do not
+// see, in the rotated order.
+__device__ __forceinline__ int straddle_excluded_start(int s, int ew, bool second) {
+  return (second ? ew : ew - 1) * s;
+}
+
 }  // namespace vattn

@@ -16,14 +16,7 @@ struct Params {
   int mode;
   int G;             // rows per TMA sub-box of a key block (divides the tile volume)
   int q_blocks_per_tile;
-  // STA query blocks.  With a tile volume an odd multiple of BM/2 (e.g. 192
-  // rows), adjacent tiles of a tile row (w = 2i, 2i+1) share their query
-  // blocks: pair_k = s / BM whole blocks of each and one block straddling the
-  // two; an odd last tile of the row takes pair_k + 1 blocks of its own.  Then
-  // pair_nw = Nw tiles and pair_np = Nw / 2 pairs per tile row, pair_bpr query
-  // blocks per tile row.  Unpaired: pair_nw = 1, pair_np = 0 and pair_bpr =
-  // q_blocks_per_tile (each tile a row of its own).
-  int pair_k, pair_nw, pair_np, pair_bpr;
+  PairPlan pair;     // STA query blocks (see PairPlan; used by the PAIR instance)
   int Nk;            // key rows per batch*head in the K/V tensors
   float scale_log2;  // scale * log2(e)
   __nv_bfloat16* o;
@@ -116,47 +109,25 @@ __device__ __forceinline__ Stream make_stream(const Params& p, int q_tile) {
   return s;
 }
 
-// Query block -> its rows and the key stream it attends to.  Sliding tile:
-// the block's tile (or, for a straddling block, the union of the windows of
-// tiles a and a + 1, which share t and h and whose windows along w start at
-// most one tile apart); global: every pooled key.
-struct QueryBlock {
-  int tile;      // anchor tile of the key stream (STA)
-  int row0;      // first row (tile-major)
-  int valid;     // rows of the block that exist
-  int sub;       // block within its tile (raster loads)
-  int straddle;  // rows [0, BM/2) in tile `tile`, [BM/2, BM) in tile `tile` + 1
-};
-
+// Query block -> its rows (QueryBlock) and the key stream it attends to:
+// sliding tile, the window of the block's tile or, for a straddling block, the
+// union of the windows of tiles a and a + 1; global, every pooled key.
 template <bool PAIR>
 __device__ __forceinline__ QueryBlock query_block(const Params& p, int qblk) {
   QueryBlock b;
   const DevGeom& g = p.g;
-  if (!PAIR && p.mode == FWD_STA) {
+  if (PAIR && p.mode == FWD_STA) return paired_query_block(g, p.pair, qblk);
+  b.straddle = 0;
+  if (p.mode == FWD_STA) {
     b.tile = qblk / p.q_blocks_per_tile;
     b.sub = qblk - b.tile * p.q_blocks_per_tile;
     b.row0 = b.tile * g.s + b.sub * BM;
     b.valid = min(BM, g.s - b.sub * BM);
-    b.straddle = 0;
-  } else if (p.mode == FWD_STA) {
-    // tile row r (or, unpaired, tile r), block i of it; pair pi (npair: the
-    // row's odd last tile), block sb of the pair
-    const int r = qblk / p.pair_bpr, i = qblk - r * p.pair_bpr;
-    const int span = 2 * p.pair_k + 1;
-    const int pi = min(i / span, p.pair_np);
-    const int a = r * p.pair_nw + 2 * pi, sb = i - pi * span;
-    const bool in_pair = pi < p.pair_np;
-    b.row0 = a * g.s + sb * BM;
-    b.valid = min(BM, (in_pair ? 2 * g.s : g.s) - sb * BM);
-    b.tile = a + (in_pair && sb > p.pair_k ? 1 : 0);
-    b.straddle = in_pair && sb == p.pair_k;
-    b.sub = sb;
   } else {
     b.tile = 0;
     b.row0 = qblk * BM;
     b.valid = min(BM, g.N - b.row0);
     b.sub = 0;
-    b.straddle = 0;
   }
   return b;
 }
@@ -164,14 +135,9 @@ __device__ __forceinline__ QueryBlock query_block(const Params& p, int qblk) {
 template <bool PAIR>
 __device__ __forceinline__ Stream make_block_stream(const Params& p, const QueryBlock& b) {
   Stream s = make_stream(p, b.tile);
-  if (PAIR && b.straddle) {
-    const DevGeom& g = p.g;
-    int w0b, ewb;
-    tile_range((b.tile % g.Nw + 1) / p.cfw, g.ww, p.kNw, g.wmode, &w0b, &ewb);
-    if (w0b != s.w0) {  // one tile apart (sliding windows of equal extent)
-      s.rot = 1;
-      s.run_len += g.s;
-    }
+  if (PAIR && b.straddle && straddle_shift(p.g, p.kNw, p.cfw, b.tile) != 0) {
+    s.rot = 1;
+    s.run_len += p.g.s;
   }
   return s;
 }
@@ -181,12 +147,61 @@ __device__ __forceinline__ int stream_row(const Params& p, const Stream& s, int 
   if (p.mode != FWD_STA) return v;
   const int r = v / s.run_len, o = v - r * s.run_len;
   const int kt = s.t0 + r / s.eh, kh = s.h0 + r % s.eh;
-  if (s.rot) {  // run order w0 + 1, ..., w0 + ew, w0
-    const int ti = o / p.g.s, lo = o - ti * p.g.s;
-    const int wt = ti < s.ew ? ti + 1 : 0;
-    return ((kt * p.kNh + kh) * p.kNw + s.w0 + wt) * p.g.s + lo;
-  }
+  // a branch, not a select: evaluated for every sub-box, the rotation's
+  // division cost the bf16 paired forward 20% (XU pipe, shared with exp2)
+  if (s.rot) return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + rotated_offset(o, p.g.s, s.ew);
   return ((kt * p.kNh + kh) * p.kNw + s.w0) * p.g.s + o;
+}
+
+// Walks the key stream one sub-box of G rows at a time with no integer
+// division in the loop (the e4m3 kernel's loaders; tile-major rows).  Integer
+// division runs on the XU pipe that also computes the softmax's exponentials:
+// the e4m3 kernel is bound by that pipe and instruction issue, and dropping
+// the loaders' per-sub-box divisions made it 4-8% faster, while the bf16
+// kernel, held by the power cap, measured 1-2% slower with the cursor and
+// keeps the direct address computation (stream_row, stream_box).
+// Sliding tile: run (kt, kh), tile ti of the run, row lo of the tile; global:
+// the flat position v.  Past the end of the stream `left` reaches 0.
+struct KeyCursor {
+  int kt, kh, ti, lo;
+  int left;  // sub-boxes left in the stream
+  int v;     // flat position (global)
+};
+
+__device__ __forceinline__ KeyCursor key_cursor(const Params& p, const Stream& s, int L_total) {
+  KeyCursor c;
+  c.kt = s.t0;
+  c.kh = s.h0;
+  c.ti = c.lo = 0;
+  c.left = (L_total + p.G - 1) / p.G;
+  c.v = 0;
+  return c;
+}
+
+// Key row (within the batch*head slice) of the cursor's sub-box; past the end,
+// row Nk (zero fill).
+__device__ __forceinline__ int cursor_row(const Params& p, const Stream& s, const KeyCursor& c) {
+  if (c.left <= 0) return p.Nk;
+  if (p.mode != FWD_STA) return c.v;
+  const int wt = s.rot ? (c.ti < s.ew ? c.ti + 1 : 0) : c.ti;
+  return ((c.kt * p.kNh + c.kh) * p.kNw + s.w0 + wt) * p.g.s + c.lo;
+}
+
+// Next sub-box.  G divides the tile volume, so a sub-box never crosses a tile.
+__device__ __forceinline__ void cursor_next(const Params& p, const Stream& s, KeyCursor& c, int tiles_per_run) {
+  --c.left;
+  c.v += p.G;
+  c.lo += p.G;
+  if (c.lo >= p.g.s) {
+    c.lo = 0;
+    if (++c.ti == tiles_per_run) {
+      c.ti = 0;
+      if (++c.kh == s.h0 + s.eh) {
+        c.kh = s.h0;
+        ++c.kt;
+      }
+    }
+  }
 }
 
 // Raster box of key stream position v (a multiple of the sub-box rows): the
