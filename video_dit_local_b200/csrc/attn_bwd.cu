@@ -135,7 +135,7 @@ struct DkdvSmem {
   static constexpr int ALLOC = TOTAL + 1024;
 };
 
-template <int D>
+template <int D, bool PAIR = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
@@ -172,7 +172,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   int key_row0, key_valid;
   RowStream qs;
-  if (p.mode != DKDV_GLOBAL) {
+  // PAIR, straddling key block (keys [0, 64) of tile a, [64, 128) of tile
+  // a + 1): the query stream is the union of the two inverse windows, which
+  // along w are contiguous and nested in order; the first tile's key rows
+  // (quads 0, 1) skip run offsets >= xa, the second's (quads 2, 3) offsets < xb
+  int xa = 0, xb = 0;
+  bool kmask = false;
+  if (PAIR && p.mode == DKDV_LOCAL) {
+    const QueryBlock kb = paired_query_block(g, p.pair, blockIdx.x);  // key blocks, same layout
+    key_row0 = kb.row0;
+    key_valid = kb.valid;
+    qs = inverse_stream(g, p.gk, 1, 1, 1, kb.tile);
+    if (kb.straddle) {
+      const RowStream q2 = inverse_stream(g, p.gk, 1, 1, 1, kb.tile + 1);
+      xa = qs.run_len;
+      xb = (q2.w0 - qs.w0) * g.s;
+      qs.run_len = xb + q2.run_len;
+      kmask = xa < qs.run_len || xb > 0;
+    }
+  } else if (p.mode != DKDV_GLOBAL) {
     const int kt = blockIdx.x / p.kv_blocks_per_tile;
     const int sb = blockIdx.x - kt * p.kv_blocks_per_tile;
     key_row0 = kt * g.s + sb * 128;
@@ -326,6 +344,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tS = tmem + lane_addr + (uint32_t)(w * 64);
     const uint32_t tP = tmem + lane_addr + 128u + (uint32_t)(w * 64);
     bool ok = true;
+    int o_blk = (PAIR && kmask) ? (w * 64) % qs.run_len : 0;  // run offset of this group's block
     for (int i = w; i < nblk; i += 2) {
       const int it = i >> 1, s = i % NQ;
       ok = mbar_wait(&sdp_full[w], it & 1, wc);
@@ -336,8 +355,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float2 c2x2 = make_float2(p.c2, p.c2);
       const float4* ls4 = reinterpret_cast<const float4*>(lse_s + s * 64);
       const float4* ds4 = reinterpret_cast<const float4*>(del_s + s * 64);
-      const bool full_blk = Lq - i * 64 >= 64;   // uniform: only the last block is ragged
-      const int valid = Lq - i * 64;
+      int valid = Lq - i * 64;
+      if (PAIR && kmask) {
+        // a 64-query block lies in one query tile (s is a multiple of 64): the
+        // whole block is outside this warp's key rows' window or inside it
+        if ((quad >> 1) ? o_blk < xb : o_blk >= xa) valid = 0;
+        o_blk += 128;  // this group's next block
+        while (o_blk >= qs.run_len) o_blk -= qs.run_len;
+      }
+      const bool full_blk = valid >= 64;   // uniform: the last block, or a masked one
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         // one 32-column half at a time keeps S, dP and the packed outputs in registers
@@ -781,6 +807,9 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   p.mode = global ? DKDV_GLOBAL : DKDV_LOCAL;
   p.Gq = global ? 64 : pow2_rows(g.s, 64);
   p.kv_blocks_per_tile = (g.s + 127) / 128;
+  // local keys: w-adjacent tiles of an odd multiple of 64 rows share their key
+  // blocks (PairPlan), as the forward's query blocks
+  p.pair = make_pair_plan(g, g.Nw, !global && !hk);
   p.Nk = global ? g.Np : g.N;
   if (hk && global) {
     p.gk = *hk;
@@ -806,9 +835,10 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   p.dvp_in = (!global && dual) ? a.dvp : nullptr;
   p.ctl = current_ctl();
   const long long bh = (long long)g.B * g.heads;
+  const bool pair = p.pair.np > 0;
   const int blocks = p.mode == DKDV_GLOBAL ? (g.Np + 127) / 128
                      : p.mode == DKDV_HIER ? hk->n_tiles * p.kv_blocks_per_tile
-                                           : g.n_tiles * p.kv_blocks_per_tile;
+                                           : (int)pair_plan_blocks(g, p.pair);
   if (bh == 0 || blocks == 0) return cudaSuccess;
   CUtensorMap tk, tv, tq, tdo;
   const char* err = nullptr;
@@ -817,9 +847,10 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   if (!make_tmap_rows(&tk, kp, D, p.Nk, bh, 128, &err) || !make_tmap_rows(&tv, vp, D, p.Nk, bh, 128, &err) ||
       !make_tmap_rows(&tq, a.q, D, g.N, bh, p.Gq, &err) || !make_tmap_rows(&tdo, a.dout, D, g.N, bh, p.Gq, &err))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_smem(dkdv_kernel<D>, DkdvSmem<D>::ALLOC);
+  auto kernel = pair ? dkdv_kernel<D, true> : dkdv_kernel<D, false>;
+  cudaError_t e = set_smem(kernel, DkdvSmem<D>::ALLOC);
   if (e != cudaSuccess) return e;
-  dkdv_kernel<D><<<dim3(blocks, (unsigned)bh), NTHREADS, DkdvSmem<D>::ALLOC, st>>>(tk, tv, tq, tdo, p);
+  kernel<<<dim3(blocks, (unsigned)bh), NTHREADS, DkdvSmem<D>::ALLOC, st>>>(tk, tv, tq, tdo, p);
   return cudaGetLastError();
 }
 

@@ -161,6 +161,7 @@ struct DkdvParams {
   int mode;          // DKDV_LOCAL / DKDV_GLOBAL / DKDV_HIER
   int Gq;            // query sub-box rows (divides the tile volume, <= 64)
   int kv_blocks_per_tile;
+  PairPlan pair;     // LOCAL key blocks (see PairPlan; used by the PAIR instance)
   int Nk;            // key rows per batch*head (N or Np)
   float c2;          // scale * log2(e)
   float scale;
