@@ -638,6 +638,65 @@ def dual_sym_backward(q, k, v, gvec, do, g: Geom, scale: float):
 
 
 # ---------------------------------------------------------------------------
+# symmetric global branch, learned variant ("UltraGen ..." §4.2: the latents
+# are compressed by a depthwise convolution of stride k before global
+# attention; after it, bilinear upsampling and a 3D convolution restore the
+# full grid, processing space and time jointly).  Readings taken: the
+# compression kernel equals its stride (p_t x p_h x p_w taps, non-overlapping,
+# no bias), one kernel per head and channel, applied to Q, K and V with
+# separate weights; the restoring convolution is depthwise as well, 3 x 3 x 3
+# with zero padding (output on the full grid), no bias, applied to the
+# upsampled global output before the blend; convolution means
+# cross-correlation (out[t] = sum_a w[a] x[t + a]).  The weights are inputs:
+# the method's trained values are not available, so tests draw them at random.
+# ---------------------------------------------------------------------------
+
+def conv_compress(x_raster: np.ndarray, g: Geom, w: np.ndarray) -> np.ndarray:
+    """Depthwise strided convolution; x [B, h, N, d] raster, w [h, P, d] with
+    the P = p_t*p_h*p_w taps in (dt, dy, dx) raster order:
+    x_p[t', y', x', c] = sum_taps w[h, tap, c] * x[t' p_t + dt, y' p_h + dy, x' p_w + dx, c]."""
+    PT, PH, PW = g.pooled_dims
+    pt, ph, pw = g.pool
+    B, nh, _, d = x_raster.shape
+    x = x_raster.reshape(B, nh, PT, pt, PH, ph, PW, pw, d)
+    wr = np.asarray(w, dtype=np.float64).reshape(nh, pt, ph, pw, d)
+    y = np.einsum("bhTiHjWkd,hijkd->bhTHWd", x, wr)
+    return y.reshape(B, nh, g.n_pooled, d)
+
+
+def conv3d_depthwise(x_raster: np.ndarray, g: Geom, w3: np.ndarray) -> np.ndarray:
+    """3 x 3 x 3 depthwise convolution with zero padding on the full grid;
+    x [B, h, N, d] raster, w3 [h, 27, d] with taps (a, b, e) in {-1, 0, 1}^3,
+    raster order: y[t, y, x, c] = sum w3[h, tap, c] * x[t + a, y + b, x + e, c]."""
+    B, nh, _, d = x_raster.shape
+    x = x_raster.reshape(B, nh, g.T, g.H, g.W, d)
+    xp = np.zeros((B, nh, g.T + 2, g.H + 2, g.W + 2, d))
+    xp[:, :, 1:-1, 1:-1, 1:-1, :] = x
+    w = np.asarray(w3, dtype=np.float64)
+    y = np.zeros_like(x)
+    tap = 0
+    for a in (-1, 0, 1):
+        for b in (-1, 0, 1):
+            for e in (-1, 0, 1):
+                y += w[None, :, tap, None, None, None, :] * xp[:, :, 1 + a:1 + a + g.T, 1 + b:1 + b + g.H,
+                                                                1 + e:1 + e + g.W, :]
+                tap += 1
+    return y.reshape(B, nh, g.n, d)
+
+
+def dual_sym_learned_forward(q, k, v, gvec, wq, wk, wv, w3, g: Geom, scale: float):
+    """Blend of the local branch and the learned compressed global branch
+    (raster in, raster out): O_g = conv3d(upsample(attn(cq(Q), ck(K), cv(V))))."""
+    o_l, lse_l = sta_attention(q, k, v, g, scale)
+    qp, kp, vp = conv_compress(q, g, wq), conv_compress(k, g, wk), conv_compress(v, g, wv)
+    o_p, lse_p = full_attention(qp, kp, vp, scale)
+    o_g = conv3d_depthwise(upsample(o_p, g), g, w3)
+    gb = np.asarray(gvec, dtype=np.float64)[None, :, None, None]
+    return dict(O=gb * o_l + (1.0 - gb) * o_g, O_l=o_l, LSE_l=lse_l, Q_p=qp, K_p=kp, V_p=vp, O_p=o_p,
+                LSE_p=lse_p, O_g=o_g)
+
+
+# ---------------------------------------------------------------------------
 # NEXT-2: hierarchical local attention ("UltraGen ..." §4.3, hierarchical local
 # attention: intermediate-scale attention over coarse windows).  Reading: the
 # local branch also sees K and V average-pooled by a medium factor h_pool,

@@ -31,7 +31,7 @@ from typing import Optional
 import numpy as np
 
 Q_ID, K_ID, V_ID, DO_ID = 0, 1, 2, 3
-SCALE_STREAM, G_STREAM = 10, 11
+SCALE_STREAM, G_STREAM, CONV_STREAM = 10, 11, 12
 
 
 @dataclasses.dataclass(frozen=True)
@@ -97,6 +97,27 @@ def head_scales(w: Workload) -> np.ndarray:
 def blend_g(w: Workload) -> np.ndarray:
     """Per-head blend factor g in [0, 1], float32 [heads]."""
     return _stream(w.seed, G_STREAM).uniform(0.0, 1.0, size=w.heads).astype(np.float32)
+
+
+def learned_weights(w: Workload) -> dict:
+    """Random weights of the learned compression / restoration convolutions
+    (the method's trained values are not available), float32, taps-major:
+      wq, wk, wv  [heads, p_t*p_h*p_w, d]  compression taps in (dt, dy, dx)
+                  raster order, 1/P * (1 + 0.25 z): average pooling with a
+                  perturbation, so the pooled tokens keep unit scale;
+      w3          [heads, 27, d]  restoring 3x3x3 taps in (a, b, e) raster
+                  order over {-1, 0, 1}^3: the identity tap 1 at the centre
+                  plus 0.05 z everywhere."""
+    P = w.pool[0] * w.pool[1] * w.pool[2]
+    rng = _stream(w.seed, CONV_STREAM)
+    out = {}
+    for name in ("wq", "wk", "wv"):
+        z = rng.standard_normal((w.heads, P, w.head_dim), dtype=np.float32)
+        out[name] = ((1.0 + 0.25 * z) / np.float32(P)).astype(np.float32)
+    w3 = 0.05 * rng.standard_normal((w.heads, 27, w.head_dim), dtype=np.float32)
+    w3[:, 13, :] += 1.0
+    out["w3"] = w3.astype(np.float32)
+    return out
 
 
 def draw_head(w: Workload, tensor_id: int, b: int, h: int) -> np.ndarray:
