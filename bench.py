@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic per launch of the sliding-tile forward kernel at the 720p
 # workload (read+write bytes), and the hash of the kernel source it was taken
 # from.  When the source changes the figure is stale and reported as null.
-STA_FWD_TRAFFIC = 2691194880  # DRAM read + write bytes per launch: an ncu capture of the 2-head case x 12
-STA_FWD_TRAFFIC_SRC_SHA = "a8496f71416a2f96"
+STA_FWD_TRAFFIC = 2733173760  # DRAM read + write bytes per launch: an ncu capture of the 2-head case x 12
+STA_FWD_TRAFFIC_SRC_SHA = "3e82d774c7eb019e"
 
 
 def reduce_max(values, world: int, device=None):
@@ -266,6 +266,23 @@ def run_dual_only(args, rank, world, local_rank):
                                    f"pool {'x'.join(map(str, w.pool))}"}, "status": V.vattn_get_status()}
 
 
+def run_sym_learned_only(args, rank, world, local_rank):
+    """Profiling mode: the 1080p dual forward with the learned symmetric
+    global branch alone (seeded random weights), timed with CUDA events."""
+    import torch
+
+    import video_dit_local_b200 as V
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, _ = _peaks()
+    res = _bench_sym_learned(V, dev, peaks, n=args.steps, warm=args.warmup)
+    return {"metric": METRIC, "value": res["eff_tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch N(0,1), seeded random weights)",
+            "config": {"workload": "1080p dual fwd, learned symmetric global branch: B1 h24 d128, grid 21x72x120, "
+                                   "tile 3x8x8, window 3x3x3, pool 1x4x4"}, "status": res["status"]}
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -454,6 +471,7 @@ def run_extras(V, dev):
         res["clocks"] = clk.summary()
         out[name] = res
     out["1080p_dual_sym_fwd"] = clocked(lambda: _bench_sym(V, dev, peaks))
+    out["1080p_dual_sym_learned_fwd"] = clocked(lambda: _bench_sym_learned(V, dev, peaks))
     out["720p_hier_fwd_bwd"] = clocked(lambda: _bench_hier(V, dev, peaks))
     out["720p_sta_fwd_fp8"] = clocked(lambda: _bench_fp8(V, dev, peaks))
     out["1080p_dual_fwd_fp8"] = clocked(lambda: _bench_dual_fp8(V, dev, peaks))
@@ -624,6 +642,37 @@ def _bench_hier(V, dev, peaks):
            "bwd_frac": round(fl_b / ms_b / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status(),
            "h_pool": list(hp)}
     del q, k, v, o, lse, ws, do, dq, dk, dv, wsb
+    torch.cuda.empty_cache()
+    return res
+
+
+def _bench_sym_learned(V, dev, peaks, n=4, warm=2):
+    """Dual forward with the learned symmetric global branch (depthwise
+    strided compression, 3x3x3 depthwise restoration, seeded random weights)
+    at the 1080p workload; effective FLOPs as the average-pooling form (the
+    convolutions are HBM / L2 work, reported with it, not counted)."""
+    import torch
+    from synth import inputs as S
+    w = S.WORKLOADS["1080p"]
+    geom = _geom(V, w)
+    T, H, W = w.grid
+    npool = (T // w.pool[0]) * (H // w.pool[1]) * (W // w.pool[2])
+    shape = (w.batch, w.heads, w.n_tokens, w.head_dim)
+    q, k, v = (_device_randn(shape, 700 + i) for i in range(3))
+    gvec = torch.rand(w.heads, device=dev)
+    wts = {n: torch.from_numpy(a).to(dev) for n, a in S.learned_weights(w).items()}
+    o = torch.empty_like(q)
+    ws = torch.empty(V.vattn_workspace_size(V.VATTN_OP_DUAL_SYM_LEARNED_FWD, geom), dtype=torch.uint8, device=dev)
+    fl, _ = _flops_fwd(w)
+    fl += 4 * w.head_dim * w.batch * w.heads * npool * npool
+    scale = 1 / math.sqrt(w.head_dim)
+
+    def call():
+        V.vattn_dual_sym_learned_fwd(geom, q, k, v, gvec, wts["wq"], wts["wk"], wts["wv"], wts["w3"], scale, o, ws)
+    ms = _time_ms(call, n, warm=warm)
+    res = {"ms": round(ms, 3), "eff_tflops": round(fl / ms / 1e9, 1),
+           "frac": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4), "status": V.vattn_get_status()}
+    del q, k, v, o, ws
     torch.cuda.empty_cache()
     return res
 
@@ -851,9 +900,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-chunk", type=int, default=1, help="batch*head slices per host-copy chunk (e2e)")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: fewer heads than the workload")
-    ap.add_argument("--workload", choices=["720p", "train", "fp8", "1080p", "4k"], default="720p",
-                    help="720p: the benchmark line; train, fp8, 1080p, 4k: profiling of the training step, the FP8 "
-                         "forward or the 1080p / 4K dual forward alone")
+    ap.add_argument("--workload", choices=["720p", "train", "fp8", "1080p", "4k", "sym_learned"], default="720p",
+                    help="720p: the benchmark line; train, fp8, 1080p, 4k, sym_learned: profiling of the training "
+                         "step, the FP8 forward, the 1080p / 4K dual forward or the learned symmetric branch alone")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -880,6 +929,8 @@ def main():
             result = run_fp8_only(args, rank, world, local_rank)
         elif args.workload in ("1080p", "4k"):
             result = run_dual_only(args, rank, world, local_rank)
+        elif args.workload == "sym_learned":
+            result = run_sym_learned_only(args, rank, world, local_rank)
         else:
             result = run_ours(args, rank, world, local_rank)
         if rank == 0:

@@ -86,7 +86,8 @@ enum {
   VATTN_OP_HIER_FWD = 7,     /* geom->pool = the medium pool factor h_pool */
   VATTN_OP_HIER_BWD = 8,
   VATTN_OP_STA_FWD_FP8 = 9,
-  VATTN_OP_DUAL_FWD_FP8 = 10
+  VATTN_OP_DUAL_FWD_FP8 = 10,
+  VATTN_OP_DUAL_SYM_LEARNED_FWD = 11
 };
 
 /* Raster -> tile-major row gather.  Tile-major position of raster token
@@ -294,6 +295,33 @@ int vattn_dual_fwd_noalloc(const vattn_geom* geom, const void* q, const void* k,
 int vattn_dual_sym_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
                        const float* g, float scale, void* o, void* o_l, float* lse_l, void* qp, void* kp,
                        void* vp, void* o_p, float* lse_p, void* workspace, size_t ws_bytes, void* stream);
+
+/* Dual-branch forward with the learned compressed global branch
+ * ("UltraGen ..." §4.2: depthwise convolution of stride k for the
+ * compression; bilinear upsampling and a 3D convolution for the restoration,
+ * processing space and time jointly).  Inference only; the weights are
+ * inputs (random ones stand in for trained values).
+ *  - compression: Q, K, V each by a depthwise convolution whose stride equals
+ *    its p_t x p_h x p_w kernel (geom->pool), no bias:
+ *    x_p[t',y',x',c] = sum_taps w[h][tap][c] * x[t'p_t+dt, y'p_h+dy, x'p_w+dx, c];
+ *    wq, wk, wv: fp32 [heads][p_t*p_h*p_w][d], taps in (dt, dy, dx) raster
+ *    order (uniform taps 1/(p_t p_h p_w) give vattn_dual_sym_fwd's pooling);
+ *  - the pooled queries attend to all pooled keys (scale);
+ *  - restoration: the upsampling of vattn_dual_sym_fwd, then a 3x3x3
+ *    depthwise convolution with zero padding, no bias:
+ *    O_g[t,y,x,c] = sum w3[h][tap][c] * U[t+a, y+b, x+e, c], taps (a, b, e)
+ *    over {-1, 0, 1}^3 in raster order; w3: fp32 [heads][27][d] (the
+ *    identity tap 13 alone gives vattn_dual_sym_fwd's output);
+ *  - O = g*O_l + (1-g)*O_g.
+ * q, k, v, o: bf16 [B,h,N,d] tile-major; d a multiple of 8; weight pointers
+ * 16-byte aligned.  workspace >= vattn_workspace_size
+ * (VATTN_OP_DUAL_SYM_LEARNED_FWD), in this order (each 256-byte aligned):
+ * O_l [B,h,N,d] bf16, Q_p, K_p, V_p, O_p [B,h,N_p,d] bf16 (pooled raster),
+ * U [B,h,N,d] bf16 (raster: the upsampled pooled output, rounded to bf16). */
+int vattn_dual_sym_learned_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                               const float* g, const float* wq, const float* wk, const float* wv,
+                               const float* w3, float scale, void* o, void* workspace, size_t ws_bytes,
+                               void* stream);
 
 /* Backward of vattn_dual_sym_fwd from its saved outputs: dq, dk, dv (bf16,
  * tile-major) through the pooling of all three inputs and the upsampling.

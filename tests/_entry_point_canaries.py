@@ -146,6 +146,13 @@ def main(out_path):
     V.vattn_dual_sym_fwd(geom, q, k, v, gvec, scale, osy, osl, lsl, qps, kps, vps, ops, lps)
     check("vattn_dual_sym_fwd")
     saved["sym_o"] = osy.cpu().view(torch.int16).numpy()
+    wts = {n: guarded(f"learned {n}", tuple(a.shape), torch.float32, fill=torch.from_numpy(a).cuda())
+           for n, a in S.learned_weights(w).items()}
+    olr = guarded("sym learned O", tuple(q.shape), torch.bfloat16)
+    V.vattn_dual_sym_learned_fwd(geom, q, k, v, gvec, wts["wq"], wts["wk"], wts["wv"], wts["w3"], scale, olr,
+                                 workspace("sym learned ws", V.VATTN_OP_DUAL_SYM_LEARNED_FWD, geom))
+    check("vattn_dual_sym_learned_fwd")
+    saved["sym_learned_o"] = olr.cpu().view(torch.int16).numpy()
 
     # host-buffer forward: host outputs with canaries in host memory
     ohh = guarded("host O", tuple(qr.shape), torch.bfloat16, device="cpu")

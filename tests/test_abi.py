@@ -131,6 +131,9 @@ def test_workspace_sizes(V):
         + 2 * a(bh * npool * d * 2))
     # FP8 forward: e4m3 Q, K and V bytes, the (Q, K) absmax pairs, V's absmax
     assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_FP8, g) == 3 * a(bh * n * d) + a(bh * 8) + a(bh * 4)
+    # learned symmetric branch: O_l, Q_p, K_p, V_p, O_p, the upsampled field U (all bf16)
+    assert V.vattn_workspace_size(V.VATTN_OP_DUAL_SYM_LEARNED_FWD, g) == (a(bh * n * d * 2) + 4 * a(bh * npool * d * 2)
+                                                                       + a(bh * n * d * 2))
     # host-buffer forward, per slot: 8 bf16 token tensors and 2 fp32 rows
     assert V.vattn_workspace_size(V.VATTN_OP_STA_FWD_HOST, g) == 8 * a(bh * n * d * 2) + 2 * a(bh * n * 4)
     assert V.vattn_workspace_size(V.VATTN_OP_DUAL_BWD, g) == (4 * a(bh * n * 4) + 2 * a(bh * npool * d * 4)

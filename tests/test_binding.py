@@ -69,6 +69,8 @@ def _calls(B):
         "vattn_xwin_fwd": lambda: B.vattn_xwin_fwd(g, 1, t(), t(), t(), 0.1, t(), t()),
         "vattn_xwin_bwd": lambda: B.vattn_xwin_bwd(g, 0, *(t() for _ in range(6)), 0.1, t(), t(), t(), t()),
         "vattn_dual_sym_fwd": lambda: B.vattn_dual_sym_fwd(g, t(), t(), t(), t(), 0.1, t(), workspace=t()),
+        "vattn_dual_sym_learned_fwd": lambda: B.vattn_dual_sym_learned_fwd(g, t(), t(), t(), t(), t(), t(), t(), t(), 0.1,
+                                                                           t(), t()),
         "vattn_dual_sym_bwd": lambda: B.vattn_dual_sym_bwd(g, *(t() for _ in range(12)), 0.1, t(), t(), t(), t()),
         "vattn_hier_fwd": lambda: B.vattn_hier_fwd(g, t(), t(), t(), 0.1, t(), t(), t()),
         "vattn_hier_bwd": lambda: B.vattn_hier_bwd(g, *(t() for _ in range(6)), 0.1, t(), t(), t(), t()),

@@ -39,6 +39,7 @@ VATTN_OP_HIER_FWD = 7
 VATTN_OP_HIER_BWD = 8
 VATTN_OP_STA_FWD_FP8 = 9
 VATTN_OP_DUAL_FWD_FP8 = 10
+VATTN_OP_DUAL_SYM_LEARNED_FWD = 11
 VATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 VATTN_DEBUG_SKIP_ARRIVAL = 1
@@ -101,6 +102,7 @@ _SIGS = {
     "vattn_sta_fwd_fp8": [_GP, _P, _P, _P, _F, _P, _P, _P, _SZ, _P],
     "vattn_sta_fwd_host": [_GP, _P, _P, _P, _F, _P, _P, _I64, _P, _SZ, _P],
     "vattn_dual_sym_fwd": [_GP, _P, _P, _P, _P, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "vattn_dual_sym_learned_fwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _SZ, _P],
     "vattn_dual_sym_bwd": [_GP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_xwin_bwd": [_GP, _INT, _P, _P, _P, _P, _P, _P, _F, _P, _P, _P, _P, _SZ, _P],
     "vattn_workspace_size": [_INT, _GP, ctypes.POINTER(_SZ)],
@@ -208,6 +210,17 @@ def vattn_dual_sym_fwd(geom: Geom, q, k, v, g, scale: float, o, o_l=None, lse_l=
     _check(lib.vattn_dual_sym_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), scale, _ptr(o), _ptr(o_l),
                                   _ptr(lse_l), _ptr(qp), _ptr(kp), _ptr(vp), _ptr(o_p), _ptr(lse_p), _ptr(workspace),
                                   ws_bytes, _stream(stream)))
+
+
+def vattn_dual_sym_learned_fwd(geom: Geom, q, k, v, g, wq, wk, wv, w3, scale: float, o, workspace,
+                               ws_bytes: int = 0, stream=None) -> None:
+    """Learned compressed global branch (inference): weights fp32, taps-major
+    ([heads, p_t*p_h*p_w, d] for wq/wk/wv, [heads, 27, d] for w3)."""
+    if workspace is not None and not ws_bytes:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.vattn_dual_sym_learned_fwd(ctypes.byref(geom), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(wq), _ptr(wk),
+                                          _ptr(wv), _ptr(w3), scale, _ptr(o), _ptr(workspace), ws_bytes,
+                                          _stream(stream)))
 
 
 def vattn_dual_sym_bwd(geom: Geom, q, k, v, g, o_l, lse_l, qp, kp, vp, o_p, lse_p, dout, scale: float, dq, dk, dv,

@@ -560,6 +560,266 @@ cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void*
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Learned variant of the symmetric global branch ("UltraGen ..." §4.2):
+// compression by a depthwise convolution whose stride equals its
+// p_t x p_h x p_w kernel, restoration by the upsampling above followed by a
+// 3 x 3 x 3 depthwise convolution (zero padding).  Weights are fp32, taps-major
+// ([heads][taps][d]) so that one thread's 8 (or 4) channels of one tap are
+// contiguous.  All HBM-bound except the restoring convolution, whose 27 taps
+// read the fp32 upsampled field U mostly from L1 / L2.
+// ---------------------------------------------------------------------------
+
+struct CompressWeights {
+  const float* w[3];
+};
+
+// One thread: one 16-byte vector (8 channels) of one pooled row of one
+// tensor; fp32 sum over the taps in (dt, dy, dx) order, one RNE to bf16.
+__global__ void __launch_bounds__(256) compress_kernel(PoolParams p, FastDiv per_row, FastDiv n_prow,
+                                                        FastDiv rows_per_tensor, PoolTensors ts, CompressWeights cw,
+                                                        int heads, int bh0, int* err) {
+  const uint32_t total = (uint32_t)ts.count * rows_per_tensor.d * p.vpr;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  const int taps = (int)(p.pt * p.ph * p.pw), d = (int)p.vpr * 8;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t row2 = per_row.div(i);
+    const uint32_t c = i - row2 * p.vpr;
+    const uint32_t which = rows_per_tensor.div(row2);
+    const uint32_t row = row2 - which * rows_per_tensor.d;
+    const uint32_t bh = n_prow.div(row);
+    const uint32_t u = row - bh * p.Np;
+    const uint32_t r = p.PW.div(u);
+    const uint32_t ux = u - r * p.PWv;
+    const uint32_t ut = p.PH.div(r);
+    const uint32_t uy = r - ut * p.PHv;
+    const uint4* src = ts.src[which] + (size_t)bh * p.N * p.vpr + c;
+    const float* wt = cw.w[which] + (size_t)((bh0 + (int)bh) % heads) * taps * d + c * 8;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    int tap = 0;
+    for (uint32_t a = 0; a < p.pt; ++a)
+      for (uint32_t b = 0; b < p.ph; ++b)
+        for (uint32_t x = 0; x < p.pw; ++x, ++tap) {
+          const uint32_t m = coords_to_tiled(p.rp, ut * p.pt + a, uy * p.ph + b, ux * p.pw + x);
+          if (!dcheck(m < p.N, err)) continue;
+          const uint4 v = __ldg(src + (size_t)m * p.vpr);
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wt + (size_t)tap * d));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wt + (size_t)tap * d) + 1);
+          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] = fmaf(wv[2 * e], bf16lo(vv[e]), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wv[2 * e + 1], bf16hi(vv[e]), acc[2 * e + 1]);
+          }
+        }
+    uint4 o;
+    o.x = pack_bf16(acc[0], acc[1]);
+    o.y = pack_bf16(acc[2], acc[3]);
+    o.z = pack_bf16(acc[4], acc[5]);
+    o.w = pack_bf16(acc[6], acc[7]);
+    if (!dcheck(u < p.Np, err)) continue;
+    ts.dst[which][((size_t)bh * p.Np + u) * p.vpr + c] = o;
+  }
+}
+
+cudaError_t launch_compress_qkv(const DevGeom& g, const void* q, const void* k, const void* v, const float* wq,
+                                const float* wk, const float* wv, void* qp, void* kp, void* vp, cudaStream_t st) {
+  PoolParams p = make_pool_params(g);
+  const int count = 3;
+  const long long per_bh = (long long)g.Np * p.vpr;
+  const long long bh_total = (long long)g.B * g.heads;
+  if (per_bh * bh_total == 0) return cudaSuccess;
+  if (g.d % 8 != 0) return cudaErrorInvalidValue;
+  const long long chunk = ((1ll << 31) - 1) / (per_bh * count);  // every launch below 2^31 vectors
+  if (chunk < 1) return cudaErrorInvalidValue;
+  const void* src[3] = {q, k, v};
+  void* dst[3] = {qp, kp, vp};
+  CompressWeights cw;
+  cw.w[0] = wq;
+  cw.w[1] = wk;
+  cw.w[2] = wv;
+  for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
+    const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
+    const uint32_t rows = (uint32_t)(nb * g.Np);
+    const size_t in_off = (size_t)b0 * g.N * p.vpr, out_off = (size_t)b0 * g.Np * p.vpr;
+    PoolTensors ts;
+    ts.count = count;
+    for (int i = 0; i < 3; ++i) {
+      ts.src[i] = (const uint4*)src[i] + in_off;
+      ts.dst[i] = (uint4*)dst[i] + out_off;
+    }
+    const int grid = grid_for((long long)count * rows * p.vpr, 256);
+    compress_kernel<<<grid, 256, 0, st>>>(p, FastDiv(p.vpr), FastDiv(g.Np), FastDiv(rows), ts, cw, g.heads,
+                                          (int)b0, current_ctl().err_word);
+  }
+  return cudaGetLastError();
+}
+
+// U = upsample(O_p) rounded to bf16, raster rows; one thread per 8 channels
+// of a row (bf16 halves the restoring convolution's staging traffic; O_p is
+// bf16 already).
+__global__ void __launch_bounds__(256) upsample_raster_kernel(UpParams p, FastDiv per_row, FastDiv n_rows,
+                                                               const uint4* __restrict__ op, uint4* __restrict__ u,
+                                                               uint32_t total) {
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const uint32_t row = per_row.div(i);
+    const uint32_t c = i - row * p.vpr;
+    const uint32_t bh = n_rows.div(row);
+    const uint32_t n = row - bh * p.N;  // raster token
+    const uint32_t ty = p.rp.W.div(n);
+    const uint32_t x = n - ty * p.rp.Ww;
+    const uint32_t t = p.rp.H.div(ty);
+    const uint32_t y = ty - t * p.rp.Hh;
+    const Interp it = interp_of(t, p.pt, p.PT), iy = interp_of(y, p.ph, p.PH), ix = interp_of(x, p.pw, p.PW);
+    const uint4* base = op + (size_t)bh * p.Np * p.vpr + c;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const float w = (a ? it.f : 1.f - it.f) * (b ? iy.f : 1.f - iy.f) * (cc ? ix.f : 1.f - ix.f);
+          if (w == 0.f) continue;
+          const int src = ((a ? it.i1 : it.i0) * p.PH + (b ? iy.i1 : iy.i0)) * p.PW + (cc ? ix.i1 : ix.i0);
+          const uint4 v = __ldg(base + (size_t)src * p.vpr);
+          const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += w * bf16lo(vv[e]);
+            acc[2 * e + 1] += w * bf16hi(vv[e]);
+          }
+        }
+    u[(size_t)row * p.vpr + c] = make_uint4(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]),
+                                            pack_bf16(acc[4], acc[5]), pack_bf16(acc[6], acc[7]));
+  }
+}
+
+// O[tok] = g*O_l[tok] + (1 - g)*conv3(U)[tok], tile-major out.  conv3: sum
+// over the 27 taps (a, b, e) of w3[h][tap][c] * U[t + a, y + b, x + e][c],
+// zero outside the grid.  One CTA: one (batch*head, t), CONV_Y rows of
+// CONV_X voxels, CONV_C channels.  The bf16 U box it reads (3 x (CONV_Y + 2) x
+// (CONV_X + 2) voxels x CONV_C channels) is staged in shared memory, so each
+// U value is read from L2 about 4.8 times (the halo) instead of 27; each
+// thread computes CONV_Y outputs (one x, four channels) down a column, reusing
+// every tap weight and each shared-memory row for the rows it touches.
+constexpr int CONV_X = 32, CONV_Y = 4, CONV_C = 32;
+constexpr int CONV_BX = CONV_X + 2, CONV_BY = CONV_Y + 2;
+constexpr int CONV_SMEM = 3 * CONV_BY * CONV_BX * CONV_C * 2;
+
+__global__ void __launch_bounds__(256) conv3_blend_kernel(UpParams p, const __nv_bfloat16* __restrict__ u,
+                                                           const float* __restrict__ w3,
+                                                           const uint2* __restrict__ ol, const float* __restrict__ gvec,
+                                                           uint2* __restrict__ out, int tiles_x, int tiles_y,
+                                                           int chunks_c) {
+  extern __shared__ uint2 box[];  // [3][CONV_BY][CONV_BX][CONV_C / 4]: 4 bf16 channels each
+  const int T = (int)p.rp.T, H = (int)p.rp.Hh, W = (int)p.rp.Ww;
+  const int d = (int)p.vpr * 8;
+  const uint32_t bh = blockIdx.y;
+  int rest = blockIdx.x;
+  const int cchunk = rest % chunks_c;
+  rest /= chunks_c;
+  const int xt = rest % tiles_x;
+  rest /= tiles_x;
+  const int yt = rest % tiles_y;
+  const int t = rest / tiles_y;
+  const int x0 = xt * CONV_X, y0 = yt * CONV_Y, c0 = cchunk * CONV_C;
+  const __nv_bfloat16* ub = u + (size_t)bh * p.N * d + c0;
+  // stage the box: voxel (a, b, e) of the box holds U[t - 1 + a, y0 - 1 + b, x0 - 1 + e], zero outside
+  constexpr int NV4 = 3 * CONV_BY * CONV_BX * (CONV_C / 4);
+  for (int i = threadIdx.x; i < NV4; i += blockDim.x) {
+    const int q = i % (CONV_C / 4);
+    const int vox = i / (CONV_C / 4);
+    const int e = vox % CONV_BX, b = (vox / CONV_BX) % CONV_BY, a = vox / (CONV_BX * CONV_BY);
+    const int ts = t - 1 + a, ys = y0 - 1 + b, xs = x0 - 1 + e;
+    uint2 v = make_uint2(0u, 0u);
+    if (ts >= 0 && ts < T && ys >= 0 && ys < H && xs >= 0 && xs < W)
+      v = __ldg(reinterpret_cast<const uint2*>(ub + ((size_t)(ts * H + ys) * W + xs) * d) + q);
+    box[i] = v;
+  }
+  __syncthreads();
+  const int q = threadIdx.x % (CONV_C / 4);   // channel quad
+  const int xl = threadIdx.x / (CONV_C / 4);  // 0 .. CONV_X - 1
+  const int x = x0 + xl;
+  const float* wb = w3 + (size_t)((int)(bh + p.bh_offset) % p.heads) * 27 * d + c0 + q * 4;
+  float4 acc[CONV_Y];
+#pragma unroll
+  for (int r = 0; r < CONV_Y; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+  int tap = 0;
+#pragma unroll
+  for (int a = 0; a < 3; ++a)
+#pragma unroll
+    for (int b = 0; b < 3; ++b)
+#pragma unroll
+      for (int e = 0; e < 3; ++e, ++tap) {
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(wb + (size_t)tap * d));
+#pragma unroll
+        for (int r = 0; r < CONV_Y; ++r) {
+          const uint2 uv = box[((a * CONV_BY + r + b) * CONV_BX + xl + e) * (CONV_C / 4) + q];
+          acc[r].x = fmaf(wv.x, bf16lo(uv.x), acc[r].x);
+          acc[r].y = fmaf(wv.y, bf16hi(uv.x), acc[r].y);
+          acc[r].z = fmaf(wv.z, bf16lo(uv.y), acc[r].z);
+          acc[r].w = fmaf(wv.w, bf16hi(uv.y), acc[r].w);
+        }
+      }
+  if (x >= W) return;
+  const float gh = gvec[(bh + p.bh_offset) % p.heads];
+  const uint32_t v2 = p.vpr * 2;  // 8-byte (4-channel) vectors per row
+#pragma unroll
+  for (int r = 0; r < CONV_Y; ++r) {
+    const int y = y0 + r;
+    if (y >= H) break;
+    const size_t row = (size_t)bh * p.N + coords_to_tiled(p.rp, (uint32_t)t, (uint32_t)y, (uint32_t)x);
+    const size_t idx = row * v2 + (c0 >> 2) + q;
+    const uint2 l = __ldg(ol + idx);
+    out[idx] = make_uint2(pack_bf16(gh * bf16lo(l.x) + (1.f - gh) * acc[r].x, gh * bf16hi(l.x) + (1.f - gh) * acc[r].y),
+                          pack_bf16(gh * bf16lo(l.y) + (1.f - gh) * acc[r].z, gh * bf16hi(l.y) + (1.f - gh) * acc[r].w));
+  }
+}
+
+cudaError_t launch_upsample_conv3_blend(const DevGeom& g, const void* o_p, void* u, const float* w3,
+                                        const void* o_l, const float* gvec, void* out, cudaStream_t st) {
+  const UpParams p = make_up_params(g);
+  const long long bh_total = (long long)g.B * g.heads;
+  const long long per_bh8 = (long long)g.N * p.vpr;
+  if (per_bh8 * bh_total == 0) return cudaSuccess;
+  if (g.d % CONV_C != 0) return cudaErrorInvalidValue;
+  const int tiles_x = (g.W + CONV_X - 1) / CONV_X, tiles_y = (g.H + CONV_Y - 1) / CONV_Y, chunks_c = g.d / CONV_C;
+  const long long ctas = (long long)g.T * tiles_y * tiles_x * chunks_c;
+  if (ctas >= (1ll << 31)) return cudaErrorInvalidValue;
+  const long long chunk = ((1ll << 31) - 1) / per_bh8;
+  if (chunk < 1) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(conv3_blend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CONV_SMEM);
+  if (e != cudaSuccess) return e;
+  for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
+    const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
+    UpParams q = p;
+    q.bh_offset = (int)b0;
+    const size_t pooled = (size_t)b0 * g.Np * p.vpr, full8 = (size_t)b0 * g.N * p.vpr;
+    const uint32_t total8 = (uint32_t)(nb * per_bh8);
+    upsample_raster_kernel<<<grid_for(total8, 256), 256, 0, st>>>(q, FastDiv(p.vpr), FastDiv(g.N),
+                                                                 (const uint4*)o_p + pooled, (uint4*)u + full8,
+                                                                 total8);
+    for (long long b1 = 0; b1 < nb; b1 += 65535) {  // grid.y limit
+      const long long nb1 = nb - b1 < 65535 ? nb - b1 : 65535;
+      UpParams q1 = q;
+      q1.bh_offset = (int)(b0 + b1);
+      const size_t off8 = full8 + (size_t)b1 * g.N * p.vpr;
+      conv3_blend_kernel<<<dim3((unsigned)ctas, (unsigned)nb1), 256, CONV_SMEM, st>>>(
+          q1, (const __nv_bfloat16*)u + 8 * off8, w3, (const uint2*)o_l + 2 * off8, gvec, (uint2*)out + 2 * off8,
+          tiles_x, tiles_y,
+          chunks_c);
+    }
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_upsample_transpose(const DevGeom& g, const void* dout, const float* gvec, void* dop,
                                       cudaStream_t st) {
   const UpParams p = make_up_params(g);

@@ -344,6 +344,22 @@ static SymFwdWs sym_fwd_ws(const DevGeom& g) {
   w.total = w.o_p + pooled;
   return w;
 }
+struct SymLearnedWs {
+  size_t o_l, qp, kp, vp, o_p, u, total;
+};
+static SymLearnedWs sym_learned_ws(const DevGeom& g) {
+  SymLearnedWs w;
+  const SymFwdWs f = sym_fwd_ws(g);
+  const size_t bh = (size_t)g.B * g.heads;
+  w.o_l = f.o_l;
+  w.qp = f.qp;
+  w.kp = f.kp;
+  w.vp = f.vp;
+  w.o_p = f.o_p;
+  w.u = f.total;
+  w.total = w.u + align256(bh * g.N * g.d * 2);
+  return w;
+}
 struct SymBwdWs {
   size_t dop, ndelta_l, nlse2_l, ndelta_p, nlse2_p, dkp, dvp, dqp, total;
 };
@@ -611,6 +627,7 @@ int vattn_workspace_size(int op, const vattn_geom* geom, size_t* bytes) {
     case VATTN_OP_DUAL_BWD: *bytes = bwd_ws(g, true).total; break;
     case VATTN_OP_DUAL_SYM_FWD: *bytes = sym_fwd_ws(g).total; break;
     case VATTN_OP_DUAL_SYM_BWD: *bytes = sym_bwd_ws(g).total; break;
+    case VATTN_OP_DUAL_SYM_LEARNED_FWD: *bytes = sym_learned_ws(g).total; break;
     case VATTN_OP_STA_FWD_HOST: *bytes = host_chunk_ws(g).total; break;
     case VATTN_OP_HIER_FWD: *bytes = hier_fwd_ws(g).total; break;
     case VATTN_OP_HIER_BWD: *bytes = hier_bwd_ws(g).total; break;
@@ -1202,6 +1219,57 @@ int vattn_dual_sym_fwd(const vattn_geom* geom, const void* q, const void* k, con
   b.scale = scale;
   CHECK_LAUNCH(launch_attn_fwd(pooled_as_tokens(g), FWD_GLOBAL, b, st), "dual_sym_fwd pooled attention launch");
   CHECK_LAUNCH(launch_upsample_blend(g, o_p, o_l, gvec, o, st), "dual_sym_fwd upsample launch");
+  return ok();
+}
+
+int vattn_dual_sym_learned_fwd(const vattn_geom* geom, const void* q, const void* k, const void* v,
+                               const float* gvec, const float* wq, const float* wk, const float* wv,
+                               const float* w3, float scale, void* o, void* workspace, size_t ws_bytes,
+                               void* stream) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_POOL | NEED_ATTN, &g);
+  if (r) return r;
+  if (empty_geom(g)) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(k);
+  REQUIRE_PTR(v);
+  REQUIRE_PTR(gvec);
+  REQUIRE_PTR(wq);
+  REQUIRE_PTR(wk);
+  REQUIRE_PTR(wv);
+  REQUIRE_PTR(w3);
+  REQUIRE_PTR(o);
+  if (g.d % 8 != 0) return fail(VATTN_ERR_SHAPE, "head_dim %d is not a multiple of 8", g.d);
+  if (!aligned16(wq) || !aligned16(wk) || !aligned16(wv) || !aligned16(w3))
+    return fail(VATTN_ERR_ALIGN, "weights are not 16-byte aligned");
+  const SymLearnedWs w = sym_learned_ws(g);
+  if (!workspace || ws_bytes < w.total)
+    return fail(VATTN_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", w.total, workspace ? ws_bytes : 0);
+  if (!aligned16(workspace)) return fail(VATTN_ERR_ALIGN, "workspace is not 16-byte aligned");
+  uint8_t* ws = (uint8_t*)workspace;
+  void* o_l = ws + w.o_l;
+  void* qp = ws + w.qp;
+  void* kp = ws + w.kp;
+  void* vp = ws + w.vp;
+  void* o_p = ws + w.o_p;
+  void* u = ws + w.u;
+  cudaStream_t st = (cudaStream_t)stream;
+  CHECK_LAUNCH(launch_compress_qkv(g, q, k, v, wq, wk, wv, qp, kp, vp, st), "dual_sym_learned_fwd compress launch");
+  FwdArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o_l;
+  a.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(g, FWD_STA, a, st), "dual_sym_learned_fwd local launch");
+  FwdArgs b{};
+  b.q = qp;
+  b.k = kp;
+  b.v = vp;
+  b.o = o_p;
+  b.scale = scale;
+  CHECK_LAUNCH(launch_attn_fwd(pooled_as_tokens(g), FWD_GLOBAL, b, st), "dual_sym_learned_fwd pooled attention launch");
+  CHECK_LAUNCH(launch_upsample_conv3_blend(g, o_p, u, w3, o_l, gvec, o, st), "dual_sym_learned_fwd restore launch");
   return ok();
 }
 

@@ -68,6 +68,14 @@ cudaError_t launch_pool_qkv(const DevGeom& g, const void* q, const void* k, cons
                             void* vp, cudaStream_t st);
 cudaError_t launch_upsample_blend(const DevGeom& g, const void* o_p, const void* o_l, const float* gvec, void* out,
                                   cudaStream_t st);
+// Learned symmetric branch: depthwise strided compression of Q, K, V
+// (weights [heads][p_t*p_h*p_w][d] fp32), and upsampling into the bf16 raster
+// field u followed by the 3x3x3 depthwise restoration (w3 [heads][27][d]) and
+// the blend with o_l.
+cudaError_t launch_compress_qkv(const DevGeom& g, const void* q, const void* k, const void* v, const float* wq,
+                                const float* wk, const float* wv, void* qp, void* kp, void* vp, cudaStream_t st);
+cudaError_t launch_upsample_conv3_blend(const DevGeom& g, const void* o_p, void* u, const float* w3,
+                                        const void* o_l, const float* gvec, void* out, cudaStream_t st);
 cudaError_t launch_upsample_transpose(const DevGeom& g, const void* dout, const float* gvec, void* dop,
                                       cudaStream_t st);
 
