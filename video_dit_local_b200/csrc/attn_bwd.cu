@@ -366,6 +366,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const bool full_blk = valid >= 64;   // uniform: the last block, or a masked one
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
+        if (PAIR && valid <= 0) {  // whole block outside this warp's window: P = dS = 0, no exponentials
+          const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tmem_st16(tS + hh * 16, z);
+          tmem_st16(tP + hh * 16, z);
+          continue;
+        }
         // one 32-column half at a time keeps S, dP and the packed outputs in registers
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + hh * 32, sv);
@@ -700,6 +706,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int hh = 0; hh < DQ_BN / 32; ++hh) {
         const bool dropped = (drop >> hh) & 1u;
+        if (PAIR && dropped) {  // chunk outside this warp's window: dS = 0, no exponentials
+          const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tmem_st16(tP + hh * 16, z);
+          continue;
+        }
         // one 32-column chunk at a time: S, dP and the packed dS stay in registers
         uint32_t sv[32], dv[32];
         tmem_ld32(tS + hh * 32, sv);
@@ -716,7 +727,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (cc >= valid) o2.x = 0.f;
             if (cc + 1 >= valid) o2.y = 0.f;
           }
-          if (dropped) o2 = make_float2(0.f, 0.f);
           dk[c] = pack_bf16(o2.x, o2.y);
         }
         tmem_st16(tP + hh * 16, dk);
