@@ -914,6 +914,20 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
 
 }  // namespace bwd
 
+// Blocks per batch*head slice of the preprocess: the whole launch one wave of
+// 8 resident 256-thread blocks per SM, each block's loop striding over its
+// slice (a launch of several partial waves left the HBM idle in its tail).
+static int preprocess_blocks(const DevGeom& g, long long bh) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rows_per_block = 256 / (g.d / 8);
+  long long blocks = (long long)sms * 8 / (bh > 0 ? bh : 1);
+  const long long need = (g.N + rows_per_block - 1) / rows_per_block;
+  if (blocks > need) blocks = need;
+  return (int)(blocks < 1 ? 1 : blocks);
+}
+
 cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual, cudaStream_t st) {
   const long long bh = (long long)g.B * g.heads;
   if (bh == 0 || g.N == 0) return cudaSuccess;
@@ -936,10 +950,7 @@ cudaError_t launch_bwd_preprocess(const DevGeom& g, const BwdArgs& a, bool dual,
   pa.vpr = g.d / 8;
   pa.N = g.N;
   pa.heads = g.heads;
-  const int rows_per_block = 256 / pa.vpr;
-  int blocks = (g.N + rows_per_block - 1) / rows_per_block;
-  if (blocks > 64) blocks = 64;
-  bwd::bwd_preprocess_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>(pa);
+  bwd::bwd_preprocess_kernel<<<dim3(preprocess_blocks(g, bh), (unsigned)bh), 256, 0, st>>>(pa);
   return cudaGetLastError();
 }
 
@@ -962,10 +973,7 @@ cudaError_t launch_preprocess_branch(const DevGeom& g, const void* dout, const v
   pa.vpr = g.d / 8;
   pa.N = g.N;
   pa.heads = g.heads;
-  const int rows_per_block = 256 / pa.vpr;
-  int blocks = (g.N + rows_per_block - 1) / rows_per_block;
-  if (blocks > 64) blocks = 64;
-  bwd::bwd_preprocess_kernel<<<dim3(blocks, (unsigned)bh), 256, 0, st>>>(pa);
+  bwd::bwd_preprocess_kernel<<<dim3(preprocess_blocks(g, bh), (unsigned)bh), 256, 0, st>>>(pa);
   return cudaGetLastError();
 }
 
