@@ -151,6 +151,14 @@ def test_kernel_geometry_matches_oracle_inverse_ranges():
                 assert range(s, s + min(w, n)) == O.window_range(a, w, n)
 
 
+CONSTANTS = ["VATTN_OK", "VATTN_ERR_INVALID_ARG", "VATTN_ERR_SHAPE", "VATTN_ERR_UNSUPPORTED", "VATTN_ERR_ALIGN",
+             "VATTN_ERR_CUDA", "VATTN_ERR_DEVICE_TIMEOUT", "VATTN_ERR_WORKSPACE", "VATTN_ERR_DEVICE_BOUNDS",
+             "VATTN_OP_DUAL_FWD", "VATTN_OP_STA_BWD", "VATTN_OP_DUAL_BWD", "VATTN_OP_DUAL_SYM_FWD",
+             "VATTN_OP_DUAL_SYM_BWD", "VATTN_OP_STA_FWD_HOST", "VATTN_OP_HIER_FWD", "VATTN_OP_HIER_BWD",
+             "VATTN_OP_STA_FWD_FP8", "VATTN_OP_DUAL_FWD_FP8", "VATTN_OP_DUAL_SYM_LEARNED_FWD",
+             "VATTN_DEBUG_SKIP_ARRIVAL"]
+
+
 def test_header_is_plain_c_and_links(V, tmp_path):
     """include/vattn.h compiles as C99 (no C++ or torch types in the
     signatures) and a C program links against the library; the constants the
@@ -170,7 +178,8 @@ def test_header_is_plain_c_and_links(V, tmp_path):
         "  int r = vattn_workspace_size(VATTN_OP_DUAL_FWD, &g, &bytes);\n"
         '  printf("%d %zu %s\\n", r, bytes, vattn_version());\n'
         '  printf("%llu\\n", (unsigned long long)VATTN_NOALLOC_SCRATCH_BYTES);\n'
-        "  return r;\n"
+        + "".join(f'  printf("%lld\\n", (long long){c});\n' for c in CONSTANTS)
+        + "  return r;\n"
         "}\n")
     exe = tmp_path / "use_vattn"
     lib_dir = os.path.dirname(V.binding.LIB_PATH)
@@ -180,11 +189,15 @@ def test_header_is_plain_c_and_links(V, tmp_path):
     assert r.returncode == 0, r.stderr
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, out.stderr
-    first, second = out.stdout.strip().split("\n")
+    lines = out.stdout.strip().split("\n")
+    first, second, rest = lines[0], lines[1], lines[2:]
     code, nbytes, version = first.split(maxsplit=2)
     assert code == "0" and int(nbytes) > 0 and "sm_100a" in version
-    # the binding's copy of the header's scratch limit
+    # the binding's copies of the header's scratch limit, status codes and ops
     assert int(second) == V.binding.VATTN_NOALLOC_SCRATCH_BYTES
+    assert len(rest) == len(CONSTANTS)
+    for name, value in zip(CONSTANTS, rest):
+        assert int(value) == getattr(V.binding, name), name
 
 
 def test_null_pointers_rejected_before_any_launch(V):
