@@ -67,6 +67,7 @@ def _run_dual(V, w, check):
     ((6, 16, 24), (3, 8, 8), (1, 1, 3), (1, 4, 4), 128, 1, 2),     # tile 192: half-empty second block
     ((6, 16, 32), (6, 8, 8), (1, 3, 3), (3, 4, 4), 64, 1, 1),      # tile 384, temporal pooling
     ((3, 16, 40), (3, 8, 8), (1, 3, 3), (1, 2, 2), 128, 1, 2),     # tile 192, 5 along w: paired dQ query blocks
+    ((3, 16, 48), (3, 8, 8), (1, 2, 3), (1, 2, 2), 64, 2, 1),      # paired, d = 64, batch 2, even window along h
 ])
 def test_dual_bwd_small_full(V, grid, tile, window, pool, d, batch, heads):
     w = S.small_workload("dbwd", 17, batch, heads, d, grid, tile, window, pool)
