@@ -67,6 +67,7 @@ def _check(w, o_r, lse_r, check, tiles):
     ((4, 16, 16), (1, 4, 4), (3, 1, 1), (2, 2, 2), 64, 2, 1),    # pooled in time too, d = 64, batch 2
     ((4, 8, 16), (2, 4, 4), (1, 1, 3), (1, 1, 1), 128, 1, 1),    # h_pool 1: every local key twice
     ((2, 16, 48), (2, 8, 8), (1, 1, 1), (1, 2, 3), 128, 1, 2),   # window of one tile, uneven factors
+    ((3, 8, 144), (3, 8, 8), (1, 1, 3), (1, 1, 3), 128, 1, 1),   # 192-row tiles paired; coarse windows a tile apart
 ])
 def test_hier_fwd_small_full(V, grid, tile, window, hpool, d, batch, heads):
     w = S.small_workload("hier", 61, batch, heads, d, grid, tile, window, hpool)
@@ -130,6 +131,7 @@ def _hier_fwd_bwd(V, w, check):
     ((4, 16, 16), (1, 4, 4), (3, 1, 1), (2, 2, 2), 64, 2, 1),
     ((2, 16, 48), (2, 8, 8), (1, 1, 1), (1, 2, 3), 128, 1, 1),
     ((6, 32, 48), (3, 8, 8), (1, 3, 3), (1, 2, 3), 128, 1, 1),   # fine windows clamp in H and W
+    ((3, 8, 144), (3, 8, 8), (1, 1, 3), (1, 1, 3), 128, 1, 1),   # paired dQ query blocks over coarse windows
 ])
 def test_hier_bwd_small_full(V, grid, tile, window, hpool, d, batch, heads):
     w = S.small_workload("hier_bwd", 63, batch, heads, d, grid, tile, window, hpool)
