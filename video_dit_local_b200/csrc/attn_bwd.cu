@@ -12,13 +12,18 @@
 //
 // Kernels:
 //   bwd_preprocess_kernel  D_l, D_g (and dg) from dO, O_l, O_g        HBM-bound
-//   dkdv_kernel<D>         one CTA per 128 keys; streams 64-query blocks:
+//   dkdv_kernel<D, PAIR>   one CTA per 128 keys; streams 64-query blocks:
 //                          GLOBAL  -> all queries vs pooled keys, fp32 dK_p/dV_p
 //                          LOCAL   -> the query tiles whose window holds the key
 //                                     tile ("inverse window"), pool-backward
-//                                     fused into the epilogue
-//   dq_kernel<D>           one CTA per 128 queries; streams 64-key blocks of the
-//                          kept window, then (dual) of all pooled keys
+//                                     fused into the epilogue; PAIR: key blocks
+//                                     of two w-adjacent 192-row tiles shared
+//                          HIER    -> coarse keys, fp32 dK_h/dV_h
+//   dq_kernel<D, PAIR>     one CTA per 128 queries; streams 96-key blocks:
+//                          GLOBAL  -> all pooled keys, fp32 partial dQ out
+//                          LOCAL   -> the kept window, adding the global part;
+//                                     PAIR: query blocks shared as in the forward
+//                          HIER    -> the coarse window, fp32 partial dQ out
 // TMEM holds S/dP double-buffered per softmax group plus the accumulators;
 // P and dS are written back as bf16 over their own S/dP columns and read by
 // the next MMAs as the A operand.  No atomics: dQ, dK and dV are

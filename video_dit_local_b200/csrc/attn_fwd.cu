@@ -1,8 +1,10 @@
 // Attention forward on tcgen05 tensor cores, one kernel for both branches:
 //  - FWD_STA: sliding-tile attention ("Fast Video Generation with Sliding Tile
-//    Attention", abstract).  The query block lies inside one query tile; its
-//    key stream is the box of kept tiles, computed here from the tile
-//    coordinate, so masked tiles are never loaded.
+//    Attention", abstract).  The query block lies inside one query tile, or
+//    (PAIR instance, tile volumes an odd multiple of 64 rows) straddles two
+//    w-adjacent tiles (PairPlan, common.cuh); its key stream is the box of
+//    kept tiles (for a straddling block the union of the two windows),
+//    computed here from the tile coordinate, so masked tiles are never loaded.
 //  - FWD_GLOBAL: every query attends to all pooled keys ("UltraGen ..." §4.2),
 //    with an optional blend epilogue O = g*O_local + (1-g)*O_global (§4.1).
 //
