@@ -52,6 +52,9 @@ def _xwin_tiles(q, k, v, g, scale, shifted, tiles):
 @pytest.mark.parametrize("grid,tile,window,d,batch,heads", [
     ((4, 16, 24), (2, 4, 4), (1, 2, 3), 64, 1, 2),
     ((6, 24, 40), (3, 8, 8), (2, 2, 2), 128, 2, 1),     # tile 192, truncated edge blocks
+    # tile 192, 9 tiles along w: partitions of 3 pair tiles 0-1, 3-4, 6-7 (a unit table), shifted blocks of 4
+    # (cuts at 2 and 6) pair every even tile with the next (uniform pairs)
+    ((3, 16, 72), (3, 8, 8), (1, 2, 3), 128, 1, 2),
 ])
 def test_xwin_fwd_bwd_small_full(V, shifted, grid, tile, window, d, batch, heads):
     import torch

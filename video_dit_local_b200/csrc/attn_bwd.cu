@@ -850,7 +850,7 @@ static cudaError_t launch_dkdv_d(const DevGeom& g, const BwdArgs& a, bool global
   p.dvp_in = (!global && dual) ? a.dvp : nullptr;
   p.ctl = current_ctl();
   const long long bh = (long long)g.B * g.heads;
-  const bool pair = p.pair.np > 0;
+  const bool pair = pair_plan_active(p.pair);
   const int blocks = p.mode == DKDV_GLOBAL ? (g.Np + 127) / 128
                      : p.mode == DKDV_HIER ? hk->n_tiles * p.kv_blocks_per_tile
                                            : (int)pair_plan_blocks(g, p.pair);
@@ -888,7 +888,7 @@ static cudaError_t launch_dq_d(const DevGeom& g, const BwdArgs& a, bool global, 
   // local and hierarchical passes: w-adjacent tiles of an odd multiple of 64
   // rows share their query blocks (PairPlan), as in the forward
   p.pair = make_pair_plan(g, p.gk.Nw, !global);
-  const bool pair = p.pair.np > 0;
+  const bool pair = pair_plan_active(p.pair);
   p.scale = a.scale;
   p.c2 = a.scale * LOG2E;
   p.nlse2 = global ? a.nlse2_g : a.nlse2_l;

@@ -613,7 +613,7 @@ static cudaError_t launch_fwd_d(const DevGeom& g, FwdMode mode, const FwdArgs& a
     // at least two tiles along w, so a straddling block's first key tile is in
     // both windows)
     p.pair = make_pair_plan(g, p.kNw, !p.raster);
-    if (p.pair.np > 0) {
+    if (pair_plan_active(p.pair)) {
       qblocks = (int)pair_plan_blocks(g, p.pair);
       pair = true;
     }

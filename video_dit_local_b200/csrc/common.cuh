@@ -400,30 +400,89 @@ struct TileBox {
 // start at most one tile apart (sliding windows); the rows of each tile mask
 // the key tile outside their own window.
 // ---------------------------------------------------------------------------
+constexpr int PAIR_MAX_UNITS = 64;  // tiles per tile row that a unit table can describe
+
 struct PairPlan {
   int k;    // whole 128-row blocks per tile (pairing only)
   int nw;   // tiles per tile row (Nw); 1 unpaired (each tile a row of its own)
   int np;   // pairs per tile row (Nw / 2); 0 unpaired
   int bpr;  // query blocks per tile row
+  // Unit table (partition windows): units > 0 replaces the uniform pairs
+  // (2i, 2i+1) by `units` units per tile row, each one tile or a pair of
+  // adjacent tiles whose windows coincide (pairs never cross a partition).
+  int units;
+  uint8_t unit_tile[PAIR_MAX_UNITS];            // first tile (w) of the unit
+  uint8_t unit_pair[PAIR_MAX_UNITS];            // 1: the unit is tiles w, w + 1
+  uint16_t unit_block[PAIR_MAX_UNITS + 1];      // first query block of the unit in its row
 };
 
+// Windows of w-adjacent tiles aw, aw + 1 coincide along w (then along t and h
+// too: a pair shares its tile row).
+inline bool windows_coincide(const DevGeom& g, int key_nw, int aw) {
+  int s0, e0, s1, e1;
+  tile_range(aw, g.ww, key_nw, g.wmode, &s0, &e0);
+  tile_range(aw + 1, g.ww, key_nw, g.wmode, &s1, &e1);
+  return s0 == s1 && e0 == e1;
+}
+
 // key_nw: tiles of the key grid along w (the query grid's, or the coarse grid
-// of the hierarchical branch).  A straddling block's first key tile must lie
-// in both windows, which needs windows of at least two tiles along w.
+// of the hierarchical branch).
+//  - Sliding windows: uniform pairs (2i, 2i+1); a straddling block streams
+//    the union of the two windows (one tile wider when they start a tile
+//    apart), whose first key tile must lie in both windows, so the windows
+//    need at least two tiles along w.
+//  - Partition windows (cross-window attention): a pair needs its two tiles
+//    in the same block, so that their windows coincide (no mask, no union).
+//    When every uniform pair does (e.g. shifted blocks of 4 whose cuts fall
+//    on even tiles), the uniform plan; otherwise a unit table built left to
+//    right (e.g. blocks of 3: tiles 0-1 paired, 2 alone, 3-4 paired, ...).
 inline PairPlan make_pair_plan(const DevGeom& g, int key_nw, bool allow) {
   PairPlan pp;
   pp.k = 0;
   pp.nw = 1;
   pp.np = 0;
   pp.bpr = (g.s + 127) / 128;
-  if (allow && g.s % 128 == 64 && g.wmode == WIN_SLIDING && win_extent(g.ww, key_nw) >= 2 && g.Nw >= 2) {
-    pp.k = g.s / 128;
+  pp.units = 0;
+  if (!allow || g.s % 128 != 64 || g.Nw < 2) return pp;
+  const int k = g.s / 128;
+  bool uniform = false;
+  if (g.wmode == WIN_SLIDING) {
+    uniform = win_extent(g.ww, key_nw) >= 2;
+  } else if (key_nw == g.Nw) {
+    uniform = true;
+    for (int aw = 0; aw + 1 < g.Nw; aw += 2) uniform = uniform && windows_coincide(g, key_nw, aw);
+    if (!uniform && g.Nw <= PAIR_MAX_UNITS) {
+      int u = 0, blocks = 0, pairs = 0;
+      for (int aw = 0; aw < g.Nw; ++u) {
+        const bool pair = aw + 1 < g.Nw && windows_coincide(g, key_nw, aw);
+        pp.unit_tile[u] = (uint8_t)aw;
+        pp.unit_pair[u] = pair ? 1 : 0;
+        pp.unit_block[u] = (uint16_t)blocks;
+        blocks += pair ? 2 * k + 1 : k + 1;
+        pairs += pair ? 1 : 0;
+        aw += pair ? 2 : 1;
+      }
+      pp.unit_block[u] = (uint16_t)blocks;
+      if (pairs > 0) {
+        pp.k = k;
+        pp.nw = g.Nw;
+        pp.units = u;
+        pp.bpr = blocks;
+      }
+      return pp;
+    }
+  }
+  if (uniform) {
+    pp.k = k;
     pp.nw = g.Nw;
     pp.np = g.Nw / 2;
     pp.bpr = pp.np * (2 * pp.k + 1) + (g.Nw % 2) * (pp.k + 1);
   }
   return pp;
 }
+// The plan pairs tiles (uniform pairs or a unit table): launch the PAIR
+// kernel instance with pair_plan_blocks query blocks.
+inline bool pair_plan_active(const PairPlan& pp) { return pp.np > 0 || pp.units > 0; }
 inline long long pair_plan_blocks(const DevGeom& g, const PairPlan& pp) {
   return (long long)(g.n_tiles / pp.nw) * pp.bpr;
 }
@@ -438,13 +497,24 @@ struct QueryBlock {
 
 __device__ __forceinline__ QueryBlock paired_query_block(const DevGeom& g, const PairPlan& pp, int qblk) {
   QueryBlock b;
-  // tile row r (unpaired: tile r), block i of it; pair pi (np: the row's odd
-  // last tile), block sb of the pair
   const int r = qblk / pp.bpr, i = qblk - r * pp.bpr;
-  const int span = 2 * pp.k + 1;
-  const int pi = min(i / span, pp.np);
-  const int a = r * pp.nw + 2 * pi, sb = i - pi * span;
-  const bool in_pair = pi < pp.np;
+  int a, sb;
+  bool in_pair;
+  if (pp.units > 0) {  // unit table: the unit holding block i of the row
+    int u = 0;
+    while (u + 1 < pp.units && pp.unit_block[u + 1] <= i) ++u;
+    a = r * pp.nw + pp.unit_tile[u];
+    sb = i - pp.unit_block[u];
+    in_pair = pp.unit_pair[u] != 0;
+  } else {
+    // tile row r (unpaired: tile r), block i of it; pair pi (np: the row's
+    // odd last tile), block sb of the pair
+    const int span = 2 * pp.k + 1;
+    const int pi = min(i / span, pp.np);
+    a = r * pp.nw + 2 * pi;
+    sb = i - pi * span;
+    in_pair = pi < pp.np;
+  }
   b.row0 = a * g.s + sb * 128;
   b.valid = min(128, (in_pair ? 2 * g.s : g.s) - sb * 128);
   b.tile = a + (in_pair && sb > pp.k ? 1 : 0);
