@@ -390,6 +390,17 @@ int vattn_debug_set(int flags, int64_t timeout_ns);
  * float32 [n]. */
 int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream);
 
+/* Test hook (host only, no device work): the 128-row query blocks of the
+ * sliding-tile forward for `geom` with window mode `window_mode` (0 sliding,
+ * 1 partition, 2 shifted partition), as the bf16 tile-major launch lays them
+ * out, including the pairing of w-adjacent tiles of an odd multiple of 64
+ * rows.  out: host int32 [capacity][4] = first row (tile-major), rows that
+ * exist, straddle flag (rows [0, 64) in `tile`, [64, 128) in `tile` + 1),
+ * tile whose window the key stream starts from.  *n_blocks receives the
+ * block count (entries past capacity are not written). */
+int vattn_debug_query_blocks(const vattn_geom* geom, int window_mode, int32_t* out, int64_t capacity,
+                             int64_t* n_blocks);
+
 /* Library version string. */
 const char* vattn_version(void);
 

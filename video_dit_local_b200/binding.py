@@ -111,6 +111,7 @@ _SIGS = {
     "vattn_shutdown": [],
     "vattn_debug_set": [_INT, _I64],
     "vattn_debug_exp2": [_P, _P, _I64, _P],
+    "vattn_debug_query_blocks": [_GP, _INT, _P, _I64, _P],
     "vattn_version": [],
 }
 
@@ -351,6 +352,18 @@ def vattn_debug_set(flags: int, timeout_ns: int = 0) -> None:
 
 def vattn_debug_exp2(x, y, n: Optional[int] = None, stream=None) -> None:
     _check(lib.vattn_debug_exp2(_ptr(x), _ptr(y), x.numel() if n is None else n, _stream(stream)))
+
+
+def vattn_debug_query_blocks(geom: Geom, window_mode: int):
+    """Host-side query-block plan of the sliding-tile forward: an int32 tensor
+    [n_blocks, 4] = (first tile-major row, rows that exist, straddle flag,
+    tile of the key stream).  window_mode: 0 sliding, 1 partition, 2 shifted."""
+    import torch
+    n = ctypes.c_int64(0)
+    _check(lib.vattn_debug_query_blocks(ctypes.byref(geom), window_mode, None, 0, ctypes.byref(n)))
+    out = torch.empty((n.value, 4), dtype=torch.int32)
+    _check(lib.vattn_debug_query_blocks(ctypes.byref(geom), window_mode, _hptr(out), n.value, ctypes.byref(n)))
+    return out
 
 
 def vattn_version() -> str:

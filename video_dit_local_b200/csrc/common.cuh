@@ -495,7 +495,7 @@ struct QueryBlock {
   int straddle;  // rows [0, 64) in tile `tile`, [64, 128) in tile `tile` + 1
 };
 
-__device__ __forceinline__ QueryBlock paired_query_block(const DevGeom& g, const PairPlan& pp, int qblk) {
+__host__ __device__ __forceinline__ QueryBlock paired_query_block(const DevGeom& g, const PairPlan& pp, int qblk) {
   QueryBlock b;
   const int r = qblk / pp.bpr, i = qblk - r * pp.bpr;
   int a, sb;
@@ -510,13 +510,14 @@ __device__ __forceinline__ QueryBlock paired_query_block(const DevGeom& g, const
     // tile row r (unpaired: tile r), block i of it; pair pi (np: the row's
     // odd last tile), block sb of the pair
     const int span = 2 * pp.k + 1;
-    const int pi = min(i / span, pp.np);
+    const int pi = i / span < pp.np ? i / span : pp.np;
     a = r * pp.nw + 2 * pi;
     sb = i - pi * span;
     in_pair = pi < pp.np;
   }
   b.row0 = a * g.s + sb * 128;
-  b.valid = min(128, (in_pair ? 2 * g.s : g.s) - sb * 128);
+  const int left = (in_pair ? 2 * g.s : g.s) - sb * 128;
+  b.valid = left < 128 ? left : 128;
   b.tile = a + (in_pair && sb > pp.k ? 1 : 0);
   b.straddle = in_pair && sb == pp.k;
   b.sub = sb;

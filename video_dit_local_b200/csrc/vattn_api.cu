@@ -568,6 +568,38 @@ int vattn_debug_exp2(const float* x, float* y, int64_t n, void* stream) {
   return ok();
 }
 
+int vattn_debug_query_blocks(const vattn_geom* geom, int window_mode, int32_t* out, int64_t capacity,
+                             int64_t* n_blocks) {
+  DevGeom g;
+  int r = build_geom(geom, NEED_TILE | NEED_ATTN, &g);
+  if (r) return r;
+  if (window_mode < WIN_SLIDING || window_mode > WIN_SHIFTED) return fail(VATTN_ERR_INVALID_ARG, "bad window mode");
+  REQUIRE_PTR(n_blocks);
+  if (capacity > 0) REQUIRE_PTR(out);
+  g.wmode = window_mode;
+  const PairPlan pp = make_pair_plan(g, g.Nw, true);
+  const int qbpt = (g.s + 127) / 128;
+  const long long n = pair_plan_active(pp) ? pair_plan_blocks(g, pp) : (long long)g.n_tiles * qbpt;
+  *n_blocks = n;
+  for (long long b = 0; b < n && b < capacity; ++b) {
+    QueryBlock qb;
+    if (pair_plan_active(pp)) {
+      qb = paired_query_block(g, pp, (int)b);
+    } else {
+      qb.tile = (int)(b / qbpt);
+      qb.sub = (int)(b - (long long)qb.tile * qbpt);
+      qb.row0 = qb.tile * g.s + qb.sub * 128;
+      qb.valid = g.s - qb.sub * 128 < 128 ? g.s - qb.sub * 128 : 128;
+      qb.straddle = 0;
+    }
+    out[4 * b] = qb.row0;
+    out[4 * b + 1] = qb.valid;
+    out[4 * b + 2] = qb.straddle;
+    out[4 * b + 3] = qb.tile;
+  }
+  return ok();
+}
+
 int vattn_get_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
