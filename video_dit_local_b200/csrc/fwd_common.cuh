@@ -22,7 +22,6 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   const __nv_bfloat16* o_local;
-  __nv_bfloat16* o_local_out;    // fused dual forward: where the local pass leaves O_local (read back by the blend)
   const float* gvec;
   __nv_bfloat16* blend_out;
   // key-side tile grid and coarse factor (STA): the sliding tile has the query
