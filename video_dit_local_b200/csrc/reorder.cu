@@ -709,16 +709,16 @@ __global__ void __launch_bounds__(256) upsample_raster_kernel(UpParams p, FastDi
 // U value is read from L2 about 4.8 times (the halo) instead of 27; each
 // thread computes CONV_Y outputs (one x, four channels) down a column, reusing
 // every tap weight and each shared-memory row for the rows it touches.
-constexpr int CONV_X = 32, CONV_Y = 4, CONV_C = 32;
+constexpr int CONV_X = 32, CONV_Y = 4, CONV_C = 32, CONV_THREADS = 256;
 constexpr int CONV_BX = CONV_X + 2, CONV_BY = CONV_Y + 2;
 constexpr int CONV_SMEM = 3 * CONV_BY * CONV_BX * CONV_C * 2;
 
-__global__ void __launch_bounds__(256) conv3_blend_kernel(UpParams p, const __nv_bfloat16* __restrict__ u,
+__global__ void __launch_bounds__(CONV_THREADS, 4) conv3_blend_kernel(UpParams p, const __nv_bfloat16* __restrict__ u,
                                                            const float* __restrict__ w3,
                                                            const uint2* __restrict__ ol, const float* __restrict__ gvec,
                                                            uint2* __restrict__ out, int tiles_x, int tiles_y,
                                                            int chunks_c) {
-  extern __shared__ uint2 box[];  // [3][CONV_BY][CONV_BX][CONV_C / 4]: 4 bf16 channels each
+  extern __shared__ __align__(16) uint2 box[];  // [3][CONV_BY][CONV_BX][CONV_C / 4]: 4 bf16 channels each
   const int T = (int)p.rp.T, H = (int)p.rp.Hh, W = (int)p.rp.Ww;
   const int d = (int)p.vpr * 8;
   const uint32_t bh = blockIdx.y;
@@ -731,17 +731,29 @@ __global__ void __launch_bounds__(256) conv3_blend_kernel(UpParams p, const __nv
   const int t = rest / tiles_y;
   const int x0 = xt * CONV_X, y0 = yt * CONV_Y, c0 = cchunk * CONV_C;
   const __nv_bfloat16* ub = u + (size_t)bh * p.N * d + c0;
-  // stage the box: voxel (a, b, e) of the box holds U[t - 1 + a, y0 - 1 + b, x0 - 1 + e], zero outside
-  constexpr int NV4 = 3 * CONV_BY * CONV_BX * (CONV_C / 4);
-  for (int i = threadIdx.x; i < NV4; i += blockDim.x) {
-    const int q = i % (CONV_C / 4);
-    const int vox = i / (CONV_C / 4);
+  // stage the box: voxel (a, b, e) of the box holds U[t - 1 + a, y0 - 1 + b, x0 - 1 + e], zero outside.
+  // 16-byte pieces; every load of a thread is issued before the first store,
+  // so a thread keeps all of them in flight at once.
+  constexpr int Q16 = CONV_C / 8;                       // 16-byte pieces per voxel
+  constexpr int NV16 = 3 * CONV_BY * CONV_BX * Q16;
+  constexpr int PER = (NV16 + CONV_THREADS - 1) / CONV_THREADS;
+  uint4 stage[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + k * CONV_THREADS;
+    const int q = i % Q16;
+    const int vox = i / Q16;
     const int e = vox % CONV_BX, b = (vox / CONV_BX) % CONV_BY, a = vox / (CONV_BX * CONV_BY);
     const int ts = t - 1 + a, ys = y0 - 1 + b, xs = x0 - 1 + e;
-    uint2 v = make_uint2(0u, 0u);
-    if (ts >= 0 && ts < T && ys >= 0 && ys < H && xs >= 0 && xs < W)
-      v = __ldg(reinterpret_cast<const uint2*>(ub + ((size_t)(ts * H + ys) * W + xs) * d) + q);
-    box[i] = v;
+    stage[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < NV16 && ts >= 0 && ts < T && ys >= 0 && ys < H && xs >= 0 && xs < W)
+      stage[k] = __ldg(reinterpret_cast<const uint4*>(ub + ((size_t)(ts * H + ys) * W + xs) * d) + q);
+  }
+  uint4* box16 = reinterpret_cast<uint4*>(box);
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + k * CONV_THREADS;
+    if (i < NV16) box16[i] = stage[k];
   }
   __syncthreads();
   const int q = threadIdx.x % (CONV_C / 4);   // channel quad
@@ -811,7 +823,7 @@ cudaError_t launch_upsample_conv3_blend(const DevGeom& g, const void* o_p, void*
       UpParams q1 = q;
       q1.bh_offset = (int)(b0 + b1);
       const size_t off8 = full8 + (size_t)b1 * g.N * p.vpr;
-      conv3_blend_kernel<<<dim3((unsigned)ctas, (unsigned)nb1), 256, CONV_SMEM, st>>>(
+      conv3_blend_kernel<<<dim3((unsigned)ctas, (unsigned)nb1), CONV_THREADS, CONV_SMEM, st>>>(
           q1, (const __nv_bfloat16*)u + 8 * off8, w3, (const uint2*)o_l + 2 * off8, gvec, (uint2*)out + 2 * off8,
           tiles_x, tiles_y,
           chunks_c);
