@@ -275,12 +275,12 @@ def run_sym_learned_only(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     peaks, _ = _peaks()
-    res = _bench_sym_learned(V, dev, peaks, n=args.steps, warm=args.warmup)
+    res = _bench_sym_learned(V, dev, peaks, n=args.steps, warm=args.warmup, heads=args.heads)
     return {"metric": METRIC, "value": res["eff_tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch N(0,1), seeded random weights)",
-            "config": {"workload": "1080p dual fwd, learned symmetric global branch: B1 h24 d128, grid 21x72x120, "
-                                   "tile 3x8x8, window 3x3x3, pool 1x4x4"}, "status": res["status"]}
+            "config": {"workload": f"1080p dual fwd, learned symmetric global branch: B1 h{args.heads or 24} d128, "
+                                   "grid 21x72x120, tile 3x8x8, window 3x3x3, pool 1x4x4"}, "status": res["status"]}
 
 
 def run_ours(args, rank, world, local_rank):
@@ -646,7 +646,7 @@ def _bench_hier(V, dev, peaks):
     return res
 
 
-def _bench_sym_learned(V, dev, peaks, n=4, warm=2):
+def _bench_sym_learned(V, dev, peaks, n=4, warm=2, heads=None):
     """Dual forward with the learned symmetric global branch (depthwise
     strided compression, 3x3x3 depthwise restoration, seeded random weights)
     at the 1080p workload; effective FLOPs as the average-pooling form (the
@@ -654,6 +654,9 @@ def _bench_sym_learned(V, dev, peaks, n=4, warm=2):
     import torch
     from synth import inputs as S
     w = S.WORKLOADS["1080p"]
+    if heads:   # reduced case for profiling only
+        import dataclasses
+        w = dataclasses.replace(w, heads=heads)
     geom = _geom(V, w)
     T, H, W = w.grid
     npool = (T // w.pool[0]) * (H // w.pool[1]) * (W // w.pool[2])

@@ -59,6 +59,8 @@ def _run(V, w, check, weights=None):
     ((4, 8, 8), (2, 4, 4), (1, 2, 2), (2, 2, 4), 64, 1, 2),       # temporal compression too
     ((3, 16, 24), (3, 8, 8), (1, 1, 3), (1, 4, 4), 128, 2, 1),    # frame-wise 4x4 compression, batch 2
     ((6, 24, 40), (3, 8, 8), (3, 3, 3), (3, 8, 8), 128, 1, 2),    # pooled grid 2x3x5 (restoration at every edge)
+    # 6 rows: the restoration's last 4-row band is half empty; 12 columns: one partial 32-column band
+    ((4, 6, 12), (2, 2, 4), (1, 2, 3), (1, 3, 4), 64, 1, 2),
 ])
 def test_dual_sym_learned_small_full(V, grid, tile, window, pool, d, batch, heads):
     w = S.small_workload("symlearn", 37, batch, heads, d, grid, tile, window, pool)
