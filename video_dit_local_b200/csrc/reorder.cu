@@ -705,21 +705,28 @@ __global__ void __launch_bounds__(256) upsample_raster_kernel(UpParams p, FastDi
 // over the 27 taps (a, b, e) of w3[h][tap][c] * U[t + a, y + b, x + e][c],
 // zero outside the grid.  One CTA: one (batch*head, t), CONV_Y rows of
 // CONV_X voxels, CONV_C channels.  The bf16 U box it reads (3 x (CONV_Y + 2) x
-// (CONV_X + 2) voxels x CONV_C channels) is staged in shared memory, so each
-// U value is read from L2 about 4.8 times (the halo) instead of 27; each
-// thread computes CONV_Y outputs (one x, four channels) down a column, reusing
-// every tap weight and each shared-memory row for the rows it touches.
+// (CONV_X + 2) voxels x CONV_C channels) arrives in shared memory by one
+// 5-D tensor-map copy (zero-filled outside the grid), so each U value is read
+// from L2 about 4.8 times (the halo) instead of 27 and no thread spends
+// instructions on staging; each thread computes CONV_Y outputs (one x, four
+// channels) down a column, reusing every tap weight and each shared-memory row
+// for the rows it touches.
 constexpr int CONV_X = 32, CONV_Y = 4, CONV_C = 32, CONV_THREADS = 256;
+constexpr int CONV_MIN_CTAS = 4;  // 64 registers: four CTAs per SM
 constexpr int CONV_BX = CONV_X + 2, CONV_BY = CONV_Y + 2;
-constexpr int CONV_SMEM = 3 * CONV_BY * CONV_BX * CONV_C * 2;
+constexpr int CONV_BOX = 3 * CONV_BY * CONV_BX * CONV_C * 2;
+constexpr int CONV_SMEM = CONV_BOX + 16 + 128;  // box, barrier and abort flag, alignment slack
 
-__global__ void __launch_bounds__(CONV_THREADS, 4) conv3_blend_kernel(UpParams p, const __nv_bfloat16* __restrict__ u,
-                                                           const float* __restrict__ w3,
-                                                           const uint2* __restrict__ ol, const float* __restrict__ gvec,
-                                                           uint2* __restrict__ out, int tiles_x, int tiles_y,
-                                                           int chunks_c) {
-  extern __shared__ __align__(16) uint2 box[];  // [3][CONV_BY][CONV_BX][CONV_C / 4]: 4 bf16 channels each
-  const int T = (int)p.rp.T, H = (int)p.rp.Hh, W = (int)p.rp.Ww;
+__global__ void __launch_bounds__(CONV_THREADS, CONV_MIN_CTAS)
+    conv3_blend_kernel(const __grid_constant__ CUtensorMap tm_u, UpParams p, const float* __restrict__ w3,
+                       const uint2* __restrict__ ol, const float* __restrict__ gvec, uint2* __restrict__ out,
+                       int tiles_x, int tiles_y, int chunks_c, DevCtl ctl) {
+  extern __shared__ __align__(128) uint8_t conv_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(conv_raw) + 127) & ~uintptr_t(127));
+  const uint2* box = reinterpret_cast<const uint2*>(sm);  // [3][CONV_BY][CONV_BX][CONV_C / 4]: 4 bf16 channels each
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + CONV_BOX);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + CONV_BOX + 8);
+  const int H = (int)p.rp.Hh, W = (int)p.rp.Ww;
   const int d = (int)p.vpr * 8;
   const uint32_t bh = blockIdx.y;
   int rest = blockIdx.x;
@@ -730,32 +737,27 @@ __global__ void __launch_bounds__(CONV_THREADS, 4) conv3_blend_kernel(UpParams p
   const int yt = rest % tiles_y;
   const int t = rest / tiles_y;
   const int x0 = xt * CONV_X, y0 = yt * CONV_Y, c0 = cchunk * CONV_C;
-  const __nv_bfloat16* ub = u + (size_t)bh * p.N * d + c0;
-  // stage the box: voxel (a, b, e) of the box holds U[t - 1 + a, y0 - 1 + b, x0 - 1 + e], zero outside.
-  // 16-byte pieces; every load of a thread is issued before the first store,
-  // so a thread keeps all of them in flight at once.
-  constexpr int Q16 = CONV_C / 8;                       // 16-byte pieces per voxel
-  constexpr int NV16 = 3 * CONV_BY * CONV_BX * Q16;
-  constexpr int PER = (NV16 + CONV_THREADS - 1) / CONV_THREADS;
-  uint4 stage[PER];
-#pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int i = threadIdx.x + k * CONV_THREADS;
-    const int q = i % Q16;
-    const int vox = i / Q16;
-    const int e = vox % CONV_BX, b = (vox / CONV_BX) % CONV_BY, a = vox / (CONV_BX * CONV_BY);
-    const int ts = t - 1 + a, ys = y0 - 1 + b, xs = x0 - 1 + e;
-    stage[k] = make_uint4(0u, 0u, 0u, 0u);
-    if (i < NV16 && ts >= 0 && ts < T && ys >= 0 && ys < H && xs >= 0 && xs < W)
-      stage[k] = __ldg(reinterpret_cast<const uint4*>(ub + ((size_t)(ts * H + ys) * W + xs) * d) + q);
-  }
-  uint4* box16 = reinterpret_cast<uint4*>(box);
-#pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int i = threadIdx.x + k * CONV_THREADS;
-    if (i < NV16) box16[i] = stage[k];
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
   __syncthreads();
+  // voxel (a, b, e) of the box holds U[t - 1 + a, y0 - 1 + b, x0 - 1 + e]; the
+  // innermost coordinate c0 is a multiple of 32 channels (64 bytes)
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, CONV_BOX);
+    tma_load_5d(sm, &tm_u, bar, c0, x0 - 1, y0 - 1, t - 1, (int)bh);
+  }
+  WaitCtx wc;
+  wc.abort_flag = abort_flag;
+  wc.timeout_ns = ctl.timeout_ns;
+  wc.err_word = ctl.err_word;
+  const bool landed = __syncthreads_and(mbar_wait(bar, 0, wc));
+  if (!landed) {  // let the copy in flight finish before the CTA releases its shared memory
+    if (threadIdx.x == 0) mbar_wait_drain(bar, 0, wc);
+    return;
+  }
   const int q = threadIdx.x % (CONV_C / 4);   // channel quad
   const int xl = threadIdx.x / (CONV_C / 4);  // 0 .. CONV_X - 1
   const int x = x0 + xl;
@@ -809,8 +811,10 @@ cudaError_t launch_upsample_conv3_blend(const DevGeom& g, const void* o_p, void*
   if (chunk < 1) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(conv3_blend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CONV_SMEM);
   if (e != cudaSuccess) return e;
+  const DevCtl ctl = current_ctl();
   for (long long b0 = 0; b0 < bh_total; b0 += chunk) {
     const long long nb = bh_total - b0 < chunk ? bh_total - b0 : chunk;
+    if (nb > 65535) return cudaErrorInvalidValue;  // grid.y; batch*heads < 65536 is checked up front
     UpParams q = p;
     q.bh_offset = (int)b0;
     const size_t pooled = (size_t)b0 * g.Np * p.vpr, full8 = (size_t)b0 * g.N * p.vpr;
@@ -818,16 +822,12 @@ cudaError_t launch_upsample_conv3_blend(const DevGeom& g, const void* o_p, void*
     upsample_raster_kernel<<<grid_for(total8, 256), 256, 0, st>>>(q, FastDiv(p.vpr), FastDiv(g.N),
                                                                  (const uint4*)o_p + pooled, (uint4*)u + full8,
                                                                  total8);
-    for (long long b1 = 0; b1 < nb; b1 += 65535) {  // grid.y limit
-      const long long nb1 = nb - b1 < 65535 ? nb - b1 : 65535;
-      UpParams q1 = q;
-      q1.bh_offset = (int)(b0 + b1);
-      const size_t off8 = full8 + (size_t)b1 * g.N * p.vpr;
-      conv3_blend_kernel<<<dim3((unsigned)ctas, (unsigned)nb1), CONV_THREADS, CONV_SMEM, st>>>(
-          q1, (const __nv_bfloat16*)u + 8 * off8, w3, (const uint2*)o_l + 2 * off8, gvec, (uint2*)out + 2 * off8,
-          tiles_x, tiles_y,
-          chunks_c);
-    }
+    CUtensorMap tm;
+    const char* err = nullptr;
+    if (!make_tmap_conv_box(&tm, (const uint4*)u + full8, g.d, g, nb, CONV_C, CONV_BX, CONV_BY, 3, &err))
+      return cudaErrorInvalidValue;
+    conv3_blend_kernel<<<dim3((unsigned)ctas, (unsigned)nb), CONV_THREADS, CONV_SMEM, st>>>(
+        tm, q, w3, (const uint2*)o_l + 2 * full8, gvec, (uint2*)out + 2 * full8, tiles_x, tiles_y, chunks_c, ctl);
   }
   return cudaGetLastError();
 }

@@ -195,6 +195,31 @@ bool make_tmap_raster(CUtensorMap* map, const void* base, int d, const DevGeom& 
   return true;
 }
 
+// Raster [bh][T][H][W][d] bf16 as a 5-D map with an unswizzled box of
+// box_c channels x box_x x box_y x box_t voxels of one slice: the box lands in
+// shared memory densely, channels fastest, and reads zeros outside the grid.
+bool make_tmap_conv_box(CUtensorMap* map, const void* base, int d, const DevGeom& g, long long bh, int box_c,
+                        int box_x, int box_y, int box_t, const char** err) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    *err = "cuTensorMapEncodeTiled unavailable";
+    return false;
+  }
+  const cuuint64_t row = (cuuint64_t)d * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T, (cuuint64_t)bh};
+  cuuint64_t strides[4] = {row, row * g.W, row * g.W * g.H, row * g.W * g.H * g.T};
+  cuuint32_t box[5] = {(cuuint32_t)box_c, (cuuint32_t)box_x, (cuuint32_t)box_y, (cuuint32_t)box_t, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *err = "cuTensorMapEncodeTiled failed";
+    return false;
+  }
+  return true;
+}
+
 // The same for rows of `d` bytes (e4m3): box = 128 bytes x box_rows x 1.
 bool make_tmap_rows_u8(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                        const char** err) {

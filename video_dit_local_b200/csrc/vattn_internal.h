@@ -169,6 +169,10 @@ bool make_tmap_rows(CUtensorMap* map, const void* base, int d, long long rows_pe
 // tile-w x tile-h x box_t t-slices x 1, 128-byte swizzle.
 bool make_tmap_raster(CUtensorMap* map, const void* base, int d, const DevGeom& g, long long bh, int box_t,
                       const char** err);
+// 5-D map over a raster [bh][T][H][W][d] bf16 tensor with an unswizzled box of
+// box_c channels x box_x x box_y x box_t voxels x 1 (zeros outside the grid).
+bool make_tmap_conv_box(CUtensorMap* map, const void* base, int d, const DevGeom& g, long long bh, int box_c,
+                        int box_x, int box_y, int box_t, const char** err);
 bool make_tmap_rows_u8(CUtensorMap* map, const void* base, int d, long long rows_per_bh, long long bh, int box_rows,
                        const char** err);
 
