@@ -708,9 +708,10 @@ __global__ void __launch_bounds__(256) upsample_raster_kernel(UpParams p, FastDi
 // (CONV_X + 2) voxels x CONV_C channels) arrives in shared memory by one
 // 5-D tensor-map copy (zero-filled outside the grid), so each U value is read
 // from L2 about 4.8 times (the halo) instead of 27 and no thread spends
-// instructions on staging; each thread computes CONV_Y outputs (one x, four
-// channels) down a column, reusing every tap weight and each shared-memory row
-// for the rows it touches.
+// instructions on staging.  Each thread computes CONV_Y outputs (one x, four
+// channels) down a column: per (t offset a, x offset e) it holds the three
+// y-taps' weights and reads each of the CONV_Y + 2 box rows once, unpacked
+// once and applied to every output row it feeds (sum order a, e, b).
 constexpr int CONV_X = 32, CONV_Y = 4, CONV_C = 32, CONV_THREADS = 256;
 constexpr int CONV_MIN_CTAS = 4;  // 64 registers: four CTAs per SM
 constexpr int CONV_BX = CONV_X + 2, CONV_BY = CONV_Y + 2;
@@ -765,23 +766,28 @@ __global__ void __launch_bounds__(CONV_THREADS, CONV_MIN_CTAS)
   float4 acc[CONV_Y];
 #pragma unroll
   for (int r = 0; r < CONV_Y; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-  int tap = 0;
 #pragma unroll
   for (int a = 0; a < 3; ++a)
 #pragma unroll
-    for (int b = 0; b < 3; ++b)
+    for (int e = 0; e < 3; ++e) {
+      float4 wv[3];
 #pragma unroll
-      for (int e = 0; e < 3; ++e, ++tap) {
-        const float4 wv = __ldg(reinterpret_cast<const float4*>(wb + (size_t)tap * d));
+      for (int b = 0; b < 3; ++b) wv[b] = __ldg(reinterpret_cast<const float4*>(wb + (size_t)((a * 3 + b) * 3 + e) * d));
 #pragma unroll
-        for (int r = 0; r < CONV_Y; ++r) {
-          const uint2 uv = box[((a * CONV_BY + r + b) * CONV_BX + xl + e) * (CONV_C / 4) + q];
-          acc[r].x = fmaf(wv.x, bf16lo(uv.x), acc[r].x);
-          acc[r].y = fmaf(wv.y, bf16hi(uv.x), acc[r].y);
-          acc[r].z = fmaf(wv.z, bf16lo(uv.y), acc[r].z);
-          acc[r].w = fmaf(wv.w, bf16hi(uv.y), acc[r].w);
+      for (int j = 0; j < CONV_BY; ++j) {
+        const uint2 uv = box[((a * CONV_BY + j) * CONV_BX + xl + e) * (CONV_C / 4) + q];
+        const float u0 = bf16lo(uv.x), u1 = bf16hi(uv.x), u2 = bf16lo(uv.y), u3 = bf16hi(uv.y);
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+          const int r = j - b;
+          if (r < 0 || r >= CONV_Y) continue;
+          acc[r].x = fmaf(wv[b].x, u0, acc[r].x);
+          acc[r].y = fmaf(wv[b].y, u1, acc[r].y);
+          acc[r].z = fmaf(wv[b].z, u2, acc[r].z);
+          acc[r].w = fmaf(wv[b].w, u3, acc[r].w);
         }
       }
+    }
   if (x >= W) return;
   const float gh = gvec[(bh + p.bh_offset) % p.heads];
   const uint32_t v2 = p.vpr * 2;  // 8-byte (4-channel) vectors per row
