@@ -13,8 +13,8 @@
 //   (odd key blocks); each group owns one S accumulator and one O
 //   accumulator in TMEM (S0 cols 0-127, S1 128-255, O0 256+, O1 384+), and
 //   the two partial results are merged in the epilogue;
-//   warp 8 loads Q and K, warp 9 loads V (TMA, 128-byte swizzle, no
-//   multicast); warp 10 issues the MMAs and owns the TMEM allocation.
+//   warp 8 loads Q and K, warp 9 loads V (TMA, 128-byte swizzle, each CTA
+//   its own tiles); warp 10 issues the MMAs and owns the TMEM allocation.
 // P is written back over its own S columns as bf16 and read by the P*V MMA
 // straight from TMEM.  The running max is only moved (and O rescaled) when a
 // row's max grows by more than 2^8; otherwise P may reach 2^8, which bf16 and

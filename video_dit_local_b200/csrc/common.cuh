@@ -1,5 +1,5 @@
 // Device primitives for the sm_100a kernels: mbarriers with bounded waits,
-// TMA tile loads (no multicast anywhere), tcgen05 MMA / TMEM helpers, UMMA
+// TMA tile loads (each CTA loads its own tiles), tcgen05 MMA / TMEM helpers, UMMA
 // descriptors, and the tile-window geometry shared by every kernel.
 #pragma once
 
@@ -121,7 +121,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled, 3D, no multicast)
+// TMA (tiled, 3D and 5D; every load fills only the issuing CTA's shared memory)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
