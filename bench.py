@@ -41,8 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ncu DRAM traffic per launch of the sliding-tile forward kernel at the 720p
 # workload (read+write bytes), and the hash of the kernel source it was taken
 # from.  When the source changes the figure is stale and reported as null.
-STA_FWD_TRAFFIC = 2710056960  # DRAM read + write bytes per launch: an ncu capture of the 2-head case x 12
-STA_FWD_TRAFFIC_SRC_SHA = "b18d2c6f5590f3df"
+STA_FWD_TRAFFIC = 2721076224  # DRAM read + write bytes per launch: an ncu capture of the 2-head case x 12
+STA_FWD_TRAFFIC_SRC_SHA = "657b6e246093eed6"
 
 
 def reduce_max(values, world: int, device=None):
