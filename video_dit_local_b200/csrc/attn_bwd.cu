@@ -62,7 +62,7 @@ struct PreArgs {
   int vpr, N, heads;
 };
 
-__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const PreArgs a) {
+__global__ void __launch_bounds__(256, 8) bwd_preprocess_kernel(const PreArgs a) {
   const int bh = blockIdx.y;
   const int h = bh % a.heads;
   const int groups = blockDim.x / a.vpr;
@@ -76,6 +76,14 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const PreArgs a) {
     const int r = rb + grp;
     const bool in = r < a.N;
     float sl = 0.f, sg = 0.f;
+    // the row's LSE values are fetched with its vectors, so the loop waits
+    // once per row on memory, not twice
+    float lse_l = 0.f, lse_g = 0.f;
+    if (in && lane_in == 0) {
+      const size_t i = (size_t)bh * a.N + r;
+      lse_l = __ldg(a.lse_l + i);
+      if (a.o_g) lse_g = __ldg(a.lse_g + i);
+    }
     if (in) {
       const size_t base = ((size_t)bh * a.N + r) * a.vpr + lane_in;
       const uint4 x = __ldg(a.dout + base);
@@ -97,10 +105,10 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const PreArgs a) {
     if (in && lane_in == 0) {
       const size_t i = (size_t)bh * a.N + r;
       a.ndelta_l[i] = -sl;
-      a.nlse2_l[i] = off_l - a.lse_l[i] * LOG2E;
+      a.nlse2_l[i] = off_l - lse_l * LOG2E;
       if (a.o_g) {
         a.ndelta_g[i] = -sg;
-        a.nlse2_g[i] = off_g - a.lse_g[i] * LOG2E;
+        a.nlse2_g[i] = off_g - lse_g * LOG2E;
       }
       dg_acc += sl - sg;
     }
