@@ -61,6 +61,9 @@ def _run(V, w, check, weights=None):
     ((6, 24, 40), (3, 8, 8), (3, 3, 3), (3, 8, 8), 128, 1, 2),    # pooled grid 2x3x5 (restoration at every edge)
     # 6 rows: the restoration's last 4-row band is half empty; 12 columns: one partial 32-column band
     ((4, 6, 12), (2, 2, 4), (1, 2, 3), (1, 3, 4), 64, 1, 2),
+    # pool widths 2 and 3: the compression's 2-wide load rows and its one-at-a-time loop
+    ((2, 8, 12), (1, 4, 4), (1, 2, 3), (1, 2, 2), 64, 1, 1),
+    ((2, 8, 12), (1, 4, 4), (1, 2, 3), (1, 2, 3), 64, 1, 1),
 ])
 def test_dual_sym_learned_small_full(V, grid, tile, window, pool, d, batch, heads):
     w = S.small_workload("symlearn", 37, batch, heads, d, grid, tile, window, pool)
