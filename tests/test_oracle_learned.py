@@ -1,6 +1,6 @@
 """Pins of the oracle's learned compressed global branch (CPU): the depthwise
-strided compression against explicit per-tap loops and, with uniform taps,
-against average pooling; the 3x3x3 restoring convolution against torch's
+strided compression against explicit per-tap loops, against torch's strided
+grouped conv3d and, with uniform taps, against average pooling; the 3x3x3 restoring convolution against torch's
 grouped conv3d (cross-correlation, zero padding), the identity tap and a
 one-voxel shift; and the whole learned dual forward, with uniform
 compression and the identity restoration, against the average-pooling form."""
@@ -55,6 +55,23 @@ def test_conv_compress_uniform_taps_is_average_pooling(g):
     x = _rand((1, 3, g.n, 4), 3)
     w = np.full((3, P, 4), 1.0 / P)
     np.testing.assert_allclose(O.conv_compress(x, g, w), O.pool(x, g), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("g", GEOMS)
+def test_conv_compress_matches_torch_strided_grouped_conv3d(g):
+    """Depthwise convolution with stride equal to its kernel ("UltraGen ..."
+    §4.2): torch's grouped conv3d with kernel = stride = the pool size."""
+    B, nh, d = 2, 2, 3
+    P = g.pool[0] * g.pool[1] * g.pool[2]
+    x = _rand((B, nh, g.n, d), 6)
+    w = _rand((nh, P, d), 7)
+    got = O.conv_compress(x, g, w)
+    for h in range(nh):
+        xt = torch.from_numpy(x[:, h].reshape(B, g.T, g.H, g.W, d)).permute(0, 4, 1, 2, 3).contiguous()
+        wt = torch.from_numpy(np.ascontiguousarray(w[h].T.reshape(d, 1, *g.pool)))   # taps (dt, dy, dx)
+        ref = torch.nn.functional.conv3d(xt, wt, stride=tuple(g.pool), groups=d)
+        ref = ref.permute(0, 2, 3, 4, 1).reshape(B, g.n_pooled, d).numpy()
+        np.testing.assert_allclose(got[:, h], ref, rtol=1e-12, atol=1e-12)
 
 
 @pytest.mark.parametrize("g", GEOMS)
